@@ -1,0 +1,223 @@
+"""CPU oracle of the 4-bit FlashAttention forward (HiFA4 reading), via ctypes.
+
+TEST INFRASTRUCTURE ONLY: the tests, ``__graft_entry__.smoke()`` and the
+benchmark's CPU-baseline leg may use this package; the product package never
+imports it. The arithmetic lives in ``hifa4_oracle.c`` (plain C, built with
+``build()``); this file only marshals numpy arrays.
+
+Parity status of each function (what pins it, see tests/test_oracle_pins.py):
+  e2m1/e4m3 encode+decode  pinned: closed-form code tables, midpoint ties,
+                           sweeps against ml_dtypes and torch float8 casts
+  quantize_rows/_v         pinned: worked blocks in tests/golden, error bound,
+                           independent NumPy restatement (np_ref)
+  calibrate                pinned: hand-built 2-channel example, zero channel
+  qk_row                   pinned: exact rational dot products (fractions)
+  attention_rows           pinned: brute-force fp64 softmax attention with
+                           quantization off (causal, GQA, ragged Nq), V = 1
+                           invariants for both normalizer modes, convex-hull
+                           bound, NumPy restatement on the tiny config
+  The whole quantized output has no published values to compare with; beyond
+  the pieces above its parity is pinned only through those pieces.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "hifa4_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lib = None
+
+P_REORDER = 0
+HIGH_PRECISION_L = 1
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle (gcc, OpenMP, no fast-math, no FMA contraction)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        cmd = ["gcc", "-O2", "-std=c11", "-fopenmp", "-ffp-contract=off", "-fno-fast-math",
+               "-shared", "-fPIC", "-o", _LIB, _SRC, "-lm"]
+        subprocess.check_call(cmd)
+    return _LIB
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        build()
+        L = ctypes.CDLL(_LIB)
+        u8p = np.ctypeslib.ndpointer(np.uint8, flags="C_CONTIGUOUS")
+        f32p = np.ctypeslib.ndpointer(np.float32, flags="C_CONTIGUOUS")
+        i64p = np.ctypeslib.ndpointer(np.int64, flags="C_CONTIGUOUS")
+        vp = ctypes.c_void_p
+        ci, cf, cll = ctypes.c_int, ctypes.c_float, ctypes.c_longlong
+        L.ora_e2m1_decode.argtypes = [ctypes.c_uint8]
+        L.ora_e2m1_decode.restype = ctypes.c_double
+        L.ora_e2m1_encode.argtypes = [cf]
+        L.ora_e2m1_encode.restype = ctypes.c_uint8
+        L.ora_e4m3_decode.argtypes = [ctypes.c_uint8]
+        L.ora_e4m3_decode.restype = ctypes.c_double
+        L.ora_e4m3_encode.argtypes = [cf]
+        L.ora_e4m3_encode.restype = ctypes.c_uint8
+        L.ora_scale_code.argtypes = [cf]
+        L.ora_scale_code.restype = ctypes.c_uint8
+        L.ora_quant_block16.argtypes = [f32p, u8p, u8p]
+        L.ora_quant_block16.restype = None
+        L.ora_calibrate.argtypes = [f32p, f32p, ci, ci, ci, ci, ci, cf, f32p, f32p]
+        L.ora_calibrate.restype = None
+        L.ora_quantize_rows.argtypes = [f32p, ci, ci, ci, ci, ci, vp, u8p, u8p]
+        L.ora_quantize_rows.restype = None
+        L.ora_quantize_v.argtypes = [f32p, ci, ci, ci, ci, u8p, u8p]
+        L.ora_quantize_v.restype = None
+        L.ora_qk_row.argtypes = [u8p, u8p, u8p, u8p, ci, ci, ci, ci, ci, cll, f32p]
+        L.ora_qk_row.restype = None
+        L.ora_attention_rows.argtypes = [vp] * 9 + [ci] * 6 + [cf, ci, ci, ci, i64p, cll] + [vp] * 7 + [ci]
+        L.ora_attention_rows.restype = ci
+        _lib = L
+    return _lib
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+# ------------------------------------------------------------------ formats
+
+def e2m1_encode(x) -> np.ndarray:
+    L = lib()
+    x = np.asarray(x, np.float32).ravel()
+    return np.array([L.ora_e2m1_encode(float(v)) for v in x], np.uint8)
+
+
+def e2m1_decode(codes) -> np.ndarray:
+    L = lib()
+    return np.array([L.ora_e2m1_decode(int(c)) for c in np.asarray(codes).ravel()], np.float64)
+
+
+def e4m3_encode(x) -> np.ndarray:
+    L = lib()
+    x = np.asarray(x, np.float32).ravel()
+    return np.array([L.ora_e4m3_encode(float(v)) for v in x], np.uint8)
+
+
+def e4m3_decode(codes) -> np.ndarray:
+    L = lib()
+    return np.array([L.ora_e4m3_decode(int(c)) for c in np.asarray(codes).ravel()], np.float64)
+
+
+def quant_block16(x):
+    x = np.ascontiguousarray(x, np.float32)
+    assert x.shape == (16,)
+    codes = np.zeros(16, np.uint8)
+    sf = np.zeros(1, np.uint8)
+    lib().ora_quant_block16(x, codes, sf)
+    return codes, int(sf[0])
+
+
+# ----------------------------------------------------------- path steps
+
+def calibrate(q: np.ndarray, k: np.ndarray, alpha: float = 0.5):
+    """Smooth-QK factors s, s_inv [Hkv, D] from q [B,Hq,N,D], k [B,Hkv,N,D] (float32)."""
+    q = np.ascontiguousarray(q, np.float32)
+    k = np.ascontiguousarray(k, np.float32)
+    B, Hq, N, D = q.shape
+    Hkv = k.shape[1]
+    s = np.zeros((Hkv, D), np.float32)
+    si = np.zeros((Hkv, D), np.float32)
+    lib().ora_calibrate(q, k, B, Hq, Hkv, N, D, float(alpha), s, si)
+    return s, si
+
+
+def quantize_rows(x: np.ndarray, scale: np.ndarray | None = None, group: int = 1):
+    """Q or K [B,H,N,D] -> (codes [B,H,N,D/2], scales [B,H,N,D/16]); scale = s (Q) or s_inv (K)."""
+    x = np.ascontiguousarray(x, np.float32)
+    B, H, N, D = x.shape
+    codes = np.zeros((B, H, N, D // 2), np.uint8)
+    sf = np.zeros((B, H, N, D // 16), np.uint8)
+    sc = None if scale is None else np.ascontiguousarray(scale, np.float32)
+    lib().ora_quantize_rows(x, B, H, N, D, group, _ptr(sc), codes, sf)
+    return codes, sf
+
+
+def quantize_v(v: np.ndarray):
+    """V [B,Hkv,N,D] -> (vtc [B,Hkv,D,N/2], vts [B,Hkv,D,N/16]), quantized along tokens."""
+    v = np.ascontiguousarray(v, np.float32)
+    B, H, N, D = v.shape
+    vtc = np.zeros((B, H, D, N // 2), np.uint8)
+    vts = np.zeros((B, H, D, N // 16), np.uint8)
+    lib().ora_quantize_v(v, B, H, N, D, vtc, vts)
+    return vtc, vts
+
+
+def quantize_qkv(q, k, v, s=None, s_inv=None):
+    Hq, Hkv = q.shape[1], k.shape[1]
+    qc, qs = quantize_rows(q, s, Hq // Hkv)
+    kc, ks = quantize_rows(k, s_inv, 1)
+    vtc, vts = quantize_v(v)
+    return dict(qc=qc, qs=qs, kc=kc, ks=ks, vtc=vtc, vts=vts)
+
+
+def qk_row(packed, Hq, Hkv, Nq, Nkv, D, row):
+    S = np.zeros(Nkv, np.float32)
+    p = {k: np.ascontiguousarray(a) for k, a in packed.items()}
+    lib().ora_qk_row(p["qc"], p["qs"], p["kc"], p["ks"], Hq, Hkv, Nq, Nkv, D, int(row), S)
+    return S
+
+
+def default_sm_scale(D: int) -> float:
+    return float(np.float32(1.0 / np.sqrt(float(D))))
+
+
+def attention_rows(shape, rows, *, packed=None, fp32=None, sm_scale=None, causal=False,
+                   norm_mode=P_REORDER, want_eps=False, want_p=False, n_threads=0):
+    """Run the oracle on selected query rows.
+
+    shape: (B, Hq, Hkv, Nq, Nkv, D). rows: flat ids (b*Hq + h)*Nq + i.
+    packed: dict of canonical quantized operands (4-bit path), or
+    fp32: (q, k, v) float32 operands (quantization off).
+    Returns dict with O [n,D] f64, lse [n], l_hat [n], l_hp [n] and optionally
+    eps [n, Nkv/128], p_codes [n, Nkv/2], p_sf [n, Nkv/16].
+    """
+    B, Hq, Hkv, Nq, Nkv, D = shape
+    rows = np.ascontiguousarray(np.asarray(rows, np.int64))
+    n = rows.size
+    if sm_scale is None:
+        sm_scale = default_sm_scale(D)
+    O = np.zeros((n, D), np.float64)
+    lse = np.zeros(n, np.float64)
+    lh = np.zeros(n, np.float64)
+    lp = np.zeros(n, np.float64)
+    eps = np.zeros((n, Nkv // 128), np.float64) if want_eps else None
+    pc = np.zeros((n, Nkv // 2), np.uint8) if want_p else None
+    ps = np.zeros((n, Nkv // 16), np.uint8) if want_p else None
+    if packed is not None:
+        p = {k: np.ascontiguousarray(a) for k, a in packed.items()}
+        args = [_ptr(p["qc"]), _ptr(p["qs"]), _ptr(p["kc"]), _ptr(p["ks"]), _ptr(p["vtc"]), _ptr(p["vts"]),
+                None, None, None]
+        quant = 1
+        keep = p
+    else:
+        qf, kf, vf = (np.ascontiguousarray(a, np.float32) for a in fp32)
+        args = [None] * 6 + [_ptr(qf), _ptr(kf), _ptr(vf)]
+        quant = 0
+        keep = (qf, kf, vf)
+    rc = lib().ora_attention_rows(*args, B, Hq, Hkv, Nq, Nkv, D, float(sm_scale), int(bool(causal)),
+                                  int(norm_mode), quant, rows, n, _ptr(O), _ptr(lse), _ptr(lh), _ptr(lp),
+                                  _ptr(eps), _ptr(pc), _ptr(ps), int(n_threads))
+    del keep
+    if rc != 0:
+        raise ValueError("oracle rejected the arguments")
+    out = dict(O=O, lse=lse, l_hat=lh, l_hp=lp)
+    if want_eps:
+        out["eps"] = eps
+    if want_p:
+        out["p_codes"], out["p_sf"] = pc, ps
+    return out
+
+
+def all_rows(B, Hq, Nq):
+    return np.arange(B * Hq * Nq, dtype=np.int64)
