@@ -1,0 +1,401 @@
+"""Benchmark of the 4-bit attention forward hot path on B200.
+
+One step = one pass of the hot path over the Qwen3-8B-shaped causal prefill
+(B=1, 32 q heads / 8 kv heads, D=128, N=4096, bf16 inputs, Smooth-QK from a
+512-token calibration batch, P-Reordering): smooth + quantize Q, K, V
+(hifa4_quantize_qkv) and the fused 4-bit attention (hifa4_attention_fwd).
+Calibration is offline (once per layer) and runs before the timed region.
+
+value    attention FLOPs (4*B*Hq*Nq*Nkv*D/2 for causal) per second over the
+         whole step, inputs resident in HBM, L2 flushed between steps
+e2e      the same metric through the public API with host buffers: pinned
+         host->device copy of Q, K, V, the step, device->host copy of O, LSE
+roofline the attention kernel alone against the FP4 dense tensor peak
+cpu_baseline  the CPU oracle on a bounded sample of the same workload
+
+``--impl reference`` times the CPU oracle (the slow, plainly written CPU
+implementation of the same computation) on the host cores instead.
+Multi-GPU (torchrun): every rank runs its own replica of the workload (the
+path has no exchange step); value sums the ranks' work over the max time.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as W  # noqa: E402
+
+METRIC = "4-bit attn fwd TFLOPS & % of B200 FP4 tensor peak, Qwen3-8B shape N=4096"
+L2_FLUSH_BYTES = 256 << 20
+
+
+def peaks():
+    """Measured HBM and bf16 peaks of this machine (driver-written); FP4 = 4 x bf16 (nominal 9 / 2.25)."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            m = json.load(f)
+        return dict(hbm=float(m["hbm_gbs"]), bf16=float(m["bf16_tflops"]),
+                    bf16_sus=float(m["bf16_tflops_sustained"]), src="measured")
+    except Exception:
+        return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, src="fallback")
+
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+class Clocks:
+    """nvidia-smi sampler running during the timed region."""
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_gpu{index}.csv")
+
+    def __enter__(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index),
+                 "--query-gpu=index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+                 "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                 "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap",
+                 "--format=csv,noheader,nounits", "-lms", "100"], stdout=self.f, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        try:
+            rows = [r.split(",") for r in open(self.path).read().strip().splitlines()]
+            rows = [[c.strip() for c in r] for r in rows if len(r) >= 9]
+        except Exception:
+            return None
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ------------------------------------------------------------------ inputs
+
+def make_inputs(cfg, device, rank=0):
+    """Seeded inputs on the device, built slice by slice (rank > 0: other data seeds)."""
+    import torch
+    TORCH_DT = {"bf16": torch.bfloat16, "fp16": torch.float16}
+    if rank:
+        cfg = cfg.replace(index=cfg.index + 100 * rank)
+    gains = W.k_gains(cfg)
+    dt = TORCH_DT[cfg.dtype]
+
+    def up(x):
+        return torch.from_numpy(W.to_bits(x, cfg.dtype).view(np.int16).copy()).to(device).view(dt)
+
+    q = torch.empty(cfg.B, cfg.Hq, cfg.Nq, cfg.D, dtype=dt, device=device)
+    k = torch.empty(cfg.B, cfg.Hkv, cfg.Nkv, cfg.D, dtype=dt, device=device)
+    v = torch.empty_like(k)
+    for b in range(cfg.B):
+        for h in range(cfg.Hq):
+            q[b, h] = up(W.q_slice(cfg, b, h))
+        for g in range(cfg.Hkv):
+            k[b, g] = up(W.k_slice(cfg, b, g, gains))
+            v[b, g] = up(W.v_slice(cfg, b, g))
+    cal = None
+    if cfg.smooth == "calib":
+        cq = torch.stack([up(W.qcal_slice(cfg, h)) for h in range(cfg.Hq)])[None]
+        ck = torch.stack([up(W.kcal_slice(cfg, g, gains)) for g in range(cfg.Hkv)])[None]
+        cal = (cq.contiguous(), ck.contiguous())
+    elif cfg.smooth == "self":
+        cal = (q, k)
+    return q, k, v, cal
+
+
+# -------------------------------------------------------------- CPU oracle
+
+def oracle_sample(cfg, seconds_target=12.0, n_threads=0, rows_per_head=None):
+    """Time the CPU oracle on a bounded sample of the workload: one kv group's
+    quantization plus the attention of a strided subset of its query rows.
+    Returns (flops_of_sample / seconds, description, threads)."""
+    import oracle
+    gains = W.k_gains(cfg)
+    b, g = 0, 0
+    G = cfg.G
+    q = np.stack([W.q_slice(cfg, b, g * G + hh) for hh in range(G)])[None]
+    k = W.k_slice(cfg, b, g, gains)[None, None]
+    v = W.v_slice(cfg, b, g)[None, None]
+    s = si = None
+    if cfg.smooth == "calib":
+        qc = np.stack([W.qcal_slice(cfg, g * G + hh) for hh in range(G)])[None]
+        kc = W.kcal_slice(cfg, g, gains)[None, None]
+        s, si = oracle.calibrate(qc, kc, cfg.alpha)
+    elif cfg.smooth == "self":
+        s, si = oracle.calibrate(q, k, cfg.alpha)
+    shape = (1, G, 1, cfg.Nq, cfg.Nkv, cfg.D)
+    # rows spread over the causal range (stride keeps the average key count of the full set)
+    n_rows = rows_per_head or max(8, min(cfg.Nq, 64))
+    idx = np.linspace(0, cfg.Nq - 1, n_rows).astype(np.int64)
+    rows = np.concatenate([hh * cfg.Nq + idx for hh in range(G)])
+    t0 = time.perf_counter()
+    pk = oracle.quantize_qkv(q, k, v, s, si)
+    oracle.attention_rows(shape, rows, packed=pk, causal=cfg.causal, n_threads=n_threads)
+    dt = time.perf_counter() - t0
+    if cfg.causal:
+        keys = np.minimum(idx + cfg.Nkv - cfg.Nq + 1, cfg.Nkv)
+    else:
+        keys = np.full(idx.shape, cfg.Nkv)
+    flops = 4.0 * cfg.D * float(keys.sum()) * G
+    # grow the sample to the target CPU time
+    if dt < seconds_target / 4 and n_rows < cfg.Nq:
+        scale = min(cfg.Nq / n_rows, max(2.0, seconds_target / max(dt, 1e-3)))
+        return oracle_sample(cfg, seconds_target, n_threads, int(min(cfg.Nq, n_rows * scale)))
+    desc = (f"quantize one (b, kv head) group (Q {G}x{cfg.Nq}x{cfg.D}, K/V {cfg.Nkv}x{cfg.D}) + attention of "
+            f"{rows.size} query rows ({n_rows} per head, evenly spaced) of that group")
+    return flops / dt, desc, dt
+
+
+# ----------------------------------------------------------------- our arm
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    import bit_quantized_flashattention_b200 as H
+    ws, rank, local = dist_env()
+    if ws > 1:
+        dist.init_process_group("nccl", init_method="env://", timeout=__import__("datetime").timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    cfg = W.get(args.config)
+    norm = args.norm
+    q, k, v, cal = make_inputs(cfg, dev, rank)
+    s = s_inv = None
+    if cal is not None:
+        s, s_inv = H.calibrate_smooth(cal[0], cal[1], cfg.alpha)
+    packed = H.alloc_packed(cfg.B, cfg.Hq, cfg.Hkv, cfg.Nq, cfg.Nkv, cfg.D, dev)
+    o = torch.empty(cfg.B, cfg.Hq, cfg.Nq, cfg.D, dtype=torch.bfloat16, device=dev)
+    lse = torch.empty(cfg.B, cfg.Hq, cfg.Nq, dtype=torch.float32, device=dev)
+    wsp = H.alloc_workspace(cfg.B, cfg.Hq, cfg.Hkv, cfg.Nq, cfg.Nkv, cfg.D, dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        H.quantize_qkv(q, k, v, s, s_inv, out=packed)
+        H.attention_fwd(packed, causal=cfg.causal, norm=norm, out=o, lse=lse, workspace=wsp)
+
+    launches_per_step = 4          # Q rows, K rows, V (transposed), attention
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    st = H.get_status(wsp)
+    if st != 0:
+        raise RuntimeError(f"kernel status {st} during warm-up")
+
+    n = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+    if ws > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with Clocks(local) as clk:
+        for i in range(n):
+            flush.random_(0, 255) if i == 0 else flush.fill_(i & 0xFF)
+            ev[i][0].record(stream)
+            H.quantize_qkv(q, k, v, s, s_inv, out=packed)
+            ev[i][1].record(stream)
+            H.attention_fwd(packed, causal=cfg.causal, norm=norm, out=o, lse=lse, workspace=wsp)
+            ev[i][2].record(stream)
+        torch.cuda.synchronize()
+    if ws > 1:
+        dist.barrier()
+    step_ms = [a.elapsed_time(c) for a, _, c in ev]
+    attn_ms = [b.elapsed_time(c) for _, b, c in ev]
+    quant_ms = [a.elapsed_time(b) for a, b, _ in ev]
+    total_ms = float(sum(step_ms))
+    if ws > 1:
+        t = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    st = H.get_status(wsp)
+    if st != 0:
+        raise RuntimeError(f"kernel status {st} in the timed region")
+
+    flops = cfg.flops()
+    value = ws * flops * n / (total_ms * 1e-3) / 1e12
+    attn_mean = statistics.mean(attn_ms)
+    attn_tflops = flops / (attn_mean * 1e-3) / 1e12
+    pk = peaks()
+    fp4_peak = 4.0 * pk["bf16"]                       # burst: the kernel is timed alone, per launch
+
+    # end to end through the public API: pinned host buffers in, host results out
+    hq = q.cpu().pin_memory()
+    hk = k.cpu().pin_memory()
+    hv = v.cpu().pin_memory()
+    ho = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+    hl = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+    e2e_ms = []
+    for i in range(max(args.warmup, 3) + n):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        flush.fill_(i & 0xFF)
+        e0.record(stream)
+        q.copy_(hq, non_blocking=True)
+        k.copy_(hk, non_blocking=True)
+        v.copy_(hv, non_blocking=True)
+        step()
+        ho.copy_(o, non_blocking=True)
+        hl.copy_(lse, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        if i >= max(args.warmup, 3):
+            e2e_ms.append(e0.elapsed_time(e1))
+    e2e_total = float(sum(e2e_ms))
+    if ws > 1:
+        t = torch.tensor([e2e_total], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_total = float(t.item())
+    h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv))
+    d2h = ho.numel() * ho.element_size() + hl.numel() * hl.element_size()
+
+    line = {
+        "metric": METRIC,
+        "value": round(value, 3),
+        "unit": "TFLOPS",
+        "n_gpus": ws,
+        "steps": n,
+        "warmup": args.warmup,
+        "ms_per_step": round(total_ms / n, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "e2m1",
+        "data": "synthetic (seeded normal Q/K/V, lognormal K channel gains + outlier channels)",
+        "config": {"workload": cfg.name, "B": cfg.B, "Hq": cfg.Hq, "Hkv": cfg.Hkv, "Nq": cfg.Nq, "Nkv": cfg.Nkv,
+                   "D": cfg.D, "causal": cfg.causal, "norm": norm, "smooth_qk": cfg.smooth != "off",
+                   "inputs": cfg.dtype, "output": "bf16", "parallelism": f"replicas{ws}" if ws > 1 else "single",
+                   "l2": "flushed between steps (256 MiB write)",
+                   "step": "quantize_qkv + attention_fwd (calibration offline)"},
+        "fp4_tensor_pct": round(100.0 * value / ws / fp4_peak, 2),
+        "breakdown_ms": {"quantize": round(statistics.mean(quant_ms), 5), "attention": round(attn_mean, 5)},
+        "attention_only_tflops": round(attn_tflops, 2),
+        "roofline": {"bound": "tensor", "achieved": round(attn_tflops, 2), "peak": round(fp4_peak, 1),
+                     "unit": "TFLOP/s", "frac": round(attn_tflops / fp4_peak, 4), "traffic": None,
+                     "kernel": "attn_fwd_kernel", "peak_source": f"4 x {pk['src']} bf16 burst"},
+        "e2e": {"value": round(ws * flops * n / (e2e_total * 1e-3) / 1e12, 3), "unit": "TFLOPS",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches_per_step * n,
+        "clocks": clk.summary(),
+    }
+    # the HBM-bound quantize pass: algorithmic bytes (read 2 B/elem, write 0.5625 B/elem)
+    elems = cfg.B * cfg.Hq * cfg.Nq * cfg.D + 2 * cfg.B * cfg.Hkv * cfg.Nkv * cfg.D
+    qbytes = elems * (2 + 0.5625)
+    line["quantize_gbs"] = round(qbytes / (statistics.mean(quant_ms) * 1e-3) / 1e9, 1)
+    if args.sdpa and rank == 0:
+        line["sdpa_bf16_tflops"] = sdpa_context(q, k, v, cfg, flush)
+    if rank == 0 and not args.no_cpu:
+        v_cpu, desc, secs = oracle_sample(cfg)
+        line["cpu_baseline"] = {"value": round(v_cpu / 1e12, 8), "unit": "TFLOPS", "cores": os.cpu_count(),
+                                "kind": "oracle", "sample": desc, "seconds": round(secs, 2)}
+    if ws > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def sdpa_context(q, k, v, cfg, flush):
+    import torch
+    import torch.nn.functional as F
+    ts = []
+    for i in range(8):
+        flush.fill_(i)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        F.scaled_dot_product_attention(q, k, v, is_causal=cfg.causal, enable_gqa=True)
+        e1.record()
+        torch.cuda.synchronize()
+        if i >= 3:
+            ts.append(e0.elapsed_time(e1))
+    return round(cfg.flops() / (statistics.mean(ts) * 1e-3) / 1e12, 2)
+
+
+# ----------------------------------------------------------- reference arm
+
+def run_reference(args):
+    ws, rank, _ = dist_env()
+    if rank != 0:
+        return
+    cfg = W.get(args.config)
+    for _ in range(args.warmup):
+        oracle_sample(cfg, seconds_target=2.0)
+    vals, secs = [], []
+    desc = ""
+    t_all = time.perf_counter()
+    for _ in range(args.steps):
+        v_cpu, desc, s = oracle_sample(cfg, seconds_target=2.0)
+        vals.append(v_cpu)
+        secs.append(s)
+    total = time.perf_counter() - t_all
+    value = statistics.mean(vals) / 1e12
+    line = {
+        "metric": METRIC, "value": round(value, 8), "unit": "TFLOPS", "n_gpus": ws, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(1e3 * total / args.steps, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "e2m1", "data": "synthetic",
+        "config": {"workload": cfg.name, "B": cfg.B, "Hq": cfg.Hq, "Hkv": cfg.Hkv, "Nq": cfg.Nq, "Nkv": cfg.Nkv,
+                   "D": cfg.D, "causal": cfg.causal, "norm": args.norm, "smooth_qk": cfg.smooth != "off"},
+        "impl": "reference",
+        "cpu_baseline": {"value": round(value, 8), "unit": "TFLOPS", "cores": os.cpu_count(), "kind": "oracle",
+                         "sample": f"each step: {desc}"},
+        "e2e": {"value": round(value, 8), "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", type=int, default=2, help="workload index 1..5 (2 = the headline)")
+    ap.add_argument("--norm", choices=["p_reorder", "high_precision_l"], default="p_reorder")
+    ap.add_argument("--sdpa", action="store_true", help="also time torch bf16 SDPA as context")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle sample")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,262 @@
+// C ABI of the 4-bit attention library (declared in include/hifa4.h):
+// argument validation, TMA tensor maps and kernel launches. No allocation.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+
+#include "../../include/hifa4.h"
+#include "hifa4_kernels.h"
+
+using namespace hifa4;
+
+namespace {
+
+constexpr unsigned long long kDefaultWaitNs = 2000000000ull;   // 2 s
+std::atomic<long long> g_wait_limit_ns{0};
+std::atomic<int> g_stall_loads{0};
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool shape_ok(int B, int Hq, int Hkv, int Nq, int Nkv, int D) {
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || Nq <= 0 || Nkv <= 0) return false;
+    if (Hq % Hkv != 0) return false;
+    if (D != 64 && D != 128 && D != 256) return false;
+    if (Nkv % 128 != 0 || Nq % 16 != 0) return false;
+    return true;
+}
+
+struct Sizes {
+    size_t qc, qs, kc, ks, vtc, vts;
+    int Tq;
+};
+
+Sizes sizes_of(int B, int Hq, int Hkv, int Nq, int Nkv, int D) {
+    Sizes s{};
+    const int G = Hq / Hkv;
+    s.Tq = (G * Nq + 127) / 128;
+    const size_t KS = (size_t)D / 64;
+    const size_t NRB = ((size_t)D + 127) / 128;
+    s.qc = (size_t)B * Hq * Nq * (D / 2);
+    s.qs = (size_t)B * Hkv * s.Tq * KS * 512;
+    s.kc = (size_t)B * Hkv * Nkv * (D / 2);
+    s.ks = (size_t)B * Hkv * (Nkv / 128) * KS * 512;
+    s.vtc = (size_t)B * Hkv * D * (Nkv / 2);
+    s.vts = (size_t)B * Hkv * (Nkv / 128) * NRB * 2 * 512;
+    return s;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (fn == nullptr) {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    }
+    return fn;
+}
+
+// 2-D u8 tensor map: `rows` rows of `row_bytes` bytes, box of box_rows x row_bytes... (inner box = box_x bytes).
+bool make_map(CUtensorMap* m, const void* base, uint64_t inner_bytes, uint64_t rows, uint32_t box_x, uint32_t box_y,
+              CUtensorMapSwizzle swz) {
+    auto fn = encode_fn();
+    if (fn == nullptr) return false;
+    cuuint64_t dims[2] = {inner_bytes, rows};
+    cuuint64_t strides[1] = {inner_bytes};
+    cuuint32_t box[2] = {box_x, box_y};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+hifa4_status from_cuda(cudaError_t e) { return e == cudaSuccess ? HIFA4_OK : HIFA4_ERR_CUDA; }
+
+hifa4_status attention_impl(const hifa4_packed* in, int B, int Hq, int Hkv, int Nq, int Nkv, int D, float sm_scale,
+                            unsigned flags, hifa4_norm_mode norm, void* o, hifa4_dtype o_dtype, float* lse,
+                            uint8_t* p_codes, uint8_t* p_sf, bool dump, void* workspace, hifa4_stream_t stream) {
+    if (in == nullptr || o == nullptr || workspace == nullptr) return HIFA4_ERR_INVALID_ARG;
+    if (!shape_ok(B, Hq, Hkv, Nq, Nkv, D)) return HIFA4_ERR_UNSUPPORTED;
+    if (!(sm_scale > 0.0f) || !std::isfinite(sm_scale)) return HIFA4_ERR_INVALID_ARG;
+    if ((flags & ~(unsigned)HIFA4_CAUSAL) != 0) return HIFA4_ERR_INVALID_ARG;
+    const bool causal = (flags & HIFA4_CAUSAL) != 0;
+    if (causal && Nq > Nkv) return HIFA4_ERR_UNSUPPORTED;
+    if (norm != HIFA4_NORM_P_REORDER && norm != HIFA4_NORM_HIGH_PRECISION_L) return HIFA4_ERR_INVALID_ARG;
+    if (o_dtype != HIFA4_F16 && o_dtype != HIFA4_BF16 && o_dtype != HIFA4_F32) return HIFA4_ERR_INVALID_ARG;
+    const void* ptrs[6] = {in->qc, in->qs, in->kc, in->ks, in->vtc, in->vts};
+    for (const void* q : ptrs)
+        if (q == nullptr || !aligned16(q)) return HIFA4_ERR_INVALID_ARG;
+    if (!aligned16(o) || !aligned16(workspace) || (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u)))
+        return HIFA4_ERR_INVALID_ARG;
+    if (dump && (p_codes == nullptr || p_sf == nullptr || !aligned16(p_codes) || !aligned16(p_sf)))
+        return HIFA4_ERR_INVALID_ARG;
+    const long long rows_q = (long long)B * Hq * Nq, rows_k = (long long)B * Hkv * Nkv, rows_v = (long long)B * Hkv * D;
+    if (rows_q > INT32_MAX || rows_k > INT32_MAX || rows_v > INT32_MAX) return HIFA4_ERR_UNSUPPORTED;
+    const Sizes sz = sizes_of(B, Hq, Hkv, Nq, Nkv, D);
+    const long long n_work = (long long)B * Hkv * sz.Tq;
+    if (n_work > INT32_MAX) return HIFA4_ERR_UNSUPPORTED;
+
+    const CUtensorMapSwizzle swz_qk =
+        D == 64 ? CU_TENSOR_MAP_SWIZZLE_32B : (D == 128 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B);
+    CUtensorMap tq, tk, tv;
+    if (!make_map(&tq, in->qc, (uint64_t)D / 2, (uint64_t)rows_q, D / 2, 128, swz_qk)) return HIFA4_ERR_CUDA;
+    if (!make_map(&tk, in->kc, (uint64_t)D / 2, (uint64_t)rows_k, D / 2, 128, swz_qk)) return HIFA4_ERR_CUDA;
+    if (!make_map(&tv, in->vtc, (uint64_t)Nkv / 2, (uint64_t)rows_v, 64, (uint32_t)D, CU_TENSOR_MAP_SWIZZLE_64B))
+        return HIFA4_ERR_CUDA;
+
+    AttnParams p{};
+    p.qs = static_cast<const uint8_t*>(in->qs);
+    p.ks = static_cast<const uint8_t*>(in->ks);
+    p.vts = static_cast<const uint8_t*>(in->vts);
+    p.o = o;
+    p.lse = lse;
+    p.p_codes = p_codes;
+    p.p_sf = p_sf;
+    p.status = static_cast<uint32_t*>(workspace);
+    p.B = B;
+    p.Hq = Hq;
+    p.Hkv = Hkv;
+    p.Nq = Nq;
+    p.Nkv = Nkv;
+    p.G = Hq / Hkv;
+    p.Tq = sz.Tq;
+    p.n_kv_tiles = Nkv / 128;
+    p.n_work = (int)n_work;
+    p.heavy_first = (causal && Nq % 128 == 0) ? 1 : 0;
+    p.c = (float)((double)sm_scale * 1.4426950408889634074);
+    const long long lim = g_wait_limit_ns.load();
+    p.wait_limit_ns = lim > 0 ? (unsigned long long)lim : kDefaultWaitNs;
+    p.stall_loads = g_stall_loads.load();
+    const int out = o_dtype == HIFA4_F16 ? 0 : (o_dtype == HIFA4_BF16 ? 1 : 2);
+    return from_cuda(launch_attention(&tq, &tk, &tv, p, D, (int)norm, causal, out, dump,
+                                      reinterpret_cast<cudaStream_t>(stream)));
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t hifa4_packed_bytes(int B, int Hq, int Hkv, int Nq, int Nkv, int D, size_t out[6]) {
+    if (!shape_ok(B, Hq, Hkv, Nq, Nkv, D)) return 0;
+    const Sizes s = sizes_of(B, Hq, Hkv, Nq, Nkv, D);
+    if (out != nullptr) {
+        out[0] = s.qc;
+        out[1] = s.qs;
+        out[2] = s.kc;
+        out[3] = s.ks;
+        out[4] = s.vtc;
+        out[5] = s.vts;
+    }
+    return s.qc + s.qs + s.kc + s.ks + s.vtc + s.vts;
+}
+
+size_t hifa4_workspace_bytes(int B, int Hq, int Hkv, int Nq, int Nkv, int D) {
+    (void)B; (void)Hq; (void)Hkv; (void)Nq; (void)Nkv; (void)D;
+    return 256;
+}
+
+hifa4_status hifa4_calibrate_smooth(const void* q, const void* k, hifa4_dtype dtype, int B, int Hq, int Hkv, int N,
+                                    int D, float alpha, float* s, float* s_inv, hifa4_stream_t stream) {
+    if (q == nullptr || k == nullptr || s == nullptr || s_inv == nullptr) return HIFA4_ERR_INVALID_ARG;
+    if (dtype != HIFA4_F16 && dtype != HIFA4_BF16) return HIFA4_ERR_INVALID_ARG;
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || N <= 0 || Hq % Hkv != 0) return HIFA4_ERR_INVALID_ARG;
+    if (D != 64 && D != 128 && D != 256) return HIFA4_ERR_UNSUPPORTED;
+    if (!(alpha > 0.0f && alpha <= 1.0f)) return HIFA4_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(s) || !aligned16(s_inv)) return HIFA4_ERR_INVALID_ARG;
+    if ((long long)B * Hq > 65535) return HIFA4_ERR_UNSUPPORTED;
+    return from_cuda(launch_calibrate(dtype == HIFA4_BF16, q, k, B, Hq, Hkv, N, D, alpha, s, s_inv,
+                                      reinterpret_cast<cudaStream_t>(stream)));
+}
+
+hifa4_status hifa4_quantize_kv(const void* k, const void* v, hifa4_dtype dtype, int B, int Hkv, int Nkv, int D,
+                               const float* s_inv, const hifa4_packed* out, hifa4_stream_t stream) {
+    if (k == nullptr || v == nullptr || out == nullptr) return HIFA4_ERR_INVALID_ARG;
+    if (dtype != HIFA4_F16 && dtype != HIFA4_BF16) return HIFA4_ERR_INVALID_ARG;
+    if (!shape_ok(B, Hkv, Hkv, 16, Nkv, D)) return HIFA4_ERR_UNSUPPORTED;
+    const void* ptrs[6] = {k, v, out->kc, out->ks, out->vtc, out->vts};
+    for (const void* q : ptrs)
+        if (q == nullptr || !aligned16(q)) return HIFA4_ERR_INVALID_ARG;
+    if (s_inv != nullptr && !aligned16(s_inv)) return HIFA4_ERR_INVALID_ARG;
+    if ((long long)B * Hkv > 65535) return HIFA4_ERR_UNSUPPORTED;
+    const bool bf = dtype == HIFA4_BF16;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const long long n_grp = (long long)B * Hkv;
+    cudaError_t e = launch_quantize_rows(bf, k, s_inv, static_cast<uint8_t*>(out->kc), static_cast<uint8_t*>(out->ks),
+                                         n_grp, Nkv, Nkv / 128, 1, Hkv, Nkv, D, st);
+    if (e != cudaSuccess) return HIFA4_ERR_CUDA;
+    e = launch_quantize_v(bf, v, static_cast<uint8_t*>(out->vtc), static_cast<uint8_t*>(out->vts), n_grp, Nkv, D, st);
+    return from_cuda(e);
+}
+
+hifa4_status hifa4_quantize_qkv(const void* q, const void* k, const void* v, hifa4_dtype dtype, int B, int Hq, int Hkv,
+                                int Nq, int Nkv, int D, const float* s, const float* s_inv, const hifa4_packed* out,
+                                hifa4_stream_t stream) {
+    if (q == nullptr || out == nullptr) return HIFA4_ERR_INVALID_ARG;
+    if ((s == nullptr) != (s_inv == nullptr)) return HIFA4_ERR_INVALID_ARG;
+    if (dtype != HIFA4_F16 && dtype != HIFA4_BF16) return HIFA4_ERR_INVALID_ARG;
+    if (!shape_ok(B, Hq, Hkv, Nq, Nkv, D)) return HIFA4_ERR_UNSUPPORTED;
+    if (!aligned16(q) || out->qc == nullptr || out->qs == nullptr || !aligned16(out->qc) || !aligned16(out->qs) ||
+        (s != nullptr && !aligned16(s)))
+        return HIFA4_ERR_INVALID_ARG;
+    const Sizes sz = sizes_of(B, Hq, Hkv, Nq, Nkv, D);
+    const int G = Hq / Hkv;
+    const long long n_grp = (long long)B * Hkv;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = launch_quantize_rows(dtype == HIFA4_BF16, q, s, static_cast<uint8_t*>(out->qc),
+                                         static_cast<uint8_t*>(out->qs), n_grp, G * Nq, sz.Tq, G, Hkv, Nq, D, st);
+    if (e != cudaSuccess) return HIFA4_ERR_CUDA;
+    return hifa4_quantize_kv(k, v, dtype, B, Hkv, Nkv, D, s_inv, out, stream);
+}
+
+hifa4_status hifa4_attention_fwd(const hifa4_packed* in, int B, int Hq, int Hkv, int Nq, int Nkv, int D,
+                                 float sm_scale, unsigned flags, hifa4_norm_mode norm, void* o, hifa4_dtype o_dtype,
+                                 float* lse, void* workspace, hifa4_stream_t stream) {
+    return attention_impl(in, B, Hq, Hkv, Nq, Nkv, D, sm_scale, flags, norm, o, o_dtype, lse, nullptr, nullptr, false,
+                          workspace, stream);
+}
+
+hifa4_status hifa4_attention_fwd_debug(const hifa4_packed* in, int B, int Hq, int Hkv, int Nq, int Nkv, int D,
+                                       float sm_scale, unsigned flags, hifa4_norm_mode norm, void* o,
+                                       hifa4_dtype o_dtype, float* lse, uint8_t* p_codes, uint8_t* p_scales,
+                                       void* workspace, hifa4_stream_t stream) {
+    return attention_impl(in, B, Hq, Hkv, Nq, Nkv, D, sm_scale, flags, norm, o, o_dtype, lse, p_codes, p_scales, true,
+                          workspace, stream);
+}
+
+hifa4_status hifa4_get_status(void* workspace, hifa4_stream_t stream) {
+    if (workspace == nullptr) return HIFA4_ERR_INVALID_ARG;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(st) != cudaSuccess) return HIFA4_ERR_CUDA;
+    uint32_t word = 0;
+    if (cudaMemcpy(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess) return HIFA4_ERR_CUDA;
+    if (word != 0 && cudaMemset(workspace, 0, sizeof(word)) != cudaSuccess) return HIFA4_ERR_CUDA;
+    return word == 0 ? HIFA4_OK : (hifa4_status)word;
+}
+
+long long hifa4_debug_set_wait_limit(long long limit_ns, int stall_loads) {
+    g_stall_loads.store(stall_loads ? 1 : 0);
+    const long long prev = g_wait_limit_ns.exchange(limit_ns > 0 ? limit_ns : 0);
+    return prev > 0 ? prev : (long long)kDefaultWaitNs;
+}
+
+const char* hifa4_status_string(hifa4_status s) {
+    switch (s) {
+        case HIFA4_OK: return "ok";
+        case HIFA4_ERR_INVALID_ARG: return "invalid argument";
+        case HIFA4_ERR_UNSUPPORTED: return "unsupported shape or option";
+        case HIFA4_ERR_CUDA: return "CUDA error";
+        case HIFA4_ERR_TIMEOUT: return "bounded wait expired inside a kernel";
+        default: return "unknown status";
+    }
+}
+
+int hifa4_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,560 @@
+// Fused 4-bit attention forward for sm_100a (tcgen05 block-scaled FP4 MMA).
+//
+// HiFA4 abstract: QK^T and PV both run as 4-bit GEMMs inside FlashAttention,
+// the online-softmax state stays in a wider float format, and with
+// P-Reordering the softmax normalizer is accumulated from the same quantized
+// probabilities P_hat that feed the PV GEMM, fused into that GEMM.
+//
+// One CTA computes one 128-row query tile of one (batch, kv head) group. The
+// tile's rows are the group's query rows stacked head after head (GQA), so a
+// tile may mix heads when Nq is small. Warp roles:
+//   warp 0      TMA / bulk-copy producer: Q_hat tile once, then K_hat and V_hat^T
+//               tiles (128 keys) with their scale atoms through 3-stage rings
+//   warp 1      TMEM owner and MMA issuer (one thread): scale atoms shared->TMEM
+//               with tcgen05.cp, S = Q_hat K_hat^T into TMEM, then O += P_hat V_hat
+//   warps 4-11  two softmax warpgroups; warpgroup w owns keys 64w..64w+63 of
+//               every tile, thread t of a warpgroup owns row t. Per tile: load S
+//               from TMEM, causal mask, running max (exchanged between the two
+//               warpgroups), P = 2^(S*c - RN(m*c)), quantize P per 16 keys to
+//               E2M1 + E4M3 in registers, rescale O in TMEM when the max moved,
+//               write P_hat codes and scales to shared memory for the PV MMA.
+// With P-Reordering the V tile carries 16 extra rows: a row of E2M1 ones
+// (scale 1.0) and 15 zero rows, so the PV MMA also produces sum(P_hat) in
+// output column D: the normalizer from exactly the codes x scales the MMA used.
+// TMEM (512 columns): S [0,128), O [128,128+NO) with NO = D (+16), then the
+// scale-factor regions of Q, K, P and V.
+// Every mbarrier wait is bounded; when one gives up the CTA records
+// HIFA4_ERR_TIMEOUT in the workspace, drains its copies and MMAs, frees TMEM
+// and exits.
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include "hifa4_device.cuh"
+#include "hifa4_kernels.h"
+
+namespace hifa4 {
+
+constexpr int kThreads = 384;
+constexpr int kStages = 3;
+constexpr int kSoftmaxWarp0 = 4;
+
+template <int D, bool PREORDER>
+struct Cfg {
+    static constexpr int KS = D / 64;                     // 64-wide K steps of QK^T
+    static constexpr int QK_ROW = D / 2;                  // bytes per Q/K row
+    static constexpr uint32_t QK_SWZ = D == 64 ? 6u : (D == 128 ? 4u : 2u);   // 32B/64B/128B swizzle
+    static constexpr uint32_t QK_SBO = 8u * QK_ROW;       // bytes between 8-row groups
+    static constexpr int Q_BYTES = 128 * QK_ROW;
+    static constexpr int K_BYTES = 128 * QK_ROW;
+    static constexpr int SFQK_BYTES = KS * 512;
+    static constexpr int VROWS = D + 16;                  // V^T rows + normalizer block
+    static constexpr int V_BYTES = VROWS * 64;
+    static constexpr int V_TMA_BYTES = D * 64;
+    static constexpr int NRB = (D + 127) / 128;           // 128-row blocks of V^T scales
+    static constexpr int SFV_BYTES = NRB * 2 * 512;
+    static constexpr int P_BYTES = 128 * 64;
+    static constexpr int SFP_BYTES = 2 * 512;
+    static constexpr int NO = PREORDER ? D + 16 : D;      // accumulator columns
+    // TMEM columns
+    static constexpr uint32_t COL_S = 0;
+    static constexpr uint32_t COL_O = 128;
+    static constexpr uint32_t COL_SFQ = COL_O + NO;
+    static constexpr uint32_t COL_SFK = COL_SFQ + 4 * KS;
+    static constexpr uint32_t COL_SFP = COL_SFK + 4 * KS;
+    static constexpr uint32_t COL_SFV = COL_SFP + 8;
+    // scale columns per PV K step: one 4-column block per 128 rows of the B operand
+    static constexpr int SFV_PER_KS = 4 * (NRB + ((PREORDER && D >= 128) ? 1 : 0));
+    static constexpr uint32_t COL_END = COL_SFV + 2 * SFV_PER_KS;
+    static_assert(COL_END <= 512, "TMEM budget");
+    // shared memory offsets (1024-aligned operand tiles)
+    static constexpr int OFF_Q = 0;
+    static constexpr int OFF_K = OFF_Q + Q_BYTES;
+    static constexpr int OFF_V = OFF_K + kStages * K_BYTES;
+    static constexpr int OFF_P = OFF_V + kStages * ((V_BYTES + 1023) / 1024 * 1024);
+    static constexpr int V_STRIDE = (V_BYTES + 1023) / 1024 * 1024;
+    static constexpr int OFF_SFQ = OFF_P + 2 * P_BYTES;
+    static constexpr int OFF_SFK = OFF_SFQ + SFQK_BYTES;
+    static constexpr int OFF_SFV = OFF_SFK + kStages * SFQK_BYTES;
+    static constexpr int OFF_SFP = OFF_SFV + kStages * SFV_BYTES;
+    static constexpr int OFF_ONES = OFF_SFP + 2 * SFP_BYTES;
+    static constexpr int OFF_MX = OFF_ONES + 512;                     // float [2][2][128]
+    static constexpr int OFF_LUT = OFF_MX + 2 * 2 * 128 * 4;          // float [128]
+    static constexpr int OFF_BAR = OFF_LUT + 128 * 4;
+    static constexpr int N_BARS = 1 + 4 * kStages + 1 + 1 + 2 + 1 + 1 + 2 + 1;
+    static constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;
+    static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;          // + alignment slack
+};
+
+struct Bars {
+    uint64_t q_full;
+    uint64_t k_full[kStages];
+    uint64_t k_empty[kStages];
+    uint64_t v_full[kStages];
+    uint64_t v_empty[kStages];
+    uint64_t s_full;      // S of the current tile is in TMEM
+    uint64_t s_free;      // both warpgroups have read S
+    uint64_t p_full[2];   // P_hat buffer ready (and O rescaled)
+    uint64_t o_done;      // PV MMA of a tile finished
+    uint64_t drain;       // teardown of the MMA issuer
+    uint64_t mx[2];       // row-max exchange between the two warpgroups
+    uint64_t lx;          // normalizer exchange at the end
+};
+
+__device__ __forceinline__ uint32_t p_swizzle64(uint32_t row, uint32_t chunk) {
+    return row * 64u + ((chunk ^ ((row >> 1) & 3u)) << 4);
+}
+
+template <int OUT>
+__device__ __forceinline__ void store_out32(void* dst, const float (&v)[32]) {
+    if constexpr (OUT == 2) {
+        float4* d = reinterpret_cast<float4*>(dst);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) d[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+    } else {
+        uint32_t w[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            if constexpr (OUT == 1) {
+                __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+                w[i] = *reinterpret_cast<uint32_t*>(&h);
+            } else {
+                __half2 h = __floats2half2_rn(v[2 * i], v[2 * i + 1]);
+                w[i] = *reinterpret_cast<uint32_t*>(&h);
+            }
+        }
+        uint4* d = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) d[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+    }
+}
+
+template <int D, bool PREORDER, bool CAUSAL, int OUT, bool DUMP>
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                    const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
+    using C = Cfg<D, PREORDER>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    Bars* bars = reinterpret_cast<Bars*>(smem + C::OFF_BAR);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
+    float* mx_x = reinterpret_cast<float*>(smem + C::OFF_MX);
+    float* lut = reinterpret_cast<float*>(smem + C::OFF_LUT);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    // ---------------------------------------------------------------- work
+    const int w = blockIdx.x;
+    int grp, t;
+    {
+        const int n_grp = p.B * p.Hkv;
+        if (p.heavy_first) {
+            // causal, Nq % 128 == 0: largest query block first
+            const int th = p.Nq / 128;
+            const int per = n_grp * p.G;
+            const int iblk = th - 1 - w / per;
+            const int rem = w % per;
+            grp = rem / p.G;
+            t = (rem % p.G) * th + iblk;
+        } else {
+            grp = w / p.Tq;
+            t = w % p.Tq;
+        }
+    }
+    const int rows_in_grp = p.G * p.Nq;
+    const int p0 = t * 128;
+    int n_tiles = p.n_kv_tiles;
+    if (CAUSAL) {
+        const int p_max = min(p0 + 127, rows_in_grp - 1);
+        const int i_max = (p_max / p.Nq == p0 / p.Nq) ? (p_max % p.Nq) : (p.Nq - 1);
+        const int last = i_max + p.Nkv - p.Nq;
+        n_tiles = min(p.n_kv_tiles, last / 128 + 1);
+    }
+
+    // --------------------------------------------------------------- setup
+    if (threadIdx.x == 0) {
+        mbar_init(&bars->q_full, 1);
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&bars->k_full[s], 1);
+            mbar_init(&bars->k_empty[s], 1);
+            mbar_init(&bars->v_full[s], 1);
+            mbar_init(&bars->v_empty[s], 1);
+        }
+        mbar_init(&bars->s_full, 1);
+        mbar_init(&bars->s_free, 256);
+        mbar_init(&bars->p_full[0], 256);
+        mbar_init(&bars->p_full[1], 256);
+        mbar_init(&bars->o_done, 1);
+        mbar_init(&bars->drain, 1);
+        mbar_init(&bars->mx[0], 256);
+        mbar_init(&bars->mx[1], 256);
+        mbar_init(&bars->lx, 256);
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (threadIdx.x < 128) {
+        const uint32_t i = threadIdx.x;
+        lut[i] = (i == 0) ? 0.0f : __frcp_rn(e4m3_to_f32(i));
+    }
+    if (threadIdx.x >= 128 && threadIdx.x < 256) {
+        // normalizer block of V^T (rows D..D+15 of every stage): one row of E2M1
+        // ones (code 2 in both nibbles), 15 zero rows; and the scale atom of the
+        // ones row (row 0 of an atom = 1.0) for D >= 128.
+        const int i = threadIdx.x - 128;
+        for (int s = 0; s < kStages; ++s) {
+            uint32_t* row = reinterpret_cast<uint32_t*>(smem + C::OFF_V + s * C::V_STRIDE + D * 64);
+            for (int k = i; k < 16 * 16; k += 128) row[k] = (k < 16) ? 0x22222222u : 0u;
+        }
+        uint32_t* ones = reinterpret_cast<uint32_t*>(smem + C::OFF_ONES);
+        ones[i] = (i == 0) ? 0x38383838u : 0u;
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, 512);
+        tmem_relinquish();
+    }
+    if (warp == 0 && lane == 0) {
+        prefetch_tensormap(&tmQ);
+        prefetch_tensormap(&tmK);
+        prefetch_tensormap(&tmV);
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const WaitCtl ctl{abort_flag, p.status, p.wait_limit_ns};
+
+    if (warp == 0) {
+        // ---------------------------------------------------------- producer
+        if (lane == 0 && !p.stall_loads) {
+            int issued = 0;
+            bool ok = true;
+            mbar_arrive_expect_tx(&bars->q_full, C::Q_BYTES + C::SFQK_BYTES);
+            tma_load_2d(smem + C::OFF_Q, &tmQ, 0, grp * rows_in_grp + p0, &bars->q_full);
+            bulk_load(smem + C::OFF_SFQ, p.qs + ((size_t)grp * p.Tq + t) * C::SFQK_BYTES, C::SFQK_BYTES,
+                      &bars->q_full);
+            for (int j = 0; j < n_tiles && ok; ++j) {
+                const int st = j % kStages;
+                const uint32_t ph = ((j / kStages) + 1) & 1;
+                if (j >= kStages && !mbar_wait(&bars->k_empty[st], ph, ctl)) { ok = false; break; }
+                mbar_arrive_expect_tx(&bars->k_full[st], C::K_BYTES + C::SFQK_BYTES);
+                tma_load_2d(smem + C::OFF_K + st * C::K_BYTES, &tmK, 0, grp * p.Nkv + j * 128, &bars->k_full[st]);
+                bulk_load(smem + C::OFF_SFK + st * C::SFQK_BYTES,
+                          p.ks + ((size_t)grp * p.n_kv_tiles + j) * C::SFQK_BYTES, C::SFQK_BYTES, &bars->k_full[st]);
+                if (j >= kStages && !mbar_wait(&bars->v_empty[st], ph, ctl)) { ok = false; issued = 2 * j + 1; break; }
+                mbar_arrive_expect_tx(&bars->v_full[st], C::V_TMA_BYTES + C::SFV_BYTES);
+                tma_load_2d(smem + C::OFF_V + st * C::V_STRIDE, &tmV, j * 64, grp * D, &bars->v_full[st]);
+                bulk_load(smem + C::OFF_SFV + st * C::SFV_BYTES,
+                          p.vts + ((size_t)grp * p.n_kv_tiles + j) * C::SFV_BYTES, C::SFV_BYTES, &bars->v_full[st]);
+                issued = 2 * j + 2;
+            }
+            if (!ok) {
+                // drain the copies still in flight before the CTA exits
+                const int nk = (issued + 1) / 2, nv = issued / 2;
+                for (int j = max(0, nk - kStages); j < nk; ++j)
+                    mbar_wait_drain(&bars->k_full[j % kStages], (j / kStages) & 1, p.wait_limit_ns);
+                for (int j = max(0, nv - kStages); j < nv; ++j)
+                    mbar_wait_drain(&bars->v_full[j % kStages], (j / kStages) & 1, p.wait_limit_ns);
+                mbar_wait_drain(&bars->q_full, 0, p.wait_limit_ns);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            const uint32_t idesc_s = idesc_fp4_block16(128);
+            auto qk_desc = [&](uint32_t base, int s) {
+                return smem_desc(smem_u32(smem + base) + 32u * s, 16u, C::QK_SBO, C::QK_SWZ);
+            };
+            auto sf_desc = [&](uint32_t off) { return smem_desc(smem_u32(smem + off), 0u, 128u, 0u); };
+            bool ok = mbar_wait(&bars->q_full, 0, ctl);
+            if (ok) {
+                tc_fence_after();
+#pragma unroll
+                for (int s = 0; s < C::KS; ++s) tmem_cp_scale_atom(tmem + C::COL_SFQ + 4 * s, sf_desc(C::OFF_SFQ + 512 * s));
+                if constexpr (PREORDER && D >= 128) {
+#pragma unroll
+                    for (int s = 0; s < 2; ++s)
+                        tmem_cp_scale_atom(tmem + C::COL_SFV + s * C::SFV_PER_KS + 4 * C::NRB, sf_desc(C::OFF_ONES));
+                }
+            }
+            auto issue_pv = [&](int j) -> bool {
+                if (!mbar_wait(&bars->p_full[j & 1], (j >> 1) & 1, ctl)) return false;
+                const int st = j % kStages;
+                if (!mbar_wait(&bars->v_full[st], (j / kStages) & 1, ctl)) return false;
+                tc_fence_after();
+                const uint32_t pbuf = C::OFF_P + (j & 1) * C::P_BYTES;
+                const uint32_t sfp = C::OFF_SFP + (j & 1) * C::SFP_BYTES;
+                const uint32_t vbuf = C::OFF_V + st * C::V_STRIDE;
+                const uint32_t sfv = C::OFF_SFV + st * C::SFV_BYTES;
+#pragma unroll
+                for (int s = 0; s < 2; ++s) {
+                    tmem_cp_scale_atom(tmem + C::COL_SFP + 4 * s, sf_desc(sfp + 512 * s));
+#pragma unroll
+                    for (int rb = 0; rb < C::NRB; ++rb)
+                        tmem_cp_scale_atom(tmem + C::COL_SFV + s * C::SFV_PER_KS + 4 * rb, sf_desc(sfv + (rb * 2 + s) * 512));
+                }
+#pragma unroll
+                for (int s = 0; s < 2; ++s) {
+                    const uint64_t a = smem_desc(smem_u32(smem + pbuf) + 32u * s, 16u, 512u, 4u);
+                    const uint32_t acc = (j > 0 || s > 0) ? 1u : 0u;
+                    const uint32_t sfa = tmem + C::COL_SFP + 4 * s;
+                    const uint32_t sfb = tmem + C::COL_SFV + s * C::SFV_PER_KS;
+                    if constexpr (D == 256 && PREORDER) {
+                        const uint64_t b0 = smem_desc(smem_u32(smem + vbuf) + 32u * s, 16u, 512u, 4u);
+                        const uint64_t b1 = smem_desc(smem_u32(smem + vbuf + 128 * 64) + 32u * s, 16u, 512u, 4u);
+                        mma_fp4_block16(tmem + C::COL_O, a, b0, idesc_fp4_block16(128), sfa, sfb, acc);
+                        mma_fp4_block16(tmem + C::COL_O + 128, a, b1, idesc_fp4_block16(144), sfa, sfb + 4, acc);
+                    } else {
+                        const uint64_t b = smem_desc(smem_u32(smem + vbuf) + 32u * s, 16u, 512u, 4u);
+                        mma_fp4_block16(tmem + C::COL_O, a, b, idesc_fp4_block16(C::NO), sfa, sfb, acc);
+                    }
+                }
+                tc_commit(&bars->o_done);
+                tc_commit(&bars->v_empty[st]);
+                return true;
+            };
+            for (int j = 0; j < n_tiles && ok; ++j) {
+                const int st = j % kStages;
+                if (!mbar_wait(&bars->k_full[st], (j / kStages) & 1, ctl)) { ok = false; break; }
+                if (j > 0 && !mbar_wait(&bars->s_free, (j - 1) & 1, ctl)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t kbuf = C::OFF_K + st * C::K_BYTES;
+                const uint32_t sfk = C::OFF_SFK + st * C::SFQK_BYTES;
+#pragma unroll
+                for (int s = 0; s < C::KS; ++s) tmem_cp_scale_atom(tmem + C::COL_SFK + 4 * s, sf_desc(sfk + 512 * s));
+#pragma unroll
+                for (int s = 0; s < C::KS; ++s)
+                    mma_fp4_block16(tmem + C::COL_S, qk_desc(C::OFF_Q, s), qk_desc(kbuf, s), idesc_s,
+                                    tmem + C::COL_SFQ + 4 * s, tmem + C::COL_SFK + 4 * s, s > 0 ? 1u : 0u);
+                tc_commit(&bars->s_full);
+                tc_commit(&bars->k_empty[st]);
+                if (j > 0 && !issue_pv(j - 1)) { ok = false; break; }
+            }
+            if (ok && n_tiles > 0) issue_pv(n_tiles - 1);
+            // wait until every MMA / copy issued above has finished
+            tc_commit(&bars->drain);
+            mbar_wait_drain(&bars->drain, 0, p.wait_limit_ns);
+        }
+    } else if (warp >= kSoftmaxWarp0) {
+        // ------------------------------------------------------------ softmax
+        const int wg = (warp - kSoftmaxWarp0) >> 2;        // key half of every tile
+        const int wq = warp & 3;                           // TMEM lane quarter
+        const int row = wq * 32 + lane;
+        const uint32_t tl = tmem + ((uint32_t)(wq * 32) << 16);
+        const int prow = p0 + row;
+        const bool valid = prow < rows_in_grp;
+        const int qi = prow % p.Nq;
+        const int last = valid ? (CAUSAL ? qi + p.Nkv - p.Nq : p.Nkv - 1) : -1;
+        const size_t out_row = (size_t)grp * rows_in_grp + prow;
+        const float c = p.c;
+        const float one_sixth = rn_one_sixth();
+        float m_old = -INFINITY, mc_old = 0.0f, l_hp = 0.0f;
+        bool ok = true;
+        for (int j = 0; j < n_tiles; ++j) {
+            if (!__all_sync(0xFFFFFFFFu, mbar_wait(&bars->s_full, j & 1, ctl))) { ok = false; break; }
+            tc_fence_after();
+            float S[64];
+            {
+                uint32_t r0[32], r1[32];
+                tmem_ld32(tl + C::COL_S + wg * 64, r0);
+                tmem_ld32(tl + C::COL_S + wg * 64 + 32, r1);
+                tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    S[e] = __uint_as_float(r0[e]);
+                    S[32 + e] = __uint_as_float(r1[e]);
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(&bars->s_free);
+            const int n0 = j * 128 + wg * 64;
+            if (n0 + 63 > last) {
+#pragma unroll
+                for (int e = 0; e < 64; ++e)
+                    if (n0 + e > last) S[e] = -INFINITY;
+            }
+            float mx = S[0];
+#pragma unroll
+            for (int e = 1; e < 64; ++e) mx = fmaxf(mx, S[e]);
+            // exchange the partial row maxima of the two key halves
+            {
+                float* xb = mx_x + (j & 1) * 256;
+                xb[wg * 128 + row] = mx;
+                mbar_arrive(&bars->mx[j & 1]);
+                if (!__all_sync(0xFFFFFFFFu, mbar_wait(&bars->mx[j & 1], (j >> 1) & 1, ctl))) { ok = false; break; }
+                mx = fmaxf(xb[row], xb[128 + row]);
+            }
+            const float m_new = fmaxf(m_old, mx);
+            const float mc_new = (m_new == -INFINITY) ? 0.0f : __fmul_rn(m_new, c);
+            const float alpha = (m_old == -INFINITY) ? 0.0f : ex2_approx(mc_old - mc_new);
+            float psum = 0.0f;
+#pragma unroll
+            for (int e = 0; e < 64; ++e) {
+                S[e] = ex2_approx(__fmaf_rn(S[e], c, -mc_new));
+                if constexpr (!PREORDER) psum += S[e];
+            }
+            if constexpr (!PREORDER) l_hp = __fmaf_rn(alpha, l_hp, psum);
+            // quantize P: 4 blocks of 16 keys
+            uint32_t code[8];
+            uint32_t sfw = 0;
+#pragma unroll
+            for (int blk = 0; blk < 4; ++blk) {
+                float amax = S[16 * blk];
+#pragma unroll
+                for (int e = 1; e < 16; ++e) amax = fmaxf(amax, S[16 * blk + e]);
+                const uint32_t sf = cvt_e4m3(__fmul_rn(amax, one_sixth));
+                const float r = lut[sf & 127u];
+                float y[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) y[e] = __fmul_rn(S[16 * blk + e], r);
+                code[2 * blk] = cvt_e2m1x8(y[0], y[1], y[2], y[3], y[4], y[5], y[6], y[7]);
+                code[2 * blk + 1] = cvt_e2m1x8(y[8], y[9], y[10], y[11], y[12], y[13], y[14], y[15]);
+                sfw |= sf << (8 * blk);
+            }
+            if constexpr (DUMP) {
+                if (valid) {
+                    uint4* dc = reinterpret_cast<uint4*>(p.p_codes + out_row * (size_t)(p.Nkv / 2) + n0 / 2);
+                    dc[0] = make_uint4(code[0], code[1], code[2], code[3]);
+                    dc[1] = make_uint4(code[4], code[5], code[6], code[7]);
+                    *reinterpret_cast<uint32_t*>(p.p_sf + out_row * (size_t)(p.Nkv / 16) + n0 / 16) = sfw;
+                }
+            }
+            if (j > 0) {
+                // PV of the previous tile is done: O is stable, P buffer j&1 is free
+                if (!__all_sync(0xFFFFFFFFu, mbar_wait(&bars->o_done, (j - 1) & 1, ctl))) { ok = false; break; }
+                tc_fence_after();
+                if (__any_sync(0xFFFFFFFFu, alpha != 1.0f)) {
+                    constexpr int HALF = D / 2;
+#pragma unroll 1
+                    for (int cc = wg * HALF; cc < (wg + 1) * HALF; cc += 32) {
+                        uint32_t o[32];
+                        tmem_ld32(tl + C::COL_O + cc, o);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__fmul_rn(__uint_as_float(o[e]), alpha));
+                        tmem_st32(tl + C::COL_O + cc, o);
+                    }
+                    if constexpr (PREORDER) {
+                        if (wg == 1) {
+                            uint32_t lv;
+                            tmem_ld1(tl + C::COL_O + D, lv);
+                            tmem_wait_ld();
+                            lv = __float_as_uint(__fmul_rn(__uint_as_float(lv), alpha));
+                            asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(tl + C::COL_O + D),
+                                         "r"(lv)
+                                         : "memory");
+                        }
+                    }
+                    tmem_wait_st();
+                }
+            }
+            {
+                uint8_t* pb = smem + C::OFF_P + (j & 1) * C::P_BYTES;
+                *reinterpret_cast<uint4*>(pb + p_swizzle64(row, 2 * wg)) = make_uint4(code[0], code[1], code[2], code[3]);
+                *reinterpret_cast<uint4*>(pb + p_swizzle64(row, 2 * wg + 1)) = make_uint4(code[4], code[5], code[6], code[7]);
+                *reinterpret_cast<uint32_t*>(smem + C::OFF_SFP + (j & 1) * C::SFP_BYTES + wg * 512 +
+                                             16 * (row & 31) + 4 * (row >> 5)) = sfw;
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(&bars->p_full[j & 1]);
+            m_old = m_new;
+            mc_old = mc_new;
+        }
+        // ---------------------------------------------------------- epilogue
+        if (ok && n_tiles > 0) ok = __all_sync(0xFFFFFFFFu, mbar_wait(&bars->o_done, (n_tiles - 1) & 1, ctl));
+        if (ok) {
+            tc_fence_after();
+            float l;
+            if constexpr (PREORDER) {
+                uint32_t lv;
+                tmem_ld1(tl + C::COL_O + D, lv);
+                tmem_wait_ld();
+                l = __uint_as_float(lv);
+            } else {
+                float* lx = mx_x;                       // reuse: the row-max buffers are idle now
+                lx[wg * 128 + row] = l_hp;
+                mbar_arrive(&bars->lx);
+                ok = __all_sync(0xFFFFFFFFu, mbar_wait(&bars->lx, 0, ctl));
+                l = lx[row] + lx[128 + row];
+            }
+            if (ok) {
+                const float inv = l > 0.0f ? __frcp_rn(l) : 0.0f;
+                constexpr int HALF = D / 2;
+#pragma unroll 1
+                for (int cc = wg * HALF; cc < (wg + 1) * HALF; cc += 32) {
+                    uint32_t o[32];
+                    tmem_ld32(tl + C::COL_O + cc, o);
+                    tmem_wait_ld();
+                    float v[32];
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) v[e] = __uint_as_float(o[e]) * inv;
+                    if (valid) {
+                        uint8_t* dst = reinterpret_cast<uint8_t*>(p.o) + (out_row * D + cc) * (OUT == 2 ? 4 : 2);
+                        store_out32<OUT>(dst, v);
+                    }
+                }
+                if (wg == 0 && valid && p.lse != nullptr)
+                    p.lse[out_row] = l > 0.0f ? mc_old * 0.69314718055994531f + __logf(l) : -INFINITY;
+            }
+        }
+        (void)ok;
+    }
+    // ---------------------------------------------------------------- teardown
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem, 512);
+}
+
+template <int D, bool PRE, bool CAUSAL, int OUT, bool DUMP>
+static cudaError_t launch_one(const CUtensorMap* q, const CUtensorMap* k, const CUtensorMap* v, const AttnParams& p,
+                              cudaStream_t st) {
+    using C = Cfg<D, PRE>;
+    auto kern = attn_fwd_kernel<D, PRE, CAUSAL, OUT, DUMP>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    kern<<<p.n_work, kThreads, C::SMEM_BYTES, st>>>(*q, *k, *v, p);
+    return cudaGetLastError();
+}
+
+template <int D, bool PRE, bool CAUSAL, int OUT>
+static cudaError_t launch_dump(const CUtensorMap* q, const CUtensorMap* k, const CUtensorMap* v, const AttnParams& p,
+                               bool dump, cudaStream_t st) {
+    return dump ? launch_one<D, PRE, CAUSAL, OUT, true>(q, k, v, p, st)
+                : launch_one<D, PRE, CAUSAL, OUT, false>(q, k, v, p, st);
+}
+
+template <int D, bool PRE, bool CAUSAL>
+static cudaError_t launch_out(const CUtensorMap* q, const CUtensorMap* k, const CUtensorMap* v, const AttnParams& p,
+                              int out, bool dump, cudaStream_t st) {
+    switch (out) {
+        case 0: return launch_dump<D, PRE, CAUSAL, 0>(q, k, v, p, dump, st);
+        case 1: return launch_dump<D, PRE, CAUSAL, 1>(q, k, v, p, dump, st);
+        default: return launch_dump<D, PRE, CAUSAL, 2>(q, k, v, p, dump, st);
+    }
+}
+
+template <int D>
+static cudaError_t launch_d(const CUtensorMap* q, const CUtensorMap* k, const CUtensorMap* v, const AttnParams& p,
+                            int norm, bool causal, int out, bool dump, cudaStream_t st) {
+    if (norm == 0)
+        return causal ? launch_out<D, true, true>(q, k, v, p, out, dump, st)
+                      : launch_out<D, true, false>(q, k, v, p, out, dump, st);
+    return causal ? launch_out<D, false, true>(q, k, v, p, out, dump, st)
+                  : launch_out<D, false, false>(q, k, v, p, out, dump, st);
+}
+
+cudaError_t launch_attention(const CUtensorMap* tmQ, const CUtensorMap* tmK, const CUtensorMap* tmV,
+                             const AttnParams& p, int D, int norm, bool causal, int out_dtype, bool dump,
+                             cudaStream_t st) {
+    switch (D) {
+        case 64: return launch_d<64>(tmQ, tmK, tmV, p, norm, causal, out_dtype, dump, st);
+        case 128: return launch_d<128>(tmQ, tmK, tmV, p, norm, causal, out_dtype, dump, st);
+        case 256: return launch_d<256>(tmQ, tmK, tmV, p, norm, causal, out_dtype, dump, st);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace hifa4

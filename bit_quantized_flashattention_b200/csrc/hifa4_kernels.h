@@ -1,0 +1,45 @@
+// Launchers shared between the C ABI (api.cu) and the kernel files.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace hifa4 {
+
+cudaError_t launch_quantize_rows(bool bf16, const void* x, const float* scale, uint8_t* codes, uint8_t* sfs,
+                                 long long n_groups, int rows_per_group, int tiles_per_group, int heads_per_kv,
+                                 int hkv, int n_per_head, int D, cudaStream_t st);
+
+cudaError_t launch_quantize_v(bool bf16, const void* v, uint8_t* vtc, uint8_t* vts, long long n_groups, int nkv, int D,
+                              cudaStream_t st);
+
+cudaError_t launch_calibrate(bool bf16, const void* q, const void* k, int B, int Hq, int Hkv, int N, int D, float alpha,
+                             float* s, float* s_inv, cudaStream_t st);
+
+struct AttnParams {
+    const uint8_t* qs;       // MMA-ready scales of Q
+    const uint8_t* ks;       // ... of K
+    const uint8_t* vts;      // ... of V^T
+    void* o;                 // [B,Hq,Nq,D] output
+    float* lse;              // [B,Hq,Nq] or null
+    uint8_t* p_codes;        // P_hat dump (debug variant only)
+    uint8_t* p_sf;
+    uint32_t* status;        // workspace status word
+    int B, Hq, Hkv, Nq, Nkv, G;
+    int Tq;                  // 128-row tiles per (b, kv head) group
+    int n_kv_tiles;          // Nkv / 128
+    int n_work;              // grid size = B * Hkv * Tq
+    int heavy_first;         // causal: longest tiles first
+    float c;                 // RN(sm_scale * log2 e)
+    unsigned long long wait_limit_ns;
+    int stall_loads;         // test hook: issue no loads (all waits time out)
+};
+
+// D in {64,128,256}; norm 0 = P-Reordering, 1 = high-precision l;
+// out_dtype 0 = f16, 1 = bf16, 2 = f32.
+cudaError_t launch_attention(const CUtensorMap* tmQ, const CUtensorMap* tmK, const CUtensorMap* tmV,
+                             const AttnParams& p, int D, int norm, bool causal, int out_dtype, bool dump,
+                             cudaStream_t st);
+
+}  // namespace hifa4

@@ -1,0 +1,184 @@
+/*
+ * hifa4.h - C ABI of the B200 (sm_100a) 4-bit FlashAttention forward.
+ *
+ * The method is the HiFA4 operator described in "HiFA4: Training-Free 4-bit
+ * FlashAttention on Ascend HIF4 NPUs for LLM Inference" (abstract; the same
+ * text is printed on the scholarfeed, hf.space, thelatestinai, fugumt and
+ * mlsanity pages): both QK^T and PV run as 4-bit GEMMs, the online-softmax
+ * state stays in a wider float format, Smooth-QK rescales Q and K per channel
+ * with calibration-static factors after RoPE, and P-Reordering accumulates the
+ * softmax normalizer from the same quantized probabilities that feed PV.
+ * The 4-bit format here is E2M1 elements with one E4M3 scale per 16 elements
+ * along the contraction dimension (D for Q and K, tokens for V), rounded to
+ * nearest even; the abstract names the Ascend HIF4 format, whose encoding it
+ * does not give.
+ *
+ * Conventions for every entry point:
+ *  - All tensor pointers are DEVICE pointers owned by the caller. The library
+ *    never allocates, frees or synchronises device memory (hifa4_get_status is
+ *    the only call that waits on the stream).
+ *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default).
+ *  - Arguments are validated on the host before anything is launched; a
+ *    violation returns HIFA4_ERR_INVALID_ARG or HIFA4_ERR_UNSUPPORTED and
+ *    launches nothing. A launch failure returns HIFA4_ERR_CUDA.
+ *  - Every pointer must be 16-byte aligned.
+ *  - Tensors are contiguous, row-major, with the shapes given below.
+ *  - Q is [B, Hq, Nq, D]; K and V are [B, Hkv, Nkv, D]. GQA: q head h reads
+ *    kv head h / (Hq / Hkv).
+ *  - Supported: D in {64, 128, 256}; Hq % Hkv == 0; Nkv % 128 == 0;
+ *    Nq % 16 == 0; causal needs Nq <= Nkv (bottom-right aligned: key j is
+ *    visible to query i iff j <= i + Nkv - Nq).
+ */
+#ifndef HIFA4_H
+#define HIFA4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* hifa4_stream_t;   /* same type as cudaStream_t */
+
+typedef enum {
+    HIFA4_OK = 0,
+    HIFA4_ERR_INVALID_ARG = 1,   /* bad pointer, shape, alignment or value */
+    HIFA4_ERR_UNSUPPORTED = 2,   /* valid request outside what the kernels cover */
+    HIFA4_ERR_CUDA = 3,          /* a CUDA call or launch failed */
+    HIFA4_ERR_TIMEOUT = 4        /* a bounded wait inside a kernel expired */
+} hifa4_status;
+
+/* Normalizer modes of the attention kernel (HiFA4 abstract, P-Reordering):
+ * P_REORDER            l accumulated from the quantized P_hat that feeds the
+ *                      PV GEMM, fused into that GEMM as an extra V column of ones.
+ * HIGH_PRECISION_L     l accumulated from the unquantized fp32 P (the
+ *                      "higher-precision reconstruction" the abstract compares with). */
+typedef enum { HIFA4_NORM_P_REORDER = 0, HIFA4_NORM_HIGH_PRECISION_L = 1 } hifa4_norm_mode;
+
+typedef enum { HIFA4_F16 = 0, HIFA4_BF16 = 1, HIFA4_F32 = 2 } hifa4_dtype;
+
+enum { HIFA4_CAUSAL = 1u << 0 };
+
+/* Quantized operands. Layouts (u8 everywhere; codes hold two E2M1 elements
+ * per byte, element 2i in the low nibble; scales are E4M3 bytes):
+ *   qc  [B, Hq, Nq, D/2]         Q codes, row-major
+ *   kc  [B, Hkv, Nkv, D/2]       K codes, row-major
+ *   vtc [B, Hkv, D, Nkv/2]       V codes, transposed (tokens contiguous)
+ *   qs, ks, vts                  scales in the MMA-ready layout below
+ * MMA-ready scale layout: 512-byte atoms, each holding the scales of 128 rows x
+ * 64 contraction elements (4 scales per row); row r, scale k (0..3) of an atom
+ * sits at byte 16*(r%32) + 4*(r/32) + k.
+ *   qs: atoms ordered [B, Hkv, Tq, D/64], Tq = ceil(G*Nq/128), G = Hq/Hkv. The
+ *       rows of atom (b, g, t) are the query rows p = 128*t + r of the group's
+ *       heads stacked head after head, p = (h % G)*Nq + i. Rows past G*Nq are 0.
+ *   ks: atoms ordered [B, Hkv, Nkv/128, D/64], row r = token % 128.
+ *   vts: atoms ordered [B, Hkv, Nkv/128, ceil(D/128), 2], row r = channel % 128
+ *       of the 128-channel block, k = (token % 64)/16 of the 64-token half.
+ *       When D = 64 the padding row 64 holds 0x38 (1.0): the scale of the
+ *       normalizer column used by P-Reordering. Other padding rows are 0.
+ * The canonical scale tensors Qs [B,Hq,Nq,D/16], Ks [B,Hkv,Nkv,D/16] and
+ * Vts [B,Hkv,D,Nkv/16] map one-to-one onto these bytes. */
+typedef struct {
+    void* qc;
+    void* qs;
+    void* kc;
+    void* ks;
+    void* vtc;
+    void* vts;
+} hifa4_packed;
+
+/* Bytes of each packed buffer, in the order qc, qs, kc, ks, vtc, vts, written
+ * to out[6] (may be NULL). Returns their sum, or 0 for an unsupported shape. */
+size_t hifa4_packed_bytes(int B, int Hq, int Hkv, int Nq, int Nkv, int D, size_t out[6]);
+
+/* Bytes of the device workspace hifa4_attention_fwd needs: a status word and
+ * a work counter. The caller zeroes it once after allocating; the kernels
+ * leave the counter at zero when they finish. */
+size_t hifa4_workspace_bytes(int B, int Hq, int Hkv, int Nq, int Nkv, int D);
+
+/* Smooth-QK calibration (HiFA4 abstract: "calibration-static per-channel
+ * equivalent rescaling ... transferring quantization difficulty from K to Q").
+ * For each kv head g and channel c: aQ = max |Q| over the batch, the N tokens
+ * and the q heads of group g; aK = max |K| over the batch and tokens;
+ * s = aK^alpha / aQ^(1-alpha) (alpha = 0.5 gives sqrt(aK/aQ), computed as
+ * correctly rounded fp32 division and square root), s = 1 when aQ or aK is 0,
+ * s_inv = RN(1/s). q: [B,Hq,N,D], k: [B,Hkv,N,D] in `dtype` (F16 or BF16);
+ * s, s_inv: fp32 [Hkv, D], written (their previous contents are overwritten;
+ * they also serve as the reduction scratch). alpha in (0, 1]. */
+hifa4_status hifa4_calibrate_smooth(const void* q, const void* k, hifa4_dtype dtype,
+                                    int B, int Hq, int Hkv, int N, int D, float alpha,
+                                    float* s, float* s_inv, hifa4_stream_t stream);
+
+/* Smooth and quantize Q, K and V (HiFA4 abstract: Smooth-QK "after RoPE",
+ * then 4-bit QK^T and PV GEMMs). Q' = RN(Q*s[g]), K' = RN(K*s_inv[g]) in fp32
+ * (s and s_inv both NULL: no smoothing). Per 16-element block along the
+ * contraction dimension: sf = E4M3_rn_satfinite(amax * RN(1/6)), r = RN(1/sf)
+ * (0 when sf = 0), code = E2M1_rn_satfinite(RN(x*r)). Q and K are blocked
+ * along D, V along tokens (written transposed). q, k, v in `dtype`
+ * (F16 or BF16); out points at caller-allocated buffers sized by
+ * hifa4_packed_bytes. */
+hifa4_status hifa4_quantize_qkv(const void* q, const void* k, const void* v, hifa4_dtype dtype,
+                                int B, int Hq, int Hkv, int Nq, int Nkv, int D,
+                                const float* s, const float* s_inv,
+                                const hifa4_packed* out, hifa4_stream_t stream);
+
+/* Quantize only K and V (a KV cache is quantized once, when it is appended).
+ * Same rules and layouts as hifa4_quantize_qkv; out->qc / out->qs are ignored. */
+hifa4_status hifa4_quantize_kv(const void* k, const void* v, hifa4_dtype dtype,
+                               int B, int Hkv, int Nkv, int D, const float* s_inv,
+                               const hifa4_packed* out, hifa4_stream_t stream);
+
+/* 4-bit attention forward (HiFA4 abstract). For each query row, one pass over
+ * 128-key tiles in ascending order: S = Q_hat K_hat^T (block-scaled FP4 MMA,
+ * fp32 accumulate), running max m updated every tile, c = RN(sm_scale*log2 e),
+ * P = 2^(S*c - RN(m*c)), P quantized per 16 keys to P_hat with the element
+ * rule above, O_acc = alpha*O_acc + P_hat V_hat (block-scaled FP4 MMA), and the
+ * normalizer l per `norm` (see hifa4_norm_mode). Output O = O_acc / l in
+ * `o_dtype` [B,Hq,Nq,D]; lse (fp32 [B,Hq,Nq], may be NULL) =
+ * RN(m*c)*ln 2 + ln l, the natural-log log-sum-exp of sm_scale*S.
+ * sm_scale: finite and > 0 (1/sqrt(D) is the usual value). flags: HIFA4_CAUSAL.
+ * workspace: hifa4_workspace_bytes() bytes, zeroed once by the caller; a
+ * bounded wait that expires inside the kernel records HIFA4_ERR_TIMEOUT there
+ * (read it with hifa4_get_status). Concurrent calls must use different
+ * workspaces. */
+hifa4_status hifa4_attention_fwd(const hifa4_packed* in, int B, int Hq, int Hkv, int Nq, int Nkv, int D,
+                                 float sm_scale, unsigned flags, hifa4_norm_mode norm,
+                                 void* o, hifa4_dtype o_dtype, float* lse,
+                                 void* workspace, hifa4_stream_t stream);
+
+/* Same as hifa4_attention_fwd, and also writes the quantized probabilities
+ * P_hat the PV GEMM consumed: p_codes [B,Hq,Nq,Nkv/2] (two E2M1 codes per byte,
+ * key 2i in the low nibble) and p_scales [B,Hq,Nq,Nkv/16] (E4M3). Tiles the
+ * kernel skips (entirely above the causal diagonal for the row's 128-row
+ * tile) are not written, so the caller zeroes both buffers first. A debugging
+ * aid for checking P_hat against a reference; slower than the plain call. */
+hifa4_status hifa4_attention_fwd_debug(const hifa4_packed* in, int B, int Hq, int Hkv, int Nq, int Nkv, int D,
+                                       float sm_scale, unsigned flags, hifa4_norm_mode norm,
+                                       void* o, hifa4_dtype o_dtype, float* lse,
+                                       uint8_t* p_codes, uint8_t* p_scales,
+                                       void* workspace, hifa4_stream_t stream);
+
+/* Synchronises `stream`, then returns the status a kernel recorded in
+ * `workspace` (HIFA4_OK or HIFA4_ERR_TIMEOUT) or HIFA4_ERR_CUDA if the stream
+ * reported an error. Clears the recorded status. */
+hifa4_status hifa4_get_status(void* workspace, hifa4_stream_t stream);
+
+/* Test hook for the timeout path: sets the wait limit (nanoseconds) that the
+ * attention kernel's bounded waits use from the next launch on (0 restores the
+ * default of 2 s), and, when `stall_loads` is nonzero, makes the next launches'
+ * load warp issue no loads, so every consumer wait runs out with nothing in
+ * flight. Returns the previous limit. */
+long long hifa4_debug_set_wait_limit(long long limit_ns, int stall_loads);
+
+/* Human-readable name of a status code. */
+const char* hifa4_status_string(hifa4_status status);
+
+/* Library version, major*10000 + minor*100 + patch. */
+int hifa4_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HIFA4_H */
