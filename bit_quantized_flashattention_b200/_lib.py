@@ -14,7 +14,7 @@ CAUSAL = 1
 
 EXPORTS = ["hifa4_packed_bytes", "hifa4_workspace_bytes", "hifa4_calibrate_smooth", "hifa4_quantize_qkv",
            "hifa4_quantize_kv", "hifa4_attention_fwd", "hifa4_attention_fwd_debug", "hifa4_get_status",
-           "hifa4_debug_set_wait_limit", "hifa4_status_string", "hifa4_version"]
+           "hifa4_debug_set_wait_limit", "hifa4_status_string", "hifa4_version", "hifa4_attention_fwd_noalloc"]
 
 
 class Packed(ctypes.Structure):
@@ -54,6 +54,8 @@ def load():
     L.hifa4_attention_fwd.restype = ci
     L.hifa4_attention_fwd_debug.argtypes = [pk] + [ci] * 6 + [cf, cu, ci, vp, ci, vp, vp, vp, vp, vp]
     L.hifa4_attention_fwd_debug.restype = ci
+    L.hifa4_attention_fwd_noalloc.argtypes = [pk] + [ci] * 6 + [cf, cu, ci, vp, ci, vp, vp]
+    L.hifa4_attention_fwd_noalloc.restype = ci
     L.hifa4_get_status.argtypes = [vp, vp]
     L.hifa4_get_status.restype = ci
     L.hifa4_debug_set_wait_limit.argtypes = [ctypes.c_longlong, ci]

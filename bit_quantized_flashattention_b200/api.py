@@ -162,6 +162,26 @@ def attention_fwd(packed: PackedQKV, sm_scale: float | None = None, causal: bool
     return out, lse
 
 
+def attention_fwd_noalloc(packed: PackedQKV, sm_scale: float | None = None, causal: bool = False,
+                          norm="p_reorder", out_dtype=torch.bfloat16, out=None, lse=None, stream=None):
+    """attention_fwd for callers that cannot allocate device memory: the library
+    uses its own fixed scratch (see hifa4_attention_fwd_noalloc in hifa4.h).
+    ``out``/``lse`` are still the caller's buffers (allocated here when None)."""
+    B, Hq, Hkv, Nq, Nkv, D = packed.shape
+    dev = packed.qc.device
+    if sm_scale is None:
+        sm_scale = 1.0 / math.sqrt(D)
+    if out is None:
+        out = torch.empty(B, Hq, Nq, D, dtype=out_dtype, device=dev)
+    if lse is None:
+        lse = torch.empty(B, Hq, Nq, dtype=torch.float32, device=dev)
+    st = packed.struct()
+    L.check(L.load().hifa4_attention_fwd_noalloc(ctypes.byref(st), B, Hq, Hkv, Nq, Nkv, D, float(sm_scale),
+                                                 L.CAUSAL if causal else 0, _NORM[norm], _ptr(out), _DT[out.dtype],
+                                                 _ptr(lse), _stream(stream)), "attention_fwd_noalloc")
+    return out, lse
+
+
 def attention_fwd_debug(packed: PackedQKV, sm_scale: float | None = None, causal: bool = False,
                         norm="p_reorder", out_dtype=torch.float32, workspace=None, stream=None):
     """attention_fwd plus the P_hat the PV GEMM consumed: (O, LSE, p_codes, p_scales)."""

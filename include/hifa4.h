@@ -159,6 +159,31 @@ hifa4_status hifa4_attention_fwd_debug(const hifa4_packed* in, int B, int Hq, in
                                        uint8_t* p_codes, uint8_t* p_scales,
                                        void* workspace, hifa4_stream_t stream);
 
+/* hifa4_attention_fwd without a caller-provided workspace, for callers that
+ * cannot allocate device memory: for example a plugin inside a host runtime
+ * that owns all device memory and exposes no allocator, or a latency-critical
+ * path that cannot afford cudaMalloc's implicit device synchronisation. It
+ * allocates nothing (no cudaMalloc, cudaFree or allocating library routine);
+ * its scratch is a fixed 4096-byte array in the library's device image, which
+ * every GPU that loads the library holds until the process exits. (The HiFA4
+ * paper has no counterpart of this call; it is an integration aid.)
+ * Arguments, layouts and results are those of hifa4_attention_fwd.
+ *  - The first call on each device looks up the array's device address
+ *    (cudaGetSymbolAddress, no allocation) with that device current; make that
+ *    first call before any stream capture.
+ *  - Every call clears the part of the array it uses (the status word and the
+ *    work counter) on `stream` before launching.
+ *  - Problems whose hifa4_workspace_bytes exceeds 4096 return
+ *    HIFA4_ERR_UNSUPPORTED without launching.
+ *  - All calls on a device share the one array: calls that overlap on the GPU
+ *    (different streams without ordering between them) race on it. Order them.
+ *  - A bounded wait that expires in the kernel is not reported back by this
+ *    call (it has no workspace to read); use hifa4_attention_fwd with a
+ *    workspace when that status is needed. */
+hifa4_status hifa4_attention_fwd_noalloc(const hifa4_packed* in, int B, int Hq, int Hkv, int Nq, int Nkv, int D,
+                                         float sm_scale, unsigned flags, hifa4_norm_mode norm,
+                                         void* o, hifa4_dtype o_dtype, float* lse, hifa4_stream_t stream);
+
 /* Synchronises `stream`, then returns the status a kernel recorded in
  * `workspace` (HIFA4_OK or HIFA4_ERR_TIMEOUT) or HIFA4_ERR_CUDA if the stream
  * reported an error. Clears the recorded status. */
