@@ -88,3 +88,50 @@ def row_errors(o_gpu: np.ndarray, o_ref: np.ndarray):
     den = np.linalg.norm(o_ref, axis=-1)
     rel = np.where(den < 1e-6, num, num / np.maximum(den, 1e-30))
     return max_abs, rel
+
+
+def upload_config(cfg, device="cuda"):
+    """Seeded inputs of a workload config on the device, built slice by slice.
+    Returns (q, k, v, calib) with calib = (Qcal, Kcal) device tensors or None."""
+    dt = TORCH_DT[cfg.dtype]
+    gains = W.k_gains(cfg)
+
+    def up(x):
+        return torch.from_numpy(W.to_bits(x, cfg.dtype).view(np.int16).copy()).to(device).view(dt)
+
+    q = torch.empty(cfg.B, cfg.Hq, cfg.Nq, cfg.D, dtype=dt, device=device)
+    k = torch.empty(cfg.B, cfg.Hkv, cfg.Nkv, cfg.D, dtype=dt, device=device)
+    v = torch.empty_like(k)
+    for b in range(cfg.B):
+        for h in range(cfg.Hq):
+            q[b, h] = up(W.q_slice(cfg, b, h))
+        for g in range(cfg.Hkv):
+            k[b, g] = up(W.k_slice(cfg, b, g, gains))
+            v[b, g] = up(W.v_slice(cfg, b, g))
+    calib = None
+    if cfg.smooth == "calib":
+        calib = (torch.stack([up(W.qcal_slice(cfg, h)) for h in range(cfg.Hq)])[None].contiguous(),
+                 torch.stack([up(W.kcal_slice(cfg, g, gains)) for g in range(cfg.Hkv)])[None].contiguous())
+    elif cfg.smooth == "self":
+        calib = (q, k)
+    return q, k, v, calib
+
+
+def group_arrays(cfg, b, g):
+    """Host copies (exact dtype values, float32) of one (batch, kv head) group:
+    q [1,G,Nq,D], k [1,1,Nkv,D], v [1,1,Nkv,D]."""
+    gains = W.k_gains(cfg)
+    q = np.stack([W.q_slice(cfg, b, g * cfg.G + hh) for hh in range(cfg.G)])[None]
+    k = W.k_slice(cfg, b, g, gains)[None, None]
+    v = W.v_slice(cfg, b, g)[None, None]
+    return q, k, v
+
+
+def calib_arrays(cfg):
+    """Host calibration tensors of a config (None when smoothing is off)."""
+    if cfg.smooth == "off":
+        return None
+    if cfg.smooth == "self":
+        q, k, _ = W.full(cfg)
+        return q, k
+    return W.calib_full(cfg)

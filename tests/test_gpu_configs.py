@@ -1,0 +1,112 @@
+"""Parity on the five full-size workloads, in the launch configuration the
+benchmark times (same kernels, same shapes), against the CPU oracle on
+sampled (batch, kv head) groups and sampled query rows.
+
+Bars as in test_gpu_parity.py: calibration factors and quantized operands
+bit-exact; P_hat code mismatch <= 1e-4; O (fp32 output) max abs <= 5e-3 and
+per-row relative L2 <= 1e-3; LSE max abs <= 1e-3.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads as W
+from tests import hifa4_testutil as U
+
+pytestmark = pytest.mark.gpu
+
+O_MAX_ABS = 5e-3
+O_ROW_REL = 1e-3
+LSE_ABS = 1e-3
+P_MISMATCH = 1e-4
+ROWS_PER_HEAD = 24
+
+
+@pytest.fixture(scope="module")
+def H():
+    import bit_quantized_flashattention_b200 as H
+    H.load()
+    return H
+
+
+def _sample_groups(cfg, rng):
+    grps = [(0, 0), (cfg.B - 1, cfg.Hkv - 1)]
+    if cfg.B * cfg.Hkv > 2:
+        grps.append((int(rng.integers(cfg.B)), int(rng.integers(cfg.Hkv))))
+    return sorted(set(grps))
+
+
+def _sample_rows(cfg, rng):
+    i = np.unique(np.concatenate([np.arange(min(4, cfg.Nq)), cfg.Nq - 1 - np.arange(min(4, cfg.Nq)),
+                                  rng.integers(0, cfg.Nq, ROWS_PER_HEAD)]))
+    return np.sort(i)
+
+
+@pytest.mark.parametrize("index", [1, 2, 3, 4, 5])
+def test_config_parity(H, index):
+    cfg = W.get(index)
+    rng = np.random.default_rng(100 + index)
+    q, k, v, calib = U.upload_config(cfg)
+    s = s_inv = None
+    ref_s = ref_si = None
+    if calib is not None:
+        s, s_inv = H.calibrate_smooth(calib[0], calib[1], cfg.alpha)
+        cq, ck = U.calib_arrays(cfg)
+        ref_s, ref_si = oracle.calibrate(cq, ck, cfg.alpha)
+        assert np.array_equal(s.cpu().numpy(), ref_s) and np.array_equal(s_inv.cpu().numpy(), ref_si)
+    pk = H.quantize_qkv(q, k, v, s, s_inv)
+    dump = cfg.B * cfg.Hq * cfg.Nq * cfg.Nkv // 2 <= (1 << 30)
+    results = {}
+    for norm in cfg.modes:
+        if dump:
+            o, lse, pc, ps = H.attention_fwd_debug(pk, causal=cfg.causal, norm=norm)
+        else:
+            o, lse = H.attention_fwd(pk, causal=cfg.causal, norm=norm, out_dtype=torch.float32)
+            pc = ps = None
+        o_bf16, _ = H.attention_fwd(pk, causal=cfg.causal, norm=norm, out_dtype=torch.bfloat16)
+        torch.cuda.synchronize()
+        results[norm] = (o, lse, pc, ps, o_bf16)
+
+    qs_all, ks_all, vts_all = U.canonical_scales(pk, cfg.B, cfg.Hq, cfg.Hkv, cfg.Nq, cfg.Nkv, cfg.D)
+    qc_all = pk.qc.view(cfg.B, cfg.Hq, cfg.Nq, cfg.D // 2)
+    kc_all = pk.kc.view(cfg.B, cfg.Hkv, cfg.Nkv, cfg.D // 2)
+    vtc_all = pk.vtc.view(cfg.B, cfg.Hkv, cfg.D, cfg.Nkv // 2)
+    G = cfg.G
+    n_codes = n_mism = 0
+    for (b, g) in _sample_groups(cfg, rng):
+        qh, kh, vh = U.group_arrays(cfg, b, g)
+        sg = None if ref_s is None else ref_s[g:g + 1]
+        sgi = None if ref_si is None else ref_si[g:g + 1]
+        ref_p = oracle.quantize_qkv(qh, kh, vh, sg, sgi)
+        hs = slice(g * G, (g + 1) * G)
+        assert np.array_equal(qc_all[b, hs].cpu().numpy(), ref_p["qc"][0])
+        assert np.array_equal(qs_all[b, hs], ref_p["qs"][0])
+        assert np.array_equal(kc_all[b, g].cpu().numpy(), ref_p["kc"][0, 0])
+        assert np.array_equal(ks_all[b, g], ref_p["ks"][0, 0])
+        assert np.array_equal(vtc_all[b, g].cpu().numpy(), ref_p["vtc"][0, 0])
+        assert np.array_equal(vts_all[b, g], ref_p["vts"][0, 0])
+        idx = _sample_rows(cfg, rng)
+        rows_local = np.concatenate([hh * cfg.Nq + idx for hh in range(G)])
+        for norm in cfg.modes:
+            o, lse, pc, ps, o_bf16 = results[norm]
+            ref = oracle.attention_rows((1, G, 1, cfg.Nq, cfg.Nkv, cfg.D), rows_local, packed=ref_p,
+                                        causal=cfg.causal, norm_mode=0 if norm == "p_reorder" else 1,
+                                        want_p=dump)
+            og = o[b, hs][:, idx].reshape(-1, cfg.D).float().cpu().numpy()
+            max_abs, rel = U.row_errors(og, ref["O"])
+            assert max_abs <= O_MAX_ABS, (norm, b, g, max_abs)
+            assert rel.max() <= O_ROW_REL, (norm, b, g, rel.max())
+            lg = lse[b, hs][:, idx].reshape(-1).cpu().numpy()
+            assert np.abs(lg - ref["lse"]).max() <= LSE_ABS
+            ob = o_bf16[b, hs][:, idx].reshape(-1, cfg.D).float().cpu().numpy()
+            rb = torch.from_numpy(ref["O"]).to(torch.bfloat16).float().numpy()
+            assert np.all(np.abs(ob - rb) <= 2.0 ** -7 * np.maximum(np.abs(rb), 2 ** -6) + 5e-4)
+            if dump:
+                pcg = pc[b, hs][:, idx].reshape(len(rows_local), -1).cpu().numpy()
+                nib_g = np.stack([pcg & 15, pcg >> 4], -1)
+                nib_r = np.stack([ref["p_codes"] & 15, ref["p_codes"] >> 4], -1)
+                n_codes += nib_g.size
+                n_mism += int((nib_g != nib_r).sum())
+    if dump:
+        assert n_mism <= P_MISMATCH * n_codes, (n_mism, n_codes)

@@ -164,6 +164,8 @@ def _check_attention(o, lse, pc, ps, ref, D, out_dtype=torch.float32):
     ((2, 4, 2, 176, 512, 128), True),          # Nq < Nkv, G*Nq = 352: tiles mix heads, ragged tail
     ((1, 2, 2, 256, 256, 256), True),
     ((1, 8, 2, 16, 512, 128), False),          # decode-style: 4 heads x 16 queries in one tile
+    ((1, 4, 2, 512, 512, 128), True),          # Nq % 256 == 0: paired query tiles, longest first
+    ((1, 2, 1, 384, 384, 64), True),
 ])
 @pytest.mark.parametrize("norm", ["p_reorder", "high_precision_l"])
 def test_attention_matches_oracle(H, shape, causal, norm):
