@@ -100,7 +100,8 @@ hifa4_status attention_impl(const hifa4_packed* in, int B, int Hq, int Hkv, int 
     const long long rows_q = (long long)B * Hq * Nq, rows_k = (long long)B * Hkv * Nkv, rows_v = (long long)B * Hkv * D;
     if (rows_q > INT32_MAX || rows_k > INT32_MAX || rows_v > INT32_MAX) return HIFA4_ERR_UNSUPPORTED;
     const Sizes sz = sizes_of(B, Hq, Hkv, Nq, Nkv, D);
-    const long long n_work = (long long)B * Hkv * sz.Tq;
+    const int nqt = D == 256 ? 1 : 2;              // query tiles per CTA (see attention.cu)
+    const long long n_work = (long long)B * Hkv * ((sz.Tq + nqt - 1) / nqt);
     if (n_work > INT32_MAX) return HIFA4_ERR_UNSUPPORTED;
 
     const CUtensorMapSwizzle swz_qk =
@@ -129,7 +130,7 @@ hifa4_status attention_impl(const hifa4_packed* in, int B, int Hq, int Hkv, int 
     p.Tq = sz.Tq;
     p.n_kv_tiles = Nkv / 128;
     p.n_work = (int)n_work;
-    p.heavy_first = (causal && Nq % 128 == 0) ? 1 : 0;
+    p.heavy_first = (causal && Nq % (128 * nqt) == 0) ? 1 : 0;
     p.c = (float)((double)sm_scale * 1.4426950408889634074);
     const long long lim = g_wait_limit_ns.load();
     p.wait_limit_ns = lim > 0 ? (unsigned long long)lim : kDefaultWaitNs;

@@ -34,12 +34,13 @@
 
 namespace hifa4 {
 
-constexpr int kThreads = 384;
 constexpr int kStages = 3;
-constexpr int kSoftmaxWarp0 = 4;
+constexpr int kSmWarp0 = 2;          // first softmax warp
 
 template <int D, bool PREORDER>
 struct Cfg {
+    static constexpr int NQT = D == 256 ? 1 : 2;          // 128-row query tiles per CTA
+    static constexpr int THREADS = 64 + 128 * NQT;
     static constexpr int KS = D / 64;                     // 64-wide K steps of QK^T
     static constexpr int QK_ROW = D / 2;                  // bytes per Q/K row
     static constexpr uint32_t QK_SWZ = D == 64 ? 6u : (D == 128 ? 4u : 2u);   // 32B/64B/128B swizzle
@@ -49,40 +50,38 @@ struct Cfg {
     static constexpr int SFQK_BYTES = KS * 512;
     static constexpr int VROWS = D + 16;                  // V^T rows + normalizer block
     static constexpr int V_BYTES = VROWS * 64;
+    static constexpr int V_STRIDE = (V_BYTES + 1023) / 1024 * 1024;
     static constexpr int V_TMA_BYTES = D * 64;
     static constexpr int NRB = (D + 127) / 128;           // 128-row blocks of V^T scales
     static constexpr int SFV_BYTES = NRB * 2 * 512;
     static constexpr int P_BYTES = 128 * 64;
     static constexpr int SFP_BYTES = 2 * 512;
-    static constexpr int NO = PREORDER ? D + 16 : D;      // accumulator columns
+    static constexpr int NO = PREORDER ? D + 16 : D;      // accumulator columns per query tile
     // TMEM columns
     static constexpr uint32_t COL_S = 0;
-    static constexpr uint32_t COL_O = 128;
-    static constexpr uint32_t COL_SFQ = COL_O + NO;
-    static constexpr uint32_t COL_SFK = COL_SFQ + 4 * KS;
-    static constexpr uint32_t COL_SFP = COL_SFK + 4 * KS;
-    static constexpr uint32_t COL_SFV = COL_SFP + 8;
+    static constexpr uint32_t COL_O = 128;                                // + qt * NO
+    static constexpr uint32_t COL_SFQ = COL_O + NQT * NO;                 // + qt * 4 * KS
+    static constexpr uint32_t COL_SFK = COL_SFQ + NQT * 4 * KS;
+    static constexpr uint32_t COL_SFP = COL_SFK + 4 * KS;                 // + qt * 8
+    static constexpr uint32_t COL_SFV = COL_SFP + NQT * 8;
     // scale columns per PV K step: one 4-column block per 128 rows of the B operand
     static constexpr int SFV_PER_KS = 4 * (NRB + ((PREORDER && D >= 128) ? 1 : 0));
     static constexpr uint32_t COL_END = COL_SFV + 2 * SFV_PER_KS;
     static_assert(COL_END <= 512, "TMEM budget");
-    // shared memory offsets (1024-aligned operand tiles)
-    static constexpr int OFF_Q = 0;
-    static constexpr int OFF_K = OFF_Q + Q_BYTES;
+    // shared memory offsets (operand tiles 1024-aligned)
+    static constexpr int OFF_Q = 0;                                       // + qt * Q_BYTES
+    static constexpr int OFF_K = OFF_Q + NQT * Q_BYTES;
     static constexpr int OFF_V = OFF_K + kStages * K_BYTES;
-    static constexpr int OFF_P = OFF_V + kStages * ((V_BYTES + 1023) / 1024 * 1024);
-    static constexpr int V_STRIDE = (V_BYTES + 1023) / 1024 * 1024;
-    static constexpr int OFF_SFQ = OFF_P + 2 * P_BYTES;
-    static constexpr int OFF_SFK = OFF_SFQ + SFQK_BYTES;
+    static constexpr int OFF_P = OFF_V + kStages * V_STRIDE;              // + (qt * 2 + buf) * P_BYTES
+    static constexpr int OFF_SFQ = OFF_P + NQT * 2 * P_BYTES;             // + qt * SFQK_BYTES
+    static constexpr int OFF_SFK = OFF_SFQ + NQT * SFQK_BYTES;
     static constexpr int OFF_SFV = OFF_SFK + kStages * SFQK_BYTES;
-    static constexpr int OFF_SFP = OFF_SFV + kStages * SFV_BYTES;
-    static constexpr int OFF_ONES = OFF_SFP + 2 * SFP_BYTES;
-    static constexpr int OFF_MX = OFF_ONES + 512;                     // float [2][2][128]
-    static constexpr int OFF_LUT = OFF_MX + 2 * 2 * 128 * 4;          // float [128]
+    static constexpr int OFF_SFP = OFF_SFV + kStages * SFV_BYTES;         // + (qt * 2 + buf) * SFP_BYTES
+    static constexpr int OFF_ONES = OFF_SFP + NQT * 2 * SFP_BYTES;
+    static constexpr int OFF_LUT = OFF_ONES + 512;                        // float [128]
     static constexpr int OFF_BAR = OFF_LUT + 128 * 4;
-    static constexpr int N_BARS = 1 + 4 * kStages + 1 + 1 + 2 + 1 + 1 + 2 + 1;
-    static constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;
-    static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;          // + alignment slack
+    static constexpr int OFF_MISC = OFF_BAR + 256;
+    static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;              // + alignment slack
 };
 
 struct Bars {
@@ -91,14 +90,13 @@ struct Bars {
     uint64_t k_empty[kStages];
     uint64_t v_full[kStages];
     uint64_t v_empty[kStages];
-    uint64_t s_full;      // S of the current tile is in TMEM
-    uint64_t s_free;      // both warpgroups have read S
-    uint64_t p_full[2];   // P_hat buffer ready (and O rescaled)
-    uint64_t o_done;      // PV MMA of a tile finished
-    uint64_t drain;       // teardown of the MMA issuer
-    uint64_t mx[2];       // row-max exchange between the two warpgroups
-    uint64_t lx;          // normalizer exchange at the end
+    uint64_t s_full[2];      // S of query tile qt is in TMEM
+    uint64_t s_free[2];      // its warpgroup has read it (the S columns are free again)
+    uint64_t p_full[2][2];   // P_hat buffer (qt, j & 1) ready and O of qt rescaled
+    uint64_t o_done[2];      // PV MMA of query tile qt finished
+    uint64_t drain;          // teardown of the MMA issuer
 };
+static_assert(sizeof(Bars) <= 256, "barrier area");
 
 __device__ __forceinline__ uint32_t p_swizzle64(uint32_t row, uint32_t chunk) {
     return row * 64u + ((chunk ^ ((row >> 1) & 3u)) << 4);
@@ -128,49 +126,76 @@ __device__ __forceinline__ void store_out32(void* dst, const float (&v)[32]) {
     }
 }
 
+// Row maximum of 128 values: a three-input max tree (64 instructions, depth 5).
+__device__ __forceinline__ float row_max128(const float (&v)[128]) {
+    float a[43];
+#pragma unroll
+    for (int i = 0; i < 42; ++i) a[i] = fmax3f(v[3 * i], v[3 * i + 1], v[3 * i + 2]);
+    a[42] = fmaxf(v[126], v[127]);
+    float b[15];
+#pragma unroll
+    for (int i = 0; i < 14; ++i) b[i] = fmax3f(a[3 * i], a[3 * i + 1], a[3 * i + 2]);
+    b[14] = a[42];
+    float c[5];
+#pragma unroll
+    for (int i = 0; i < 5; ++i) c[i] = fmax3f(b[3 * i], b[3 * i + 1], b[3 * i + 2]);
+    return fmax3f(fmax3f(c[0], c[1], c[2]), c[3], c[4]);
+}
+
+// Maximum of 16 non-negative values (8 instructions, depth 3).
+__device__ __forceinline__ float block_max16(const float* v) {
+    const float a0 = fmax3f(v[0], v[1], v[2]), a1 = fmax3f(v[3], v[4], v[5]), a2 = fmax3f(v[6], v[7], v[8]);
+    const float a3 = fmax3f(v[9], v[10], v[11]), a4 = fmax3f(v[12], v[13], v[14]);
+    return fmax3f(fmax3f(a0, a1, a2), fmax3f(a3, a4, v[15]), 0.0f);
+}
+
 template <int D, bool PREORDER, bool CAUSAL, int OUT, bool DUMP>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(Cfg<D, PREORDER>::THREADS, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
     using C = Cfg<D, PREORDER>;
+    constexpr int NQT = C::NQT;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     Bars* bars = reinterpret_cast<Bars*>(smem + C::OFF_BAR);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
-    float* mx_x = reinterpret_cast<float*>(smem + C::OFF_MX);
     float* lut = reinterpret_cast<float*>(smem + C::OFF_LUT);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
     // ---------------------------------------------------------------- work
+    // One work unit = up to NQT consecutive 128-row query tiles of one group.
     const int w = blockIdx.x;
-    int grp, t;
-    {
-        const int n_grp = p.B * p.Hkv;
-        if (p.heavy_first) {
-            // causal, Nq % 128 == 0: largest query block first
-            const int th = p.Nq / 128;
-            const int per = n_grp * p.G;
-            const int iblk = th - 1 - w / per;
-            const int rem = w % per;
-            grp = rem / p.G;
-            t = (rem % p.G) * th + iblk;
-        } else {
-            grp = w / p.Tq;
-            t = w % p.Tq;
-        }
+    const int units_per_grp = (p.Tq + NQT - 1) / NQT;
+    int grp, t0;
+    if (p.heavy_first) {
+        // causal with Nq % (128 * NQT) == 0: units with the most keys first
+        const int per_head = p.Nq / (128 * NQT);
+        const int per = p.B * p.Hkv * p.G;
+        const int u = per_head - 1 - w / per;
+        const int rem = w % per;
+        grp = rem / p.G;
+        t0 = (rem % p.G) * (p.Nq / 128) + u * NQT;
+    } else {
+        grp = w / units_per_grp;
+        t0 = (w % units_per_grp) * NQT;
     }
+    const int n_qt = min(NQT, p.Tq - t0);
     const int rows_in_grp = p.G * p.Nq;
-    const int p0 = t * 128;
-    int n_tiles = p.n_kv_tiles;
-    if (CAUSAL) {
+    // kv tiles each query tile visits (causal: up to the last visible key of its last row)
+    auto kv_tiles_of = [&](int qt) -> int {
+        if (qt >= n_qt) return 0;
+        if (!CAUSAL) return p.n_kv_tiles;
+        const int p0 = (t0 + qt) * 128;
         const int p_max = min(p0 + 127, rows_in_grp - 1);
         const int i_max = (p_max / p.Nq == p0 / p.Nq) ? (p_max % p.Nq) : (p.Nq - 1);
-        const int last = i_max + p.Nkv - p.Nq;
-        n_tiles = min(p.n_kv_tiles, last / 128 + 1);
-    }
+        return min(p.n_kv_tiles, (i_max + p.Nkv - p.Nq) / 128 + 1);
+    };
+    const int n_tiles0 = kv_tiles_of(0);
+    const int n_tiles1 = kv_tiles_of(1);
+    const int n_tiles_max = max(n_tiles0, n_tiles1);
 
     // --------------------------------------------------------------- setup
     if (threadIdx.x == 0) {
@@ -181,33 +206,28 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&bars->v_full[s], 1);
             mbar_init(&bars->v_empty[s], 1);
         }
-        mbar_init(&bars->s_full, 1);
-        mbar_init(&bars->s_free, 256);
-        mbar_init(&bars->p_full[0], 256);
-        mbar_init(&bars->p_full[1], 256);
-        mbar_init(&bars->o_done, 1);
+        for (int qt = 0; qt < 2; ++qt) {
+            mbar_init(&bars->s_full[qt], 1);
+            mbar_init(&bars->s_free[qt], 128);
+            mbar_init(&bars->p_full[qt][0], 128);
+            mbar_init(&bars->p_full[qt][1], 128);
+            mbar_init(&bars->o_done[qt], 1);
+        }
         mbar_init(&bars->drain, 1);
-        mbar_init(&bars->mx[0], 256);
-        mbar_init(&bars->mx[1], 256);
-        mbar_init(&bars->lx, 256);
         *abort_flag = 0;
         fence_barrier_init();
     }
-    if (threadIdx.x < 128) {
-        const uint32_t i = threadIdx.x;
+    if (threadIdx.x >= 64 && threadIdx.x < 192) {
+        const uint32_t i = threadIdx.x - 64;
         lut[i] = (i == 0) ? 0.0f : __frcp_rn(e4m3_to_f32(i));
-    }
-    if (threadIdx.x >= 128 && threadIdx.x < 256) {
         // normalizer block of V^T (rows D..D+15 of every stage): one row of E2M1
         // ones (code 2 in both nibbles), 15 zero rows; and the scale atom of the
-        // ones row (row 0 of an atom = 1.0) for D >= 128.
-        const int i = threadIdx.x - 128;
+        // ones row (row 0 of an atom = 1.0) used when D >= 128.
         for (int s = 0; s < kStages; ++s) {
             uint32_t* row = reinterpret_cast<uint32_t*>(smem + C::OFF_V + s * C::V_STRIDE + D * 64);
             for (int k = i; k < 16 * 16; k += 128) row[k] = (k < 16) ? 0x22222222u : 0u;
         }
-        uint32_t* ones = reinterpret_cast<uint32_t*>(smem + C::OFF_ONES);
-        ones[i] = (i == 0) ? 0x38383838u : 0u;
+        reinterpret_cast<uint32_t*>(smem + C::OFF_ONES)[i] = (i == 0) ? 0x38383838u : 0u;
     }
     if (warp == 1) {
         tmem_alloc(tmem_slot, 512);
@@ -230,11 +250,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0 && !p.stall_loads) {
             int issued = 0;
             bool ok = true;
-            mbar_arrive_expect_tx(&bars->q_full, C::Q_BYTES + C::SFQK_BYTES);
-            tma_load_2d(smem + C::OFF_Q, &tmQ, 0, grp * rows_in_grp + p0, &bars->q_full);
-            bulk_load(smem + C::OFF_SFQ, p.qs + ((size_t)grp * p.Tq + t) * C::SFQK_BYTES, C::SFQK_BYTES,
-                      &bars->q_full);
-            for (int j = 0; j < n_tiles && ok; ++j) {
+            mbar_arrive_expect_tx(&bars->q_full, n_qt * (C::Q_BYTES + C::SFQK_BYTES));
+            for (int qt = 0; qt < n_qt; ++qt) {
+                tma_load_2d(smem + C::OFF_Q + qt * C::Q_BYTES, &tmQ, 0, grp * rows_in_grp + (t0 + qt) * 128,
+                            &bars->q_full);
+                bulk_load(smem + C::OFF_SFQ + qt * C::SFQK_BYTES,
+                          p.qs + ((size_t)grp * p.Tq + t0 + qt) * C::SFQK_BYTES, C::SFQK_BYTES, &bars->q_full);
+            }
+            for (int j = 0; j < n_tiles_max && ok; ++j) {
                 const int st = j % kStages;
                 const uint32_t ph = ((j / kStages) + 1) & 1;
                 if (j >= kStages && !mbar_wait(&bars->k_empty[st], ph, ctl)) { ok = false; break; }
@@ -263,243 +286,271 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ------------------------------------------------------- MMA issuer
         if (lane == 0) {
             const uint32_t idesc_s = idesc_fp4_block16(128);
-            auto qk_desc = [&](uint32_t base, int s) {
-                return smem_desc(smem_u32(smem + base) + 32u * s, 16u, C::QK_SBO, C::QK_SWZ);
-            };
             auto sf_desc = [&](uint32_t off) { return smem_desc(smem_u32(smem + off), 0u, 128u, 0u); };
             bool ok = mbar_wait(&bars->q_full, 0, ctl);
             if (ok) {
                 tc_fence_after();
+                for (int qt = 0; qt < n_qt; ++qt) {
 #pragma unroll
-                for (int s = 0; s < C::KS; ++s) tmem_cp_scale_atom(tmem + C::COL_SFQ + 4 * s, sf_desc(C::OFF_SFQ + 512 * s));
+                    for (int s = 0; s < C::KS; ++s)
+                        tmem_cp_scale_atom(tmem + C::COL_SFQ + qt * 4 * C::KS + 4 * s,
+                                           sf_desc(C::OFF_SFQ + qt * C::SFQK_BYTES + 512 * s));
+                }
                 if constexpr (PREORDER && D >= 128) {
 #pragma unroll
                     for (int s = 0; s < 2; ++s)
                         tmem_cp_scale_atom(tmem + C::COL_SFV + s * C::SFV_PER_KS + 4 * C::NRB, sf_desc(C::OFF_ONES));
                 }
             }
-            auto issue_pv = [&](int j) -> bool {
-                if (!mbar_wait(&bars->p_full[j & 1], (j >> 1) & 1, ctl)) return false;
+            int prev_qt = -1, prev_j = 0;     // the S MMA issued last
+            int sfv_j = -1;                    // V tile whose scales sit in TMEM
+            // S = Q_hat(qt) K_hat(j)^T into the shared S columns
+            auto issue_s = [&](int qt, int j, bool new_k) -> bool {
+                const int st = j % kStages;
+                if (new_k && !mbar_wait(&bars->k_full[st], (j / kStages) & 1, ctl)) return false;
+                if (prev_qt >= 0 && !mbar_wait(&bars->s_free[prev_qt], prev_j & 1, ctl)) return false;
+                tc_fence_after();
+                const uint32_t kbuf = C::OFF_K + st * C::K_BYTES;
+                if (new_k) {
+#pragma unroll
+                    for (int s = 0; s < C::KS; ++s)
+                        tmem_cp_scale_atom(tmem + C::COL_SFK + 4 * s, sf_desc(C::OFF_SFK + st * C::SFQK_BYTES + 512 * s));
+                }
+#pragma unroll
+                for (int s = 0; s < C::KS; ++s) {
+                    const uint64_t a = smem_desc(smem_u32(smem + C::OFF_Q + qt * C::Q_BYTES) + 32u * s, 16u, C::QK_SBO,
+                                                 C::QK_SWZ);
+                    const uint64_t b = smem_desc(smem_u32(smem + kbuf) + 32u * s, 16u, C::QK_SBO, C::QK_SWZ);
+                    mma_fp4_block16(tmem + C::COL_S, a, b, idesc_s, tmem + C::COL_SFQ + qt * 4 * C::KS + 4 * s,
+                                    tmem + C::COL_SFK + 4 * s, s > 0 ? 1u : 0u);
+                }
+                tc_commit(&bars->s_full[qt]);
+                prev_qt = qt;
+                prev_j = j;
+                return true;
+            };
+            // O(qt) += P_hat(qt, j) V_hat(j)
+            auto issue_pv = [&](int qt, int j) -> bool {
+                if (!mbar_wait(&bars->p_full[qt][j & 1], (j >> 1) & 1, ctl)) return false;
                 const int st = j % kStages;
                 if (!mbar_wait(&bars->v_full[st], (j / kStages) & 1, ctl)) return false;
                 tc_fence_after();
-                const uint32_t pbuf = C::OFF_P + (j & 1) * C::P_BYTES;
-                const uint32_t sfp = C::OFF_SFP + (j & 1) * C::SFP_BYTES;
+                const uint32_t pbuf = C::OFF_P + (qt * 2 + (j & 1)) * C::P_BYTES;
+                const uint32_t sfp = C::OFF_SFP + (qt * 2 + (j & 1)) * C::SFP_BYTES;
                 const uint32_t vbuf = C::OFF_V + st * C::V_STRIDE;
                 const uint32_t sfv = C::OFF_SFV + st * C::SFV_BYTES;
 #pragma unroll
                 for (int s = 0; s < 2; ++s) {
-                    tmem_cp_scale_atom(tmem + C::COL_SFP + 4 * s, sf_desc(sfp + 512 * s));
+                    tmem_cp_scale_atom(tmem + C::COL_SFP + qt * 8 + 4 * s, sf_desc(sfp + 512 * s));
+                    if (sfv_j != j) {
 #pragma unroll
-                    for (int rb = 0; rb < C::NRB; ++rb)
-                        tmem_cp_scale_atom(tmem + C::COL_SFV + s * C::SFV_PER_KS + 4 * rb, sf_desc(sfv + (rb * 2 + s) * 512));
+                        for (int rb = 0; rb < C::NRB; ++rb)
+                            tmem_cp_scale_atom(tmem + C::COL_SFV + s * C::SFV_PER_KS + 4 * rb,
+                                               sf_desc(sfv + (rb * 2 + s) * 512));
+                    }
                 }
+                sfv_j = j;
+                const uint32_t o = tmem + C::COL_O + qt * C::NO;
 #pragma unroll
                 for (int s = 0; s < 2; ++s) {
                     const uint64_t a = smem_desc(smem_u32(smem + pbuf) + 32u * s, 16u, 512u, 4u);
                     const uint32_t acc = (j > 0 || s > 0) ? 1u : 0u;
-                    const uint32_t sfa = tmem + C::COL_SFP + 4 * s;
+                    const uint32_t sfa = tmem + C::COL_SFP + qt * 8 + 4 * s;
                     const uint32_t sfb = tmem + C::COL_SFV + s * C::SFV_PER_KS;
                     if constexpr (D == 256 && PREORDER) {
                         const uint64_t b0 = smem_desc(smem_u32(smem + vbuf) + 32u * s, 16u, 512u, 4u);
                         const uint64_t b1 = smem_desc(smem_u32(smem + vbuf + 128 * 64) + 32u * s, 16u, 512u, 4u);
-                        mma_fp4_block16(tmem + C::COL_O, a, b0, idesc_fp4_block16(128), sfa, sfb, acc);
-                        mma_fp4_block16(tmem + C::COL_O + 128, a, b1, idesc_fp4_block16(144), sfa, sfb + 4, acc);
+                        mma_fp4_block16(o, a, b0, idesc_fp4_block16(128), sfa, sfb, acc);
+                        mma_fp4_block16(o + 128, a, b1, idesc_fp4_block16(144), sfa, sfb + 4, acc);
                     } else {
                         const uint64_t b = smem_desc(smem_u32(smem + vbuf) + 32u * s, 16u, 512u, 4u);
-                        mma_fp4_block16(tmem + C::COL_O, a, b, idesc_fp4_block16(C::NO), sfa, sfb, acc);
+                        mma_fp4_block16(o, a, b, idesc_fp4_block16(C::NO), sfa, sfb, acc);
                     }
                 }
-                tc_commit(&bars->o_done);
-                tc_commit(&bars->v_empty[st]);
+                tc_commit(&bars->o_done[qt]);
                 return true;
             };
-            for (int j = 0; j < n_tiles && ok; ++j) {
-                const int st = j % kStages;
-                if (!mbar_wait(&bars->k_full[st], (j / kStages) & 1, ctl)) { ok = false; break; }
-                if (j > 0 && !mbar_wait(&bars->s_free, (j - 1) & 1, ctl)) { ok = false; break; }
-                tc_fence_after();
-                const uint32_t kbuf = C::OFF_K + st * C::K_BYTES;
-                const uint32_t sfk = C::OFF_SFK + st * C::SFQK_BYTES;
-#pragma unroll
-                for (int s = 0; s < C::KS; ++s) tmem_cp_scale_atom(tmem + C::COL_SFK + 4 * s, sf_desc(sfk + 512 * s));
-#pragma unroll
-                for (int s = 0; s < C::KS; ++s)
-                    mma_fp4_block16(tmem + C::COL_S, qk_desc(C::OFF_Q, s), qk_desc(kbuf, s), idesc_s,
-                                    tmem + C::COL_SFQ + 4 * s, tmem + C::COL_SFK + 4 * s, s > 0 ? 1u : 0u);
-                tc_commit(&bars->s_full);
-                tc_commit(&bars->k_empty[st]);
-                if (j > 0 && !issue_pv(j - 1)) { ok = false; break; }
+            if (ok) {
+                ok = issue_s(0, 0, true);
+                if (ok && n_qt > 1) ok = issue_s(1, 0, false);
+                if (ok) tc_commit(&bars->k_empty[0]);
             }
-            if (ok && n_tiles > 0) issue_pv(n_tiles - 1);
+            for (int j = 0; j < n_tiles_max && ok; ++j) {
+                const bool a_next = j + 1 < n_tiles0;
+                const bool b_next = j + 1 < n_tiles1;
+                if (a_next && !issue_s(0, j + 1, true)) { ok = false; break; }
+                if (j < n_tiles0 && !issue_pv(0, j)) { ok = false; break; }
+                if (b_next && !issue_s(1, j + 1, !a_next)) { ok = false; break; }
+                if (a_next || b_next) tc_commit(&bars->k_empty[(j + 1) % kStages]);
+                if (j < n_tiles1 && !issue_pv(1, j)) { ok = false; break; }
+                tc_commit(&bars->v_empty[j % kStages]);
+            }
             // wait until every MMA / copy issued above has finished
             tc_commit(&bars->drain);
             mbar_wait_drain(&bars->drain, 0, p.wait_limit_ns);
         }
-    } else if (warp >= kSoftmaxWarp0) {
+    } else {
         // ------------------------------------------------------------ softmax
-        const int wg = (warp - kSoftmaxWarp0) >> 2;        // key half of every tile
+        const int qt = (warp - kSmWarp0) >> 2;             // query tile of this warpgroup
         const int wq = warp & 3;                           // TMEM lane quarter
         const int row = wq * 32 + lane;
         const uint32_t tl = tmem + ((uint32_t)(wq * 32) << 16);
-        const int prow = p0 + row;
-        const bool valid = prow < rows_in_grp;
+        const uint32_t tO = tl + C::COL_O + qt * C::NO;
+        const int prow = (t0 + qt) * 128 + row;
+        const bool valid = qt < n_qt && prow < rows_in_grp;
         const int qi = prow % p.Nq;
         const int last = valid ? (CAUSAL ? qi + p.Nkv - p.Nq : p.Nkv - 1) : -1;
         const size_t out_row = (size_t)grp * rows_in_grp + prow;
+        const int nt = qt == 0 ? n_tiles0 : n_tiles1;
         const float c = p.c;
+        const uint64_t c2 = pack2(c, c);
         const float one_sixth = rn_one_sixth();
         float m_old = -INFINITY, mc_old = 0.0f, l_hp = 0.0f;
         bool ok = true;
-        for (int j = 0; j < n_tiles; ++j) {
-            if (!__all_sync(0xFFFFFFFFu, mbar_wait(&bars->s_full, j & 1, ctl))) { ok = false; break; }
+        for (int j = 0; j < nt; ++j) {
+            if (!__all_sync(0xFFFFFFFFu, mbar_wait(&bars->s_full[qt], j & 1, ctl))) { ok = false; break; }
             tc_fence_after();
-            float S[64];
+            float S[128];
             {
-                uint32_t r0[32], r1[32];
-                tmem_ld32(tl + C::COL_S + wg * 64, r0);
-                tmem_ld32(tl + C::COL_S + wg * 64 + 32, r1);
-                tmem_wait_ld();
+                uint32_t r[32];
 #pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    S[e] = __uint_as_float(r0[e]);
-                    S[32 + e] = __uint_as_float(r1[e]);
+                for (int q4 = 0; q4 < 4; ++q4) {
+                    tmem_ld32(tl + C::COL_S + 32 * q4, r);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) S[32 * q4 + e] = __uint_as_float(r[e]);
                 }
             }
             tc_fence_before();
-            mbar_arrive(&bars->s_free);
-            const int n0 = j * 128 + wg * 64;
-            if (n0 + 63 > last) {
+            mbar_arrive(&bars->s_free[qt]);
+            const int n0 = j * 128;
+            if (n0 + 127 > last) {
 #pragma unroll
-                for (int e = 0; e < 64; ++e)
+                for (int e = 0; e < 128; ++e)
                     if (n0 + e > last) S[e] = -INFINITY;
             }
-            float mx = S[0];
-#pragma unroll
-            for (int e = 1; e < 64; ++e) mx = fmaxf(mx, S[e]);
-            // exchange the partial row maxima of the two key halves
-            {
-                float* xb = mx_x + (j & 1) * 256;
-                xb[wg * 128 + row] = mx;
-                mbar_arrive(&bars->mx[j & 1]);
-                if (!__all_sync(0xFFFFFFFFu, mbar_wait(&bars->mx[j & 1], (j >> 1) & 1, ctl))) { ok = false; break; }
-                mx = fmaxf(xb[row], xb[128 + row]);
-            }
-            const float m_new = fmaxf(m_old, mx);
+            const float m_new = fmaxf(m_old, row_max128(S));
             const float mc_new = (m_new == -INFINITY) ? 0.0f : __fmul_rn(m_new, c);
             const float alpha = (m_old == -INFINITY) ? 0.0f : ex2_approx(mc_old - mc_new);
-            float psum = 0.0f;
+            const uint64_t nmc2 = pack2(-mc_new, -mc_new);
+            // P = 2^(S*c - mc), then 8 blocks of 16 keys to E2M1 codes + E4M3 scales
+            uint32_t code[16];
+            uint32_t sfw[2] = {0u, 0u};
+            uint64_t lsum2 = 0;
 #pragma unroll
-            for (int e = 0; e < 64; ++e) {
-                S[e] = ex2_approx(__fmaf_rn(S[e], c, -mc_new));
-                if constexpr (!PREORDER) psum += S[e];
-            }
-            if constexpr (!PREORDER) l_hp = __fmaf_rn(alpha, l_hp, psum);
-            // quantize P: 4 blocks of 16 keys
-            uint32_t code[8];
-            uint32_t sfw = 0;
+            for (int blk = 0; blk < 8; ++blk) {
+                float* P = S + 16 * blk;
 #pragma unroll
-            for (int blk = 0; blk < 4; ++blk) {
-                float amax = S[16 * blk];
+                for (int e = 0; e < 16; e += 2) {
+                    float t0f, t1f;
+                    unpack2(ffma2(pack2(P[e], P[e + 1]), c2, nmc2), t0f, t1f);
+                    P[e] = ex2_approx(t0f);
+                    P[e + 1] = ex2_approx(t1f);
+                }
+                if constexpr (!PREORDER) {
 #pragma unroll
-                for (int e = 1; e < 16; ++e) amax = fmaxf(amax, S[16 * blk + e]);
-                const uint32_t sf = cvt_e4m3(__fmul_rn(amax, one_sixth));
+                    for (int e = 0; e < 16; e += 2) lsum2 = fadd2(lsum2, pack2(P[e], P[e + 1]));
+                }
+                const uint32_t sf = cvt_e4m3(__fmul_rn(block_max16(P), one_sixth));
                 const float r = lut[sf & 127u];
+                const uint64_t r2 = pack2(r, r);
                 float y[16];
 #pragma unroll
-                for (int e = 0; e < 16; ++e) y[e] = __fmul_rn(S[16 * blk + e], r);
+                for (int e = 0; e < 16; e += 2) unpack2(fmul2(pack2(P[e], P[e + 1]), r2), y[e], y[e + 1]);
                 code[2 * blk] = cvt_e2m1x8(y[0], y[1], y[2], y[3], y[4], y[5], y[6], y[7]);
                 code[2 * blk + 1] = cvt_e2m1x8(y[8], y[9], y[10], y[11], y[12], y[13], y[14], y[15]);
-                sfw |= sf << (8 * blk);
+                sfw[blk >> 2] |= sf << (8 * (blk & 3));
+            }
+            if constexpr (!PREORDER) {
+                float la, lb;
+                unpack2(lsum2, la, lb);
+                l_hp = __fmaf_rn(alpha, l_hp, la + lb);
             }
             if constexpr (DUMP) {
                 if (valid) {
                     uint4* dc = reinterpret_cast<uint4*>(p.p_codes + out_row * (size_t)(p.Nkv / 2) + n0 / 2);
-                    dc[0] = make_uint4(code[0], code[1], code[2], code[3]);
-                    dc[1] = make_uint4(code[4], code[5], code[6], code[7]);
-                    *reinterpret_cast<uint32_t*>(p.p_sf + out_row * (size_t)(p.Nkv / 16) + n0 / 16) = sfw;
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4)
+                        dc[q4] = make_uint4(code[4 * q4], code[4 * q4 + 1], code[4 * q4 + 2], code[4 * q4 + 3]);
+                    *reinterpret_cast<uint2*>(p.p_sf + out_row * (size_t)(p.Nkv / 16) + n0 / 16) =
+                        make_uint2(sfw[0], sfw[1]);
                 }
             }
             if (j > 0) {
                 // PV of the previous tile is done: O is stable, P buffer j&1 is free
-                if (!__all_sync(0xFFFFFFFFu, mbar_wait(&bars->o_done, (j - 1) & 1, ctl))) { ok = false; break; }
+                if (!__all_sync(0xFFFFFFFFu, mbar_wait(&bars->o_done[qt], (j - 1) & 1, ctl))) { ok = false; break; }
                 tc_fence_after();
                 if (__any_sync(0xFFFFFFFFu, alpha != 1.0f)) {
-                    constexpr int HALF = D / 2;
+                    const uint64_t a2 = pack2(alpha, alpha);
 #pragma unroll 1
-                    for (int cc = wg * HALF; cc < (wg + 1) * HALF; cc += 32) {
+                    for (int cc = 0; cc < D; cc += 32) {
                         uint32_t o[32];
-                        tmem_ld32(tl + C::COL_O + cc, o);
+                        tmem_ld32(tO + cc, o);
                         tmem_wait_ld();
 #pragma unroll
-                        for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__fmul_rn(__uint_as_float(o[e]), alpha));
-                        tmem_st32(tl + C::COL_O + cc, o);
+                        for (int e = 0; e < 32; e += 2) {
+                            float x0, x1;
+                            unpack2(fmul2(pack2(__uint_as_float(o[e]), __uint_as_float(o[e + 1])), a2), x0, x1);
+                            o[e] = __float_as_uint(x0);
+                            o[e + 1] = __float_as_uint(x1);
+                        }
+                        tmem_st32(tO + cc, o);
                     }
                     if constexpr (PREORDER) {
-                        if (wg == 1) {
-                            uint32_t lv;
-                            tmem_ld1(tl + C::COL_O + D, lv);
-                            tmem_wait_ld();
-                            lv = __float_as_uint(__fmul_rn(__uint_as_float(lv), alpha));
-                            asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(tl + C::COL_O + D),
-                                         "r"(lv)
-                                         : "memory");
-                        }
+                        uint32_t lv;
+                        tmem_ld1(tO + D, lv);
+                        tmem_wait_ld();
+                        tmem_st1(tO + D, __float_as_uint(__fmul_rn(__uint_as_float(lv), alpha)));
                     }
                     tmem_wait_st();
                 }
             }
             {
-                uint8_t* pb = smem + C::OFF_P + (j & 1) * C::P_BYTES;
-                *reinterpret_cast<uint4*>(pb + p_swizzle64(row, 2 * wg)) = make_uint4(code[0], code[1], code[2], code[3]);
-                *reinterpret_cast<uint4*>(pb + p_swizzle64(row, 2 * wg + 1)) = make_uint4(code[4], code[5], code[6], code[7]);
-                *reinterpret_cast<uint32_t*>(smem + C::OFF_SFP + (j & 1) * C::SFP_BYTES + wg * 512 +
-                                             16 * (row & 31) + 4 * (row >> 5)) = sfw;
+                uint8_t* pb = smem + C::OFF_P + (qt * 2 + (j & 1)) * C::P_BYTES;
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4)
+                    *reinterpret_cast<uint4*>(pb + p_swizzle64(row, q4)) =
+                        make_uint4(code[4 * q4], code[4 * q4 + 1], code[4 * q4 + 2], code[4 * q4 + 3]);
+                uint8_t* sb = smem + C::OFF_SFP + (qt * 2 + (j & 1)) * C::SFP_BYTES + 16 * (row & 31) + 4 * (row >> 5);
+                *reinterpret_cast<uint32_t*>(sb) = sfw[0];
+                *reinterpret_cast<uint32_t*>(sb + 512) = sfw[1];
             }
             fence_proxy_async_smem();
             tc_fence_before();
-            mbar_arrive(&bars->p_full[j & 1]);
+            mbar_arrive(&bars->p_full[qt][j & 1]);
             m_old = m_new;
             mc_old = mc_new;
         }
         // ---------------------------------------------------------- epilogue
-        if (ok && n_tiles > 0) ok = __all_sync(0xFFFFFFFFu, mbar_wait(&bars->o_done, (n_tiles - 1) & 1, ctl));
-        if (ok) {
+        if (ok && nt > 0) ok = __all_sync(0xFFFFFFFFu, mbar_wait(&bars->o_done[qt], (nt - 1) & 1, ctl));
+        if (ok && nt > 0) {
             tc_fence_after();
             float l;
             if constexpr (PREORDER) {
                 uint32_t lv;
-                tmem_ld1(tl + C::COL_O + D, lv);
+                tmem_ld1(tO + D, lv);
                 tmem_wait_ld();
                 l = __uint_as_float(lv);
             } else {
-                float* lx = mx_x;                       // reuse: the row-max buffers are idle now
-                lx[wg * 128 + row] = l_hp;
-                mbar_arrive(&bars->lx);
-                ok = __all_sync(0xFFFFFFFFu, mbar_wait(&bars->lx, 0, ctl));
-                l = lx[row] + lx[128 + row];
+                l = l_hp;
             }
-            if (ok) {
-                const float inv = l > 0.0f ? __frcp_rn(l) : 0.0f;
-                constexpr int HALF = D / 2;
+            const float inv = l > 0.0f ? __frcp_rn(l) : 0.0f;
 #pragma unroll 1
-                for (int cc = wg * HALF; cc < (wg + 1) * HALF; cc += 32) {
-                    uint32_t o[32];
-                    tmem_ld32(tl + C::COL_O + cc, o);
-                    tmem_wait_ld();
-                    float v[32];
+            for (int cc = 0; cc < D; cc += 32) {
+                uint32_t o[32];
+                tmem_ld32(tO + cc, o);
+                tmem_wait_ld();
+                float v[32];
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) v[e] = __uint_as_float(o[e]) * inv;
-                    if (valid) {
-                        uint8_t* dst = reinterpret_cast<uint8_t*>(p.o) + (out_row * D + cc) * (OUT == 2 ? 4 : 2);
-                        store_out32<OUT>(dst, v);
-                    }
+                for (int e = 0; e < 32; ++e) v[e] = __uint_as_float(o[e]) * inv;
+                if (valid) {
+                    uint8_t* dst = reinterpret_cast<uint8_t*>(p.o) + (out_row * D + cc) * (OUT == 2 ? 4 : 2);
+                    store_out32<OUT>(dst, v);
                 }
-                if (wg == 0 && valid && p.lse != nullptr)
-                    p.lse[out_row] = l > 0.0f ? mc_old * 0.69314718055994531f + __logf(l) : -INFINITY;
             }
+            if (valid && p.lse != nullptr)
+                p.lse[out_row] = l > 0.0f ? mc_old * 0.69314718055994531f + __logf(l) : -INFINITY;
         }
-        (void)ok;
     }
     // ---------------------------------------------------------------- teardown
     tc_fence_before();
@@ -515,7 +566,7 @@ static cudaError_t launch_one(const CUtensorMap* q, const CUtensorMap* k, const 
     auto kern = attn_fwd_kernel<D, PRE, CAUSAL, OUT, DUMP>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    kern<<<p.n_work, kThreads, C::SMEM_BYTES, st>>>(*q, *k, *v, p);
+    kern<<<p.n_work, C::THREADS, C::SMEM_BYTES, st>>>(*q, *k, *v, p);
     return cudaGetLastError();
 }
 
