@@ -14,7 +14,8 @@ CAUSAL = 1
 
 EXPORTS = ["hifa4_packed_bytes", "hifa4_workspace_bytes", "hifa4_calibrate_smooth", "hifa4_quantize_qkv",
            "hifa4_quantize_kv", "hifa4_attention_fwd", "hifa4_attention_fwd_debug", "hifa4_get_status",
-           "hifa4_debug_set_wait_limit", "hifa4_status_string", "hifa4_version", "hifa4_attention_fwd_noalloc"]
+           "hifa4_debug_set_wait_limit", "hifa4_status_string", "hifa4_version", "hifa4_attention_fwd_noalloc",
+           "hifa4_last_cuda_error"]
 
 
 class Packed(ctypes.Structure):
@@ -24,7 +25,8 @@ class Packed(ctypes.Structure):
 class HiFA4Error(RuntimeError):
     def __init__(self, status: int, what: str):
         self.status = status
-        super().__init__(f"{what}: {status_string(status)} (status {status})")
+        detail = f" [{load().hifa4_last_cuda_error().decode()}]" if status == ERR_CUDA else ""
+        super().__init__(f"{what}: {status_string(status)} (status {status}){detail}")
 
 
 _lib = None
@@ -62,6 +64,8 @@ def load():
     L.hifa4_debug_set_wait_limit.restype = ctypes.c_longlong
     L.hifa4_status_string.argtypes = [ci]
     L.hifa4_status_string.restype = ctypes.c_char_p
+    L.hifa4_last_cuda_error.argtypes = []
+    L.hifa4_last_cuda_error.restype = ctypes.c_char_p
     L.hifa4_version.argtypes = []
     L.hifa4_version.restype = ci
     _lib = L

@@ -77,7 +77,13 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t inner_bytes, uint64_t r
     return r == CUDA_SUCCESS;
 }
 
-hifa4_status from_cuda(cudaError_t e) { return e == cudaSuccess ? HIFA4_OK : HIFA4_ERR_CUDA; }
+thread_local cudaError_t g_last_cuda_error = cudaSuccess;
+
+hifa4_status from_cuda(cudaError_t e) {
+    if (e == cudaSuccess) return HIFA4_OK;
+    g_last_cuda_error = e;
+    return HIFA4_ERR_CUDA;
+}
 
 hifa4_status attention_impl(const hifa4_packed* in, int B, int Hq, int Hkv, int Nq, int Nkv, int D, float sm_scale,
                             unsigned flags, hifa4_norm_mode norm, void* o, hifa4_dtype o_dtype, float* lse,
@@ -107,10 +113,10 @@ hifa4_status attention_impl(const hifa4_packed* in, int B, int Hq, int Hkv, int 
     const CUtensorMapSwizzle swz_qk =
         D == 64 ? CU_TENSOR_MAP_SWIZZLE_32B : (D == 128 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B);
     CUtensorMap tq, tk, tv;
-    if (!make_map(&tq, in->qc, (uint64_t)D / 2, (uint64_t)rows_q, D / 2, 128, swz_qk)) return HIFA4_ERR_CUDA;
-    if (!make_map(&tk, in->kc, (uint64_t)D / 2, (uint64_t)rows_k, D / 2, 128, swz_qk)) return HIFA4_ERR_CUDA;
-    if (!make_map(&tv, in->vtc, (uint64_t)Nkv / 2, (uint64_t)rows_v, 64, (uint32_t)D, CU_TENSOR_MAP_SWIZZLE_64B))
-        return HIFA4_ERR_CUDA;
+    if (!make_map(&tq, in->qc, (uint64_t)D / 2, (uint64_t)rows_q, D / 2, 128, swz_qk) ||
+        !make_map(&tk, in->kc, (uint64_t)D / 2, (uint64_t)rows_k, D / 2, 128, swz_qk) ||
+        !make_map(&tv, in->vtc, (uint64_t)Nkv / 2, (uint64_t)rows_v, 64, (uint32_t)D, CU_TENSOR_MAP_SWIZZLE_64B))
+        return from_cuda(cudaErrorInvalidValue);
 
     AttnParams p{};
     p.qs = static_cast<const uint8_t*>(in->qs);
@@ -190,8 +196,8 @@ hifa4_status hifa4_quantize_kv(const void* k, const void* v, hifa4_dtype dtype, 
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     const long long n_grp = (long long)B * Hkv;
     cudaError_t e = launch_quantize_rows(bf, k, s_inv, static_cast<uint8_t*>(out->kc), static_cast<uint8_t*>(out->ks),
-                                         n_grp, Nkv, Nkv / 128, 1, Hkv, Nkv, D, st);
-    if (e != cudaSuccess) return HIFA4_ERR_CUDA;
+                                         n_grp, Nkv, Nkv / 128, Hkv, D, st);
+    if (e != cudaSuccess) return from_cuda(e);
     e = launch_quantize_v(bf, v, static_cast<uint8_t*>(out->vtc), static_cast<uint8_t*>(out->vts), n_grp, Nkv, D, st);
     return from_cuda(e);
 }
@@ -211,8 +217,8 @@ hifa4_status hifa4_quantize_qkv(const void* q, const void* k, const void* v, hif
     const long long n_grp = (long long)B * Hkv;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     cudaError_t e = launch_quantize_rows(dtype == HIFA4_BF16, q, s, static_cast<uint8_t*>(out->qc),
-                                         static_cast<uint8_t*>(out->qs), n_grp, G * Nq, sz.Tq, G, Hkv, Nq, D, st);
-    if (e != cudaSuccess) return HIFA4_ERR_CUDA;
+                                         static_cast<uint8_t*>(out->qs), n_grp, G * Nq, sz.Tq, Hkv, D, st);
+    if (e != cudaSuccess) return from_cuda(e);
     return hifa4_quantize_kv(k, v, dtype, B, Hkv, Nkv, D, s_inv, out, stream);
 }
 
@@ -234,10 +240,11 @@ hifa4_status hifa4_attention_fwd_debug(const hifa4_packed* in, int B, int Hq, in
 hifa4_status hifa4_get_status(void* workspace, hifa4_stream_t stream) {
     if (workspace == nullptr) return HIFA4_ERR_INVALID_ARG;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    if (cudaStreamSynchronize(st) != cudaSuccess) return HIFA4_ERR_CUDA;
+    if (from_cuda(cudaStreamSynchronize(st)) != HIFA4_OK) return HIFA4_ERR_CUDA;
     uint32_t word = 0;
-    if (cudaMemcpy(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess) return HIFA4_ERR_CUDA;
-    if (word != 0 && cudaMemset(workspace, 0, sizeof(word)) != cudaSuccess) return HIFA4_ERR_CUDA;
+    if (from_cuda(cudaMemcpy(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost)) != HIFA4_OK)
+        return HIFA4_ERR_CUDA;
+    if (word != 0 && from_cuda(cudaMemset(workspace, 0, sizeof(word))) != HIFA4_OK) return HIFA4_ERR_CUDA;
     return word == 0 ? HIFA4_OK : (hifa4_status)word;
 }
 
@@ -246,6 +253,8 @@ long long hifa4_debug_set_wait_limit(long long limit_ns, int stall_loads) {
     const long long prev = g_wait_limit_ns.exchange(limit_ns > 0 ? limit_ns : 0);
     return prev > 0 ? prev : (long long)kDefaultWaitNs;
 }
+
+const char* hifa4_last_cuda_error(void) { return cudaGetErrorString(g_last_cuda_error); }
 
 const char* hifa4_status_string(hifa4_status s) {
     switch (s) {

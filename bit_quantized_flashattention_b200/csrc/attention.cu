@@ -5,24 +5,27 @@
 // P-Reordering the softmax normalizer is accumulated from the same quantized
 // probabilities P_hat that feed the PV GEMM, fused into that GEMM.
 //
-// One CTA computes one 128-row query tile of one (batch, kv head) group. The
-// tile's rows are the group's query rows stacked head after head (GQA), so a
-// tile may mix heads when Nq is small. Warp roles:
-//   warp 0      TMA / bulk-copy producer: Q_hat tile once, then K_hat and V_hat^T
-//               tiles (128 keys) with their scale atoms through 3-stage rings
-//   warp 1      TMEM owner and MMA issuer (one thread): scale atoms shared->TMEM
-//               with tcgen05.cp, S = Q_hat K_hat^T into TMEM, then O += P_hat V_hat
-//   warps 4-11  two softmax warpgroups; warpgroup w owns keys 64w..64w+63 of
-//               every tile, thread t of a warpgroup owns row t. Per tile: load S
-//               from TMEM, causal mask, running max (exchanged between the two
-//               warpgroups), P = 2^(S*c - RN(m*c)), quantize P per 16 keys to
-//               E2M1 + E4M3 in registers, rescale O in TMEM when the max moved,
-//               write P_hat codes and scales to shared memory for the PV MMA.
+// One CTA computes NQT 128-row query tiles (2 for D <= 128, 1 for D = 256) of
+// one (batch, kv head) group. A tile's rows are the group's query rows stacked
+// head after head (GQA), so a tile may mix heads when Nq is small. Warp roles:
+//   warp 0      TMA / bulk-copy producer: Q_hat tiles once, then K_hat and
+//               V_hat^T tiles (128 keys) with their scale atoms, 3-stage rings
+//   warp 1      TMEM owner; one thread issues S = Q_hat K_hat^T (and moves the
+//               Q and K scale atoms shared->TMEM with tcgen05.cp)
+//   warp 2      one thread issues O += P_hat V_hat (P and V scale atoms); the
+//               two issuers touch disjoint TMEM and wait independently
+//   warps 4..   one softmax warpgroup per query tile, thread t owns row t:
+//               block maxima of S, running max, P = 2^(S*c - RN(m*c)),
+//               P quantized per 16 keys to E2M1 + E4M3 in registers, O rescaled
+//               in TMEM when some row's max moved,
+//               P_hat codes and scales written to shared memory for the PV MMA.
+// The query tiles take turns in one 128-column S buffer in TMEM; each warpgroup
+// releases it right after loading its scores.
 // With P-Reordering the V tile carries 16 extra rows: a row of E2M1 ones
 // (scale 1.0) and 15 zero rows, so the PV MMA also produces sum(P_hat) in
 // output column D: the normalizer from exactly the codes x scales the MMA used.
-// TMEM (512 columns): S [0,128), O [128,128+NO) with NO = D (+16), then the
-// scale-factor regions of Q, K, P and V.
+// TMEM (512 columns): S [0,128), O tiles [128, 128 + NQT*NO), NO = D (+16),
+// then the scale-factor regions of Q, K, P and V.
 // Every mbarrier wait is bounded; when one gives up the CTA records
 // HIFA4_ERR_TIMEOUT in the workspace, drains its copies and MMAs, frees TMEM
 // and exits.
@@ -35,12 +38,12 @@
 namespace hifa4 {
 
 constexpr int kStages = 3;
-constexpr int kSmWarp0 = 2;          // first softmax warp
+constexpr int kSmWarp0 = 4;          // first softmax warp (0: loads, 1: S MMAs, 2: PV MMAs, 3: idle)
 
 template <int D, bool PREORDER>
 struct Cfg {
     static constexpr int NQT = D == 256 ? 1 : 2;          // 128-row query tiles per CTA
-    static constexpr int THREADS = 64 + 128 * NQT;
+    static constexpr int THREADS = 128 + 128 * NQT;
     static constexpr int KS = D / 64;                     // 64-wide K steps of QK^T
     static constexpr int QK_ROW = D / 2;                  // bytes per Q/K row
     static constexpr uint32_t QK_SWZ = D == 64 ? 6u : (D == 128 ? 4u : 2u);   // 32B/64B/128B swizzle
@@ -57,6 +60,7 @@ struct Cfg {
     static constexpr int P_BYTES = 128 * 64;
     static constexpr int SFP_BYTES = 2 * 512;
     static constexpr int NO = PREORDER ? D + 16 : D;      // accumulator columns per query tile
+    static constexpr int NCH = D / 32;                    // 32-column chunks of O
     // TMEM columns
     static constexpr uint32_t COL_S = 0;
     static constexpr uint32_t COL_O = 128;                                // + qt * NO
@@ -94,7 +98,7 @@ struct Bars {
     uint64_t s_free[2];      // its warpgroup has read it (the S columns are free again)
     uint64_t p_full[2][2];   // P_hat buffer (qt, j & 1) ready and O of qt rescaled
     uint64_t o_done[2];      // PV MMA of query tile qt finished
-    uint64_t drain;          // teardown of the MMA issuer
+    uint64_t drain[2];       // teardown of the two MMA issuers
 };
 static_assert(sizeof(Bars) <= 256, "barrier area");
 
@@ -126,27 +130,22 @@ __device__ __forceinline__ void store_out32(void* dst, const float (&v)[32]) {
     }
 }
 
-// Row maximum of 128 values: a three-input max tree (64 instructions, depth 5).
-__device__ __forceinline__ float row_max128(const float (&v)[128]) {
-    float a[43];
-#pragma unroll
-    for (int i = 0; i < 42; ++i) a[i] = fmax3f(v[3 * i], v[3 * i + 1], v[3 * i + 2]);
-    a[42] = fmaxf(v[126], v[127]);
-    float b[15];
-#pragma unroll
-    for (int i = 0; i < 14; ++i) b[i] = fmax3f(a[3 * i], a[3 * i + 1], a[3 * i + 2]);
-    b[14] = a[42];
-    float c[5];
-#pragma unroll
-    for (int i = 0; i < 5; ++i) c[i] = fmax3f(b[3 * i], b[3 * i + 1], b[3 * i + 2]);
-    return fmax3f(fmax3f(c[0], c[1], c[2]), c[3], c[4]);
+// Maximum of 16 values held as 8 pairs (three-input max, depth 3).
+__device__ __forceinline__ float max16(const float2* v) {
+    const float a0 = fmax3f(v[0].x, v[0].y, v[1].x), a1 = fmax3f(v[1].y, v[2].x, v[2].y);
+    const float a2 = fmax3f(v[3].x, v[3].y, v[4].x), a3 = fmax3f(v[4].y, v[5].x, v[5].y);
+    const float a4 = fmax3f(v[6].x, v[6].y, v[7].x);
+    return fmax3f(fmax3f(a0, a1, a2), fmax3f(a3, a4, v[7].y), -INFINITY);
 }
 
-// Maximum of 16 non-negative values (8 instructions, depth 3).
-__device__ __forceinline__ float block_max16(const float* v) {
-    const float a0 = fmax3f(v[0], v[1], v[2]), a1 = fmax3f(v[3], v[4], v[5]), a2 = fmax3f(v[6], v[7], v[8]);
-    const float a3 = fmax3f(v[9], v[10], v[11]), a4 = fmax3f(v[12], v[13], v[14]);
-    return fmax3f(fmax3f(a0, a1, a2), fmax3f(a3, a4, v[15]), 0.0f);
+// 32 O values (already loaded from TMEM) times alpha, in place.
+__device__ __forceinline__ void scale_chunk(uint32_t (&o)[32], float2 a2) {
+#pragma unroll
+    for (int e = 0; e < 32; e += 2) {
+        const float2 x = __fmul2_rn(make_float2(__uint_as_float(o[e]), __uint_as_float(o[e + 1])), a2);
+        o[e] = __float_as_uint(x.x);
+        o[e + 1] = __float_as_uint(x.y);
+    }
 }
 
 template <int D, bool PREORDER, bool CAUSAL, int OUT, bool DUMP>
@@ -213,12 +212,13 @@ __global__ void __launch_bounds__(Cfg<D, PREORDER>::THREADS, 1)
             mbar_init(&bars->p_full[qt][1], 128);
             mbar_init(&bars->o_done[qt], 1);
         }
-        mbar_init(&bars->drain, 1);
+        mbar_init(&bars->drain[0], 1);
+        mbar_init(&bars->drain[1], 1);
         *abort_flag = 0;
         fence_barrier_init();
     }
-    if (threadIdx.x >= 64 && threadIdx.x < 192) {
-        const uint32_t i = threadIdx.x - 64;
+    if (threadIdx.x >= 128 && threadIdx.x < 256) {
+        const uint32_t i = threadIdx.x - 128;
         lut[i] = (i == 0) ? 0.0f : __frcp_rn(e4m3_to_f32(i));
         // normalizer block of V^T (rows D..D+15 of every stage): one row of E2M1
         // ones (code 2 in both nibbles), 15 zero rows; and the scale atom of the
@@ -283,7 +283,9 @@ __global__ void __launch_bounds__(Cfg<D, PREORDER>::THREADS, 1)
             }
         }
     } else if (warp == 1) {
-        // ------------------------------------------------------- MMA issuer
+        // ----------------------------------------------------- S MMA issuer
+        // S = Q_hat(qt) K_hat(j)^T in the order (j=0,A) (0,B) (1,A) (1,B) ... through
+        // the one S buffer; each needs its K tile and the previous S consumed.
         if (lane == 0) {
             const uint32_t idesc_s = idesc_fp4_block16(128);
             auto sf_desc = [&](uint32_t off) { return smem_desc(smem_u32(smem + off), 0u, 128u, 0u); };
@@ -296,100 +298,103 @@ __global__ void __launch_bounds__(Cfg<D, PREORDER>::THREADS, 1)
                         tmem_cp_scale_atom(tmem + C::COL_SFQ + qt * 4 * C::KS + 4 * s,
                                            sf_desc(C::OFF_SFQ + qt * C::SFQK_BYTES + 512 * s));
                 }
-                if constexpr (PREORDER && D >= 128) {
-#pragma unroll
-                    for (int s = 0; s < 2; ++s)
-                        tmem_cp_scale_atom(tmem + C::COL_SFV + s * C::SFV_PER_KS + 4 * C::NRB, sf_desc(C::OFF_ONES));
-                }
             }
-            int prev_qt = -1, prev_j = 0;     // the S MMA issued last
-            int sfv_j = -1;                    // V tile whose scales sit in TMEM
-            // S = Q_hat(qt) K_hat(j)^T into the shared S columns
-            auto issue_s = [&](int qt, int j, bool new_k) -> bool {
-                const int st = j % kStages;
-                if (new_k && !mbar_wait(&bars->k_full[st], (j / kStages) & 1, ctl)) return false;
-                if (prev_qt >= 0 && !mbar_wait(&bars->s_free[prev_qt], prev_j & 1, ctl)) return false;
-                tc_fence_after();
-                const uint32_t kbuf = C::OFF_K + st * C::K_BYTES;
-                if (new_k) {
-#pragma unroll
-                    for (int s = 0; s < C::KS; ++s)
-                        tmem_cp_scale_atom(tmem + C::COL_SFK + 4 * s, sf_desc(C::OFF_SFK + st * C::SFQK_BYTES + 512 * s));
-                }
-#pragma unroll
-                for (int s = 0; s < C::KS; ++s) {
-                    const uint64_t a = smem_desc(smem_u32(smem + C::OFF_Q + qt * C::Q_BYTES) + 32u * s, 16u, C::QK_SBO,
-                                                 C::QK_SWZ);
-                    const uint64_t b = smem_desc(smem_u32(smem + kbuf) + 32u * s, 16u, C::QK_SBO, C::QK_SWZ);
-                    mma_fp4_block16(tmem + C::COL_S, a, b, idesc_s, tmem + C::COL_SFQ + qt * 4 * C::KS + 4 * s,
-                                    tmem + C::COL_SFK + 4 * s, s > 0 ? 1u : 0u);
-                }
-                tc_commit(&bars->s_full[qt]);
-                prev_qt = qt;
-                prev_j = j;
-                return true;
-            };
-            // O(qt) += P_hat(qt, j) V_hat(j)
-            auto issue_pv = [&](int qt, int j) -> bool {
-                if (!mbar_wait(&bars->p_full[qt][j & 1], (j >> 1) & 1, ctl)) return false;
-                const int st = j % kStages;
-                if (!mbar_wait(&bars->v_full[st], (j / kStages) & 1, ctl)) return false;
-                tc_fence_after();
-                const uint32_t pbuf = C::OFF_P + (qt * 2 + (j & 1)) * C::P_BYTES;
-                const uint32_t sfp = C::OFF_SFP + (qt * 2 + (j & 1)) * C::SFP_BYTES;
-                const uint32_t vbuf = C::OFF_V + st * C::V_STRIDE;
-                const uint32_t sfv = C::OFF_SFV + st * C::SFV_BYTES;
-#pragma unroll
-                for (int s = 0; s < 2; ++s) {
-                    tmem_cp_scale_atom(tmem + C::COL_SFP + qt * 8 + 4 * s, sf_desc(sfp + 512 * s));
-                    if (sfv_j != j) {
-#pragma unroll
-                        for (int rb = 0; rb < C::NRB; ++rb)
-                            tmem_cp_scale_atom(tmem + C::COL_SFV + s * C::SFV_PER_KS + 4 * rb,
-                                               sf_desc(sfv + (rb * 2 + s) * 512));
-                    }
-                }
-                sfv_j = j;
-                const uint32_t o = tmem + C::COL_O + qt * C::NO;
-#pragma unroll
-                for (int s = 0; s < 2; ++s) {
-                    const uint64_t a = smem_desc(smem_u32(smem + pbuf) + 32u * s, 16u, 512u, 4u);
-                    const uint32_t acc = (j > 0 || s > 0) ? 1u : 0u;
-                    const uint32_t sfa = tmem + C::COL_SFP + qt * 8 + 4 * s;
-                    const uint32_t sfb = tmem + C::COL_SFV + s * C::SFV_PER_KS;
-                    if constexpr (D == 256 && PREORDER) {
-                        const uint64_t b0 = smem_desc(smem_u32(smem + vbuf) + 32u * s, 16u, 512u, 4u);
-                        const uint64_t b1 = smem_desc(smem_u32(smem + vbuf + 128 * 64) + 32u * s, 16u, 512u, 4u);
-                        mma_fp4_block16(o, a, b0, idesc_fp4_block16(128), sfa, sfb, acc);
-                        mma_fp4_block16(o + 128, a, b1, idesc_fp4_block16(144), sfa, sfb + 4, acc);
-                    } else {
-                        const uint64_t b = smem_desc(smem_u32(smem + vbuf) + 32u * s, 16u, 512u, 4u);
-                        mma_fp4_block16(o, a, b, idesc_fp4_block16(C::NO), sfa, sfb, acc);
-                    }
-                }
-                tc_commit(&bars->o_done[qt]);
-                return true;
-            };
-            if (ok) {
-                ok = issue_s(0, 0, true);
-                if (ok && n_qt > 1) ok = issue_s(1, 0, false);
-                if (ok) tc_commit(&bars->k_empty[0]);
-            }
+            int prev_qt = -1, prev_j = 0;
             for (int j = 0; j < n_tiles_max && ok; ++j) {
-                const bool a_next = j + 1 < n_tiles0;
-                const bool b_next = j + 1 < n_tiles1;
-                if (a_next && !issue_s(0, j + 1, true)) { ok = false; break; }
-                if (j < n_tiles0 && !issue_pv(0, j)) { ok = false; break; }
-                if (b_next && !issue_s(1, j + 1, !a_next)) { ok = false; break; }
-                if (a_next || b_next) tc_commit(&bars->k_empty[(j + 1) % kStages]);
-                if (j < n_tiles1 && !issue_pv(1, j)) { ok = false; break; }
-                tc_commit(&bars->v_empty[j % kStages]);
+                const int st = j % kStages;
+                if (!mbar_wait(&bars->k_full[st], (j / kStages) & 1, ctl)) { ok = false; break; }
+                bool first = true;
+#pragma unroll
+                for (int qt = 0; qt < NQT; ++qt) {
+                    if (j >= (qt == 0 ? n_tiles0 : n_tiles1)) continue;
+                    if (prev_qt >= 0 && !mbar_wait(&bars->s_free[prev_qt], prev_j & 1, ctl)) { ok = false; break; }
+                    tc_fence_after();
+                    if (first) {
+#pragma unroll
+                        for (int s = 0; s < C::KS; ++s)
+                            tmem_cp_scale_atom(tmem + C::COL_SFK + 4 * s,
+                                               sf_desc(C::OFF_SFK + st * C::SFQK_BYTES + 512 * s));
+                        first = false;
+                    }
+                    const uint32_t kbuf = C::OFF_K + st * C::K_BYTES;
+#pragma unroll
+                    for (int s = 0; s < C::KS; ++s) {
+                        const uint64_t a =
+                            smem_desc(smem_u32(smem + C::OFF_Q + qt * C::Q_BYTES) + 32u * s, 16u, C::QK_SBO, C::QK_SWZ);
+                        const uint64_t b = smem_desc(smem_u32(smem + kbuf) + 32u * s, 16u, C::QK_SBO, C::QK_SWZ);
+                        mma_fp4_block16(tmem + C::COL_S, a, b, idesc_s, tmem + C::COL_SFQ + qt * 4 * C::KS + 4 * s,
+                                        tmem + C::COL_SFK + 4 * s, s > 0 ? 1u : 0u);
+                    }
+                    tc_commit(&bars->s_full[qt]);
+                    prev_qt = qt;
+                    prev_j = j;
+                }
+                if (ok) tc_commit(&bars->k_empty[st]);
             }
             // wait until every MMA / copy issued above has finished
-            tc_commit(&bars->drain);
-            mbar_wait_drain(&bars->drain, 0, p.wait_limit_ns);
+            tc_commit(&bars->drain[0]);
+            mbar_wait_drain(&bars->drain[0], 0, p.wait_limit_ns);
         }
-    } else {
+    } else if (warp == 2) {
+        // ---------------------------------------------------- PV MMA issuer
+        // O(qt) += P_hat(qt, j) V_hat(j) in the order (0,A) (0,B) (1,A) (1,B) ...
+        if (lane == 0) {
+            auto sf_desc = [&](uint32_t off) { return smem_desc(smem_u32(smem + off), 0u, 128u, 0u); };
+            bool ok = true;
+            if constexpr (PREORDER && D >= 128) {
+#pragma unroll
+                for (int s = 0; s < 2; ++s)
+                    tmem_cp_scale_atom(tmem + C::COL_SFV + s * C::SFV_PER_KS + 4 * C::NRB, sf_desc(C::OFF_ONES));
+            }
+            for (int j = 0; j < n_tiles_max && ok; ++j) {
+                const int st = j % kStages;
+                if (!mbar_wait(&bars->v_full[st], (j / kStages) & 1, ctl)) { ok = false; break; }
+                const uint32_t vbuf = C::OFF_V + st * C::V_STRIDE;
+                const uint32_t sfv = C::OFF_SFV + st * C::SFV_BYTES;
+                bool first = true;
+#pragma unroll
+                for (int qt = 0; qt < NQT; ++qt) {
+                    if (j >= (qt == 0 ? n_tiles0 : n_tiles1)) continue;
+                    if (!mbar_wait(&bars->p_full[qt][j & 1], (j >> 1) & 1, ctl)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t pbuf = C::OFF_P + (qt * 2 + (j & 1)) * C::P_BYTES;
+                    const uint32_t sfp = C::OFF_SFP + (qt * 2 + (j & 1)) * C::SFP_BYTES;
+#pragma unroll
+                    for (int s = 0; s < 2; ++s) {
+                        tmem_cp_scale_atom(tmem + C::COL_SFP + qt * 8 + 4 * s, sf_desc(sfp + 512 * s));
+                        if (first) {
+#pragma unroll
+                            for (int rb = 0; rb < C::NRB; ++rb)
+                                tmem_cp_scale_atom(tmem + C::COL_SFV + s * C::SFV_PER_KS + 4 * rb,
+                                                   sf_desc(sfv + (rb * 2 + s) * 512));
+                        }
+                    }
+                    first = false;
+                    const uint32_t o = tmem + C::COL_O + qt * C::NO;
+#pragma unroll
+                    for (int s = 0; s < 2; ++s) {
+                        const uint64_t a = smem_desc(smem_u32(smem + pbuf) + 32u * s, 16u, 512u, 4u);
+                        const uint32_t acc = (j > 0 || s > 0) ? 1u : 0u;
+                        const uint32_t sfa = tmem + C::COL_SFP + qt * 8 + 4 * s;
+                        const uint32_t sfb = tmem + C::COL_SFV + s * C::SFV_PER_KS;
+                        if constexpr (D == 256 && PREORDER) {
+                            const uint64_t b0 = smem_desc(smem_u32(smem + vbuf) + 32u * s, 16u, 512u, 4u);
+                            const uint64_t b1 = smem_desc(smem_u32(smem + vbuf + 128 * 64) + 32u * s, 16u, 512u, 4u);
+                            mma_fp4_block16(o, a, b0, idesc_fp4_block16(128), sfa, sfb, acc);
+                            mma_fp4_block16(o + 128, a, b1, idesc_fp4_block16(144), sfa, sfb + 4, acc);
+                        } else {
+                            const uint64_t b = smem_desc(smem_u32(smem + vbuf) + 32u * s, 16u, 512u, 4u);
+                            mma_fp4_block16(o, a, b, idesc_fp4_block16(C::NO), sfa, sfb, acc);
+                        }
+                    }
+                    tc_commit(&bars->o_done[qt]);
+                }
+                if (ok) tc_commit(&bars->v_empty[st]);
+            }
+            tc_commit(&bars->drain[1]);
+            mbar_wait_drain(&bars->drain[1], 0, p.wait_limit_ns);
+        }
+    } else if (warp >= kSmWarp0) {
         // ------------------------------------------------------------ softmax
         const int qt = (warp - kSmWarp0) >> 2;             // query tile of this warpgroup
         const int wq = warp & 3;                           // TMEM lane quarter
@@ -403,117 +408,115 @@ __global__ void __launch_bounds__(Cfg<D, PREORDER>::THREADS, 1)
         const size_t out_row = (size_t)grp * rows_in_grp + prow;
         const int nt = qt == 0 ? n_tiles0 : n_tiles1;
         const float c = p.c;
-        const uint64_t c2 = pack2(c, c);
+        const float2 c2 = make_float2(c, c);
         const float one_sixth = rn_one_sixth();
         float m_old = -INFINITY, mc_old = 0.0f, l_hp = 0.0f;
         bool ok = true;
         for (int j = 0; j < nt; ++j) {
             if (!__all_sync(0xFFFFFFFFu, mbar_wait(&bars->s_full[qt], j & 1, ctl))) { ok = false; break; }
             tc_fence_after();
-            float S[128];
+            float2 S[64];
             {
-                uint32_t r[32];
+                uint32_t r[128];
 #pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4) {
-                    tmem_ld32(tl + C::COL_S + 32 * q4, r);
-                    tmem_wait_ld();
+                for (int q = 0; q < 4; ++q)
+                    tmem_ld32(tl + C::COL_S + 32 * q, *reinterpret_cast<uint32_t(*)[32]>(r + 32 * q));
+                tmem_wait_ld();
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) S[32 * q4 + e] = __uint_as_float(r[e]);
-                }
+                for (int e = 0; e < 64; ++e) S[e] = make_float2(__uint_as_float(r[2 * e]), __uint_as_float(r[2 * e + 1]));
             }
             tc_fence_before();
             mbar_arrive(&bars->s_free[qt]);
             const int n0 = j * 128;
             if (n0 + 127 > last) {
 #pragma unroll
-                for (int e = 0; e < 128; ++e)
-                    if (n0 + e > last) S[e] = -INFINITY;
+                for (int e = 0; e < 64; ++e) {
+                    if (n0 + 2 * e > last) S[e].x = -INFINITY;
+                    if (n0 + 2 * e + 1 > last) S[e].y = -INFINITY;
+                }
             }
-            const float m_new = fmaxf(m_old, row_max128(S));
+            // block maxima of S (they also give the block maxima of P: 2^x is monotone)
+            float bm[8];
+#pragma unroll
+            for (int b = 0; b < 8; ++b) bm[b] = max16(S + 8 * b);
+            const float mx = fmax3f(fmax3f(bm[0], bm[1], bm[2]), fmax3f(bm[3], bm[4], bm[5]), fmaxf(bm[6], bm[7]));
+            const float m_new = fmaxf(m_old, mx);
             const float mc_new = (m_new == -INFINITY) ? 0.0f : __fmul_rn(m_new, c);
             const float alpha = (m_old == -INFINITY) ? 0.0f : ex2_approx(mc_old - mc_new);
-            const uint64_t nmc2 = pack2(-mc_new, -mc_new);
-            // P = 2^(S*c - mc), then 8 blocks of 16 keys to E2M1 codes + E4M3 scales
+            const float2 nmc2 = make_float2(-mc_new, -mc_new);
+            // P = 2^(S*c - mc), 8 blocks of 16 keys to E2M1 codes + E4M3 scales
             uint32_t code[16];
             uint32_t sfw[2] = {0u, 0u};
-            uint64_t lsum2 = 0;
+            float2 lsum2 = make_float2(0.0f, 0.0f);
 #pragma unroll
-            for (int blk = 0; blk < 8; ++blk) {
-                float* P = S + 16 * blk;
-#pragma unroll
-                for (int e = 0; e < 16; e += 2) {
-                    float t0f, t1f;
-                    unpack2(ffma2(pack2(P[e], P[e + 1]), c2, nmc2), t0f, t1f);
-                    P[e] = ex2_approx(t0f);
-                    P[e + 1] = ex2_approx(t1f);
-                }
-                if constexpr (!PREORDER) {
-#pragma unroll
-                    for (int e = 0; e < 16; e += 2) lsum2 = fadd2(lsum2, pack2(P[e], P[e + 1]));
-                }
-                const uint32_t sf = cvt_e4m3(__fmul_rn(block_max16(P), one_sixth));
+            for (int b = 0; b < 8; ++b) {
+                const float pm = ex2_approx(__fmaf_rn(bm[b], c, -mc_new));
+                const uint32_t sf = cvt_e4m3(__fmul_rn(pm, one_sixth));
                 const float r = lut[sf & 127u];
-                const uint64_t r2 = pack2(r, r);
-                float y[16];
+                const float2 r2 = make_float2(r, r);
 #pragma unroll
-                for (int e = 0; e < 16; e += 2) unpack2(fmul2(pack2(P[e], P[e + 1]), r2), y[e], y[e + 1]);
-                code[2 * blk] = cvt_e2m1x8(y[0], y[1], y[2], y[3], y[4], y[5], y[6], y[7]);
-                code[2 * blk + 1] = cvt_e2m1x8(y[8], y[9], y[10], y[11], y[12], y[13], y[14], y[15]);
-                sfw[blk >> 2] |= sf << (8 * (blk & 3));
-            }
-            if constexpr (!PREORDER) {
-                float la, lb;
-                unpack2(lsum2, la, lb);
-                l_hp = __fmaf_rn(alpha, l_hp, la + lb);
-            }
-            if constexpr (DUMP) {
-                if (valid) {
-                    uint4* dc = reinterpret_cast<uint4*>(p.p_codes + out_row * (size_t)(p.Nkv / 2) + n0 / 2);
+                for (int h = 0; h < 2; ++h) {
+                    float y[8];
 #pragma unroll
-                    for (int q4 = 0; q4 < 4; ++q4)
-                        dc[q4] = make_uint4(code[4 * q4], code[4 * q4 + 1], code[4 * q4 + 2], code[4 * q4 + 3]);
-                    *reinterpret_cast<uint2*>(p.p_sf + out_row * (size_t)(p.Nkv / 16) + n0 / 16) =
-                        make_uint2(sfw[0], sfw[1]);
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 t = __ffma2_rn(S[8 * b + 4 * h + e], c2, nmc2);
+                        const float2 P = make_float2(ex2_approx(t.x), ex2_approx(t.y));
+                        if constexpr (!PREORDER) lsum2 = __fadd2_rn(lsum2, P);
+                        const float2 yy = __fmul2_rn(P, r2);
+                        y[2 * e] = yy.x;
+                        y[2 * e + 1] = yy.y;
+                    }
+                    code[2 * b + h] = cvt_e2m1x8(y[0], y[1], y[2], y[3], y[4], y[5], y[6], y[7]);
                 }
+                sfw[b >> 2] |= sf << (8 * (b & 3));
             }
+            // rescale O of this tile's rows when some row's max moved (the previous
+            // PV must be done); two 32-column chunks in flight at a time
             if (j > 0) {
-                // PV of the previous tile is done: O is stable, P buffer j&1 is free
                 if (!__all_sync(0xFFFFFFFFu, mbar_wait(&bars->o_done[qt], (j - 1) & 1, ctl))) { ok = false; break; }
                 tc_fence_after();
                 if (__any_sync(0xFFFFFFFFu, alpha != 1.0f)) {
-                    const uint64_t a2 = pack2(alpha, alpha);
-#pragma unroll 1
-                    for (int cc = 0; cc < D; cc += 32) {
-                        uint32_t o[32];
-                        tmem_ld32(tO + cc, o);
-                        tmem_wait_ld();
+                    const float2 a2 = make_float2(alpha, alpha);
+                    uint32_t lv = 0;
+                    if constexpr (PREORDER) tmem_ld1(tO + D, lv);
 #pragma unroll
-                        for (int e = 0; e < 32; e += 2) {
-                            float x0, x1;
-                            unpack2(fmul2(pack2(__uint_as_float(o[e]), __uint_as_float(o[e + 1])), a2), x0, x1);
-                            o[e] = __float_as_uint(x0);
-                            o[e + 1] = __float_as_uint(x1);
-                        }
-                        tmem_st32(tO + cc, o);
-                    }
-                    if constexpr (PREORDER) {
-                        uint32_t lv;
-                        tmem_ld1(tO + D, lv);
+                    for (int ch = 0; ch < C::NCH; ch += 2) {
+                        uint32_t o0[32], o1[32];
+                        tmem_ld32(tO + 32 * ch, o0);
+                        if (ch + 1 < C::NCH) tmem_ld32(tO + 32 * (ch + 1), o1);
                         tmem_wait_ld();
-                        tmem_st1(tO + D, __float_as_uint(__fmul_rn(__uint_as_float(lv), alpha)));
+                        scale_chunk(o0, a2);
+                        tmem_st32(tO + 32 * ch, o0);
+                        if (ch + 1 < C::NCH) {
+                            scale_chunk(o1, a2);
+                            tmem_st32(tO + 32 * (ch + 1), o1);
+                        }
                     }
+                    if constexpr (PREORDER) tmem_st1(tO + D, __float_as_uint(__fmul_rn(__uint_as_float(lv), alpha)));
                     tmem_wait_st();
                 }
             }
+            if constexpr (!PREORDER) l_hp = __fmaf_rn(alpha, l_hp, lsum2.x + lsum2.y);
             {
                 uint8_t* pb = smem + C::OFF_P + (qt * 2 + (j & 1)) * C::P_BYTES;
-#pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4)
-                    *reinterpret_cast<uint4*>(pb + p_swizzle64(row, q4)) =
-                        make_uint4(code[4 * q4], code[4 * q4 + 1], code[4 * q4 + 2], code[4 * q4 + 3]);
                 uint8_t* sb = smem + C::OFF_SFP + (qt * 2 + (j & 1)) * C::SFP_BYTES + 16 * (row & 31) + 4 * (row >> 5);
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    *reinterpret_cast<uint4*>(pb + p_swizzle64(row, q)) =
+                        make_uint4(code[4 * q], code[4 * q + 1], code[4 * q + 2], code[4 * q + 3]);
                 *reinterpret_cast<uint32_t*>(sb) = sfw[0];
                 *reinterpret_cast<uint32_t*>(sb + 512) = sfw[1];
+                if constexpr (DUMP) {
+                    // debug copy of this row's P_hat codes and scales
+                    if (valid) {
+                        uint4* dc = reinterpret_cast<uint4*>(p.p_codes + out_row * (size_t)(p.Nkv / 2) + n0 / 2);
+#pragma unroll
+                        for (int q = 0; q < 4; ++q)
+                            dc[q] = make_uint4(code[4 * q], code[4 * q + 1], code[4 * q + 2], code[4 * q + 3]);
+                        *reinterpret_cast<uint2*>(p.p_sf + out_row * (size_t)(p.Nkv / 16) + n0 / 16) =
+                            make_uint2(sfw[0], sfw[1]);
+                    }
+                }
             }
             fence_proxy_async_smem();
             tc_fence_before();

@@ -43,14 +43,16 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
                  : "memory");
 }
 
+// One bounded test of the phase: the thread sleeps (without issuing) until the
+// phase completes or about 0.1 ms pass, then reports whether it completed.
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(100000u)
         : "memory");
     return ok != 0;
 }
@@ -67,17 +69,28 @@ struct WaitCtl {
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const WaitCtl& ctl) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
-    for (uint32_t spin = 1;; ++spin) {
+    for (;;) {
         if (mbar_try_wait(bar, parity)) return true;
-        if ((spin & 63u) == 0) {
-            if (*ctl.abort) return false;
-            if (global_timer_ns() - t0 > ctl.limit_ns) {
-                *ctl.abort = 1;
-                atomicExch(ctl.status, kStatusTimeout);
-                return false;
-            }
+        if (*ctl.abort) return false;
+        if (global_timer_ns() - t0 > ctl.limit_ns) {
+            *ctl.abort = 1;
+            atomicExch(ctl.status, kStatusTimeout);
+            return false;
         }
     }
+}
+
+// Non-blocking test of a phase.
+__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
 }
 
 // Wait that ignores the abort flag (used while draining copies in flight).

@@ -8,8 +8,8 @@
 namespace hifa4 {
 
 cudaError_t launch_quantize_rows(bool bf16, const void* x, const float* scale, uint8_t* codes, uint8_t* sfs,
-                                 long long n_groups, int rows_per_group, int tiles_per_group, int heads_per_kv,
-                                 int hkv, int n_per_head, int D, cudaStream_t st);
+                                 long long n_groups, int rows_per_group, int tiles_per_group, int hkv, int D,
+                                 cudaStream_t st);
 
 cudaError_t launch_quantize_v(bool bf16, const void* v, uint8_t* vtc, uint8_t* vts, long long n_groups, int nkv, int D,
                               cudaStream_t st);

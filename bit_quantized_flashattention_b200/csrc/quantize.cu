@@ -55,56 +55,41 @@ __device__ __forceinline__ uint32_t atom_offset(uint32_t r) { return 16u * (r & 
 
 // ---------------------------------------------------------------- Q and K
 
-// One thread per (group, tile, row-in-tile, 64-wide K step). A group is the
-// block of rows that shares a kv head: G*N consecutive rows of the input
-// (G = q heads per kv head for Q, 1 for K). Rows past G*N in a group's last
-// tile only receive zero scales.
+// One thread per 16-element block, consecutive lanes on consecutive blocks so
+// that every load and store instruction of a warp covers contiguous bytes.
+// Rows are grouped per kv head: a group is G*N consecutive input rows (G = q
+// heads per kv head for Q, 1 for K), padded to Tq tiles of 128 rows; threads
+// of padding rows only zero their scale byte. The four scale bytes of a
+// 64-element K step are gathered with shuffles into one 32-bit word of the
+// MMA-ready atom.
 template <typename T, int D>
 __global__ void __launch_bounds__(256) quantize_rows_kernel(const T* __restrict__ x, const float* __restrict__ scale,
                                                             uint8_t* __restrict__ codes, uint8_t* __restrict__ sfs,
-                                                            long long n_groups, int rows_per_group, int tiles_per_group,
-                                                            int heads_per_kv, int hkv, int n_per_head) {
-    constexpr int KS = D / 64;
-    const long long tid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-    const long long total = n_groups * tiles_per_group * 128LL * KS;
-    if (tid >= total) return;
-    const int s = (int)(tid % KS);
-    const long long tr = tid / KS;
-    const int r = (int)(tr % 128);
-    const long long gt = tr / 128;                 // group * tiles_per_group + tile
-    const int t = (int)(gt % tiles_per_group);
-    const long long grp = gt / tiles_per_group;    // b * Hkv + g
-    const int p = t * 128 + r;
-    uint32_t* sf_word = reinterpret_cast<uint32_t*>(sfs + ((size_t)gt * KS + s) * 512 + atom_offset((uint32_t)r));
-    if (p >= rows_per_group) {
-        *sf_word = 0u;
-        return;
-    }
-    const size_t row = (size_t)grp * rows_per_group + p;
-    const T* src = x + row * D + s * 64;
-    const uint4* src4 = reinterpret_cast<const uint4*>(src);
-    const float* sc = nullptr;
-    if (scale != nullptr) {
-        const int g = (int)(grp % hkv);
-        (void)heads_per_kv;
-        (void)n_per_head;
-        sc = scale + (size_t)g * D + s * 64;
-    }
-    uint32_t words[8];
-    uint32_t sfw = 0u;
-#pragma unroll
-    for (int blk = 0; blk < 4; ++blk) {
-        float v[16];
-        float a[8], b[8];
-        unpack8<T>(src4[2 * blk], a);
-        unpack8<T>(src4[2 * blk + 1], b);
+                                                            unsigned total_blocks, unsigned rows_per_group,
+                                                            unsigned padded_rows, unsigned hkv) {
+    constexpr unsigned NB = D / 16;                        // blocks per row
+    constexpr unsigned KS = D / 64;
+    const unsigned tid = blockIdx.x * blockDim.x + threadIdx.x;
+    const bool active = tid < total_blocks;
+    const unsigned kb = tid % NB;
+    const unsigned pr = tid / NB;                          // padded row index over all groups
+    const unsigned grp = pr / padded_rows;
+    const unsigned p = pr - grp * padded_rows;             // row within the group
+    const bool real = active && p < rows_per_group;
+    uint32_t sf = 0u;
+    if (real) {
+        const size_t row = (size_t)grp * rows_per_group + p;
+        const uint4* src = reinterpret_cast<const uint4*>(x + row * D + kb * 16);
+        float v[16], a[8], b[8];
+        unpack8<T>(src[0], a);
+        unpack8<T>(src[1], b);
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
             v[i] = a[i];
             v[8 + i] = b[i];
         }
-        if (sc != nullptr) {
-            const float4* sc4 = reinterpret_cast<const float4*>(sc + blk * 16);
+        if (scale != nullptr) {
+            const float4* sc4 = reinterpret_cast<const float4*>(scale + (size_t)(grp % hkv) * D + kb * 16);
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
                 const float4 m = __ldg(sc4 + q);
@@ -114,13 +99,18 @@ __global__ void __launch_bounds__(256) quantize_rows_kernel(const T* __restrict_
                 v[4 * q + 3] = __fmul_rn(v[4 * q + 3], m.w);
             }
         }
-        const uint32_t sf = quant_block16(v, words[2 * blk], words[2 * blk + 1]);
-        sfw |= sf << (8 * blk);
+        uint32_t lo, hi;
+        sf = quant_block16(v, lo, hi);
+        *reinterpret_cast<uint2*>(codes + row * (D / 2) + kb * 8) = make_uint2(lo, hi);
     }
-    uint4* dst = reinterpret_cast<uint4*>(codes + row * (D / 2) + s * 32);
-    dst[0] = make_uint4(words[0], words[1], words[2], words[3]);
-    dst[1] = make_uint4(words[4], words[5], words[6], words[7]);
-    *sf_word = sfw;
+    // gather the 4 scale bytes of this K step (lanes kb&~3 .. kb|3 are adjacent)
+    uint32_t w = sf << (8 * (kb & 3));
+    w |= __shfl_xor_sync(0xFFFFFFFFu, w, 1);
+    w |= __shfl_xor_sync(0xFFFFFFFFu, w, 2);
+    if (active && (kb & 3) == 0) {
+        const unsigned t = p / 128, r = p % 128, s = kb / 4;
+        *reinterpret_cast<uint32_t*>(sfs + (((size_t)grp * (padded_rows / 128) + t) * KS + s) * 512 + atom_offset(r)) = w;
+    }
 }
 
 // ---------------------------------------------------------------------- V
@@ -216,25 +206,23 @@ __global__ void calib_finalize_kernel(float* __restrict__ s, float* __restrict__
 
 template <typename T>
 static cudaError_t launch_rows_t(const void* x, const float* scale, uint8_t* codes, uint8_t* sfs, long long n_groups,
-                                 int rows_per_group, int tiles_per_group, int heads_per_kv, int hkv, int n_per_head,
-                                 int D, cudaStream_t st) {
-    const long long total = n_groups * tiles_per_group * 128LL * (D / 64);
+                                 int rows_per_group, int tiles_per_group, int hkv, int D, cudaStream_t st) {
+    const long long padded = (long long)tiles_per_group * 128;
+    const long long total = n_groups * padded * (D / 16);
+    if (total > 0xFFFFFFFFLL - 256) return cudaErrorInvalidConfiguration;
     const int threads = 256;
-    const long long blocks = (total + threads - 1) / threads;
-    if (blocks > 0x7FFFFFFFLL) return cudaErrorInvalidConfiguration;
+    const unsigned blocks = (unsigned)((total + threads - 1) / threads);
     const T* xp = static_cast<const T*>(x);
+    const unsigned tb = (unsigned)total, rg = (unsigned)rows_per_group, pr = (unsigned)padded, hk = (unsigned)hkv;
     switch (D) {
         case 64:
-            quantize_rows_kernel<T, 64><<<(unsigned)blocks, threads, 0, st>>>(
-                xp, scale, codes, sfs, n_groups, rows_per_group, tiles_per_group, heads_per_kv, hkv, n_per_head);
+            quantize_rows_kernel<T, 64><<<blocks, threads, 0, st>>>(xp, scale, codes, sfs, tb, rg, pr, hk);
             break;
         case 128:
-            quantize_rows_kernel<T, 128><<<(unsigned)blocks, threads, 0, st>>>(
-                xp, scale, codes, sfs, n_groups, rows_per_group, tiles_per_group, heads_per_kv, hkv, n_per_head);
+            quantize_rows_kernel<T, 128><<<blocks, threads, 0, st>>>(xp, scale, codes, sfs, tb, rg, pr, hk);
             break;
         case 256:
-            quantize_rows_kernel<T, 256><<<(unsigned)blocks, threads, 0, st>>>(
-                xp, scale, codes, sfs, n_groups, rows_per_group, tiles_per_group, heads_per_kv, hkv, n_per_head);
+            quantize_rows_kernel<T, 256><<<blocks, threads, 0, st>>>(xp, scale, codes, sfs, tb, rg, pr, hk);
             break;
         default:
             return cudaErrorInvalidValue;
@@ -243,13 +231,12 @@ static cudaError_t launch_rows_t(const void* x, const float* scale, uint8_t* cod
 }
 
 cudaError_t launch_quantize_rows(bool bf16, const void* x, const float* scale, uint8_t* codes, uint8_t* sfs,
-                                 long long n_groups, int rows_per_group, int tiles_per_group, int heads_per_kv,
-                                 int hkv, int n_per_head, int D, cudaStream_t st) {
+                                 long long n_groups, int rows_per_group, int tiles_per_group, int hkv, int D,
+                                 cudaStream_t st) {
     if (bf16)
-        return launch_rows_t<__nv_bfloat16>(x, scale, codes, sfs, n_groups, rows_per_group, tiles_per_group,
-                                            heads_per_kv, hkv, n_per_head, D, st);
-    return launch_rows_t<__half>(x, scale, codes, sfs, n_groups, rows_per_group, tiles_per_group, heads_per_kv, hkv,
-                                 n_per_head, D, st);
+        return launch_rows_t<__nv_bfloat16>(x, scale, codes, sfs, n_groups, rows_per_group, tiles_per_group, hkv, D,
+                                            st);
+    return launch_rows_t<__half>(x, scale, codes, sfs, n_groups, rows_per_group, tiles_per_group, hkv, D, st);
 }
 
 template <typename T>

@@ -196,6 +196,10 @@ hifa4_status hifa4_get_status(void* workspace, hifa4_stream_t stream);
  * flight. Returns the previous limit. */
 long long hifa4_debug_set_wait_limit(long long limit_ns, int stall_loads);
 
+/* Description of the last CUDA error behind an HIFA4_ERR_CUDA returned to
+ * the calling thread ("no error" if there was none). */
+const char* hifa4_last_cuda_error(void);
+
 /* Human-readable name of a status code. */
 const char* hifa4_status_string(hifa4_status status);
 
