@@ -33,15 +33,24 @@ __device__ __forceinline__ void unpack8(const uint4& w, float (&f)[8]) {
     for (int i = 0; i < 8; ++i) f[i] = to_f32<T>(e[i]);
 }
 
-// Quantize one 16-element block held in registers: returns the scale code,
-// writes two 32-bit code words (elements 0-7, 8-15).
-__device__ __forceinline__ uint32_t quant_block16(const float (&x)[16], uint32_t& lo, uint32_t& hi) {
-    float amax = 0.0f;
+// Byte offset of (row r, scale k) inside a 512-byte scale atom.
+__device__ __forceinline__ uint32_t atom_offset(uint32_t r) { return 16u * (r & 31u) + 4u * ((r >> 5) & 3u); }
+
+// Reciprocal table RN(1/decode(sf)) for the 128 non-negative E4M3 codes
+// (entry 0 = 0: a zero scale zeroes the block), built per CTA.
+__device__ __forceinline__ void build_rcp_lut(float* lut) {
+    for (unsigned i = threadIdx.x; i < 128; i += blockDim.x) lut[i] = (i == 0) ? 0.0f : __frcp_rn(e4m3_to_f32(i));
+    __syncthreads();
+}
+
+// Quantize 16 elements held by one thread (the rule in the file header).
+__device__ __forceinline__ uint32_t quant_block16_lut(const float (&x)[16], const float* lut, uint32_t& lo,
+                                                      uint32_t& hi) {
+    float amax = fabsf(x[0]);
 #pragma unroll
-    for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(x[i]));
+    for (int i = 1; i < 16; ++i) amax = fmaxf(amax, fabsf(x[i]));
     const uint32_t sf = cvt_e4m3(__fmul_rn(amax, rn_one_sixth()));
-    const float S = e4m3_to_f32(sf);
-    const float r = (sf == 0u) ? 0.0f : __frcp_rn(S);
+    const float r = lut[sf & 127u];
     float y[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) y[i] = __fmul_rn(x[i], r);
@@ -50,117 +59,129 @@ __device__ __forceinline__ uint32_t quant_block16(const float (&x)[16], uint32_t
     return sf;
 }
 
-// Byte offset of (row r, scale k) inside a 512-byte scale atom.
-__device__ __forceinline__ uint32_t atom_offset(uint32_t r) { return 16u * (r & 31u) + 4u * ((r >> 5) & 3u); }
-
 // ---------------------------------------------------------------- Q and K
 
-// One thread per 16-element block, consecutive lanes on consecutive blocks so
-// that every load and store instruction of a warp covers contiguous bytes.
-// Rows are grouped per kv head: a group is G*N consecutive input rows (G = q
-// heads per kv head for Q, 1 for K), padded to Tq tiles of 128 rows; threads
-// of padding rows only zero their scale byte. The four scale bytes of a
-// 64-element K step are gathered with shuffles into one 32-bit word of the
-// MMA-ready atom.
+// Rows of Q or K (quantized along D). blockIdx.y is the group: the G*N
+// consecutive input rows that share a kv head (G = q heads per kv head for Q,
+// 1 for K), padded to whole 128-row tiles; padding rows only receive zero
+// scale words. Each lane owns one 8-element chunk of a row (so a warp
+// instruction reads 512 contiguous bytes) and walks the group's rows with a
+// block stride; its 8 smoothing factors stay in registers. The two halves of a
+// 16-element block sit in neighbouring lanes (one shuffle for the maximum), and
+// the 4 scale bytes of a 64-element K step are gathered by shuffles into one
+// 32-bit word of the MMA-ready atom.
 template <typename T, int D>
 __global__ void __launch_bounds__(256) quantize_rows_kernel(const T* __restrict__ x, const float* __restrict__ scale,
                                                             uint8_t* __restrict__ codes, uint8_t* __restrict__ sfs,
-                                                            unsigned total_blocks, unsigned rows_per_group,
-                                                            unsigned padded_rows, unsigned hkv) {
-    constexpr unsigned NB = D / 16;                        // blocks per row
+                                                            unsigned rows_per_group, unsigned tiles_per_group,
+                                                            unsigned hkv) {
+    constexpr unsigned CPR = D / 8;                        // chunks per row
+    constexpr unsigned RPB = 256 / CPR;                    // rows per block step
     constexpr unsigned KS = D / 64;
-    const unsigned tid = blockIdx.x * blockDim.x + threadIdx.x;
-    const bool active = tid < total_blocks;
-    const unsigned kb = tid % NB;
-    const unsigned pr = tid / NB;                          // padded row index over all groups
-    const unsigned grp = pr / padded_rows;
-    const unsigned p = pr - grp * padded_rows;             // row within the group
-    const bool real = active && p < rows_per_group;
-    uint32_t sf = 0u;
-    if (real) {
-        const size_t row = (size_t)grp * rows_per_group + p;
-        const uint4* src = reinterpret_cast<const uint4*>(x + row * D + kb * 16);
-        float v[16], a[8], b[8];
-        unpack8<T>(src[0], a);
-        unpack8<T>(src[1], b);
+    __shared__ float lut[128];
+    build_rcp_lut(lut);
+    const unsigned grp = blockIdx.y;
+    const unsigned c = threadIdx.x % CPR;
+    const unsigned padded = tiles_per_group * 128;
+    float sc[8];
+    if (scale != nullptr) {
+        const float4* s4 = reinterpret_cast<const float4*>(scale + (size_t)(grp % hkv) * D + c * 8);
+        const float4 a = __ldg(s4), b = __ldg(s4 + 1);
+        sc[0] = a.x; sc[1] = a.y; sc[2] = a.z; sc[3] = a.w;
+        sc[4] = b.x; sc[5] = b.y; sc[6] = b.z; sc[7] = b.w;
+    }
+    const T* xg = x + (size_t)grp * rows_per_group * D;
+    uint8_t* cg = codes + (size_t)grp * rows_per_group * (D / 2);
+    uint8_t* sg = sfs + (size_t)grp * tiles_per_group * KS * 512;
+    for (unsigned p = blockIdx.x * RPB + threadIdx.x / CPR; p - (threadIdx.x / CPR) < padded;
+         p += gridDim.x * RPB) {
+        const bool in_tile = p < padded;
+        const bool real = p < rows_per_group;
+        float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        if (real) {
+            unpack8<T>(*reinterpret_cast<const uint4*>(xg + (size_t)p * D + c * 8), v);
+            if (scale != nullptr) {
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            v[i] = a[i];
-            v[8 + i] = b[i];
-        }
-        if (scale != nullptr) {
-            const float4* sc4 = reinterpret_cast<const float4*>(scale + (size_t)(grp % hkv) * D + kb * 16);
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const float4 m = __ldg(sc4 + q);
-                v[4 * q + 0] = __fmul_rn(v[4 * q + 0], m.x);
-                v[4 * q + 1] = __fmul_rn(v[4 * q + 1], m.y);
-                v[4 * q + 2] = __fmul_rn(v[4 * q + 2], m.z);
-                v[4 * q + 3] = __fmul_rn(v[4 * q + 3], m.w);
+                for (int i = 0; i < 8; ++i) v[i] = __fmul_rn(v[i], sc[i]);
             }
         }
-        uint32_t lo, hi;
-        sf = quant_block16(v, lo, hi);
-        *reinterpret_cast<uint2*>(codes + row * (D / 2) + kb * 8) = make_uint2(lo, hi);
-    }
-    // gather the 4 scale bytes of this K step (lanes kb&~3 .. kb|3 are adjacent)
-    uint32_t w = sf << (8 * (kb & 3));
-    w |= __shfl_xor_sync(0xFFFFFFFFu, w, 1);
-    w |= __shfl_xor_sync(0xFFFFFFFFu, w, 2);
-    if (active && (kb & 3) == 0) {
-        const unsigned t = p / 128, r = p % 128, s = kb / 4;
-        *reinterpret_cast<uint32_t*>(sfs + (((size_t)grp * (padded_rows / 128) + t) * KS + s) * 512 + atom_offset(r)) = w;
+        float amax = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
+        amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
+        const uint32_t sf = cvt_e4m3(__fmul_rn(amax, rn_one_sixth()));
+        const float r = lut[sf & 127u];
+        float y[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) y[i] = __fmul_rn(v[i], r);
+        const uint32_t w = cvt_e2m1x8(y[0], y[1], y[2], y[3], y[4], y[5], y[6], y[7]);
+        if (real) *reinterpret_cast<uint32_t*>(cg + (size_t)p * (D / 2) + c * 4) = w;
+        // scale word of the 64-element K step: blocks 2k..2k+1 -> byte k
+        uint32_t word = ((c & 1u) == 0u) ? (sf << (8u * ((c >> 1) & 3u))) : 0u;
+        word |= __shfl_xor_sync(0xFFFFFFFFu, word, 2);
+        word |= __shfl_xor_sync(0xFFFFFFFFu, word, 4);
+        if (in_tile && (c & 7u) == 0u)
+            *reinterpret_cast<uint32_t*>(sg + ((size_t)(p >> 7) * KS + c / 8) * 512 + atom_offset(p & 127u)) =
+                real ? word : 0u;
     }
 }
 
 // ---------------------------------------------------------------------- V
 
-// One CTA per (b*Hkv + g, 128-token tile): stage the tile [128, D] in shared
-// memory, then one thread per (channel d, 64-token half) quantizes along tokens
-// and writes the transposed codes and one scale word. For D = 64 the extra
-// threads fill the atom's padding rows (row 64 = 1.0 for the normalizer
-// column of P-Reordering, the rest 0).
+// V quantized along tokens, written transposed. A warp covers 32 channels x 64
+// tokens of one group; lane (cc, tb) owns 4 channels (cc = 0..7) x one 16-token
+// block (tb = 0..3): it reads 16 rows of 8 bytes (each load instruction reads 4
+// rows of 64 contiguous bytes), quantizes one block per channel and writes 8
+// code bytes per channel; the 4 scale bytes of a channel for the 64-token half
+// come from the lanes tb = 0..3 and are gathered by shuffles. For D = 64 one
+// warp per half also fills the padding rows of the scale atoms (row 64 = 1.0
+// for the normalizer column of P-Reordering, the rest 0).
 template <typename T, int D>
-__global__ void __launch_bounds__(2 * (D < 128 ? 128 : D)) quantize_v_kernel(const T* __restrict__ v, uint8_t* __restrict__ vtc,
-                                                                           uint8_t* __restrict__ vts, int nkv) {
-    constexpr int PITCH = D + 8;                        // elements; keeps column reads conflict-free
+__global__ void __launch_bounds__(256) quantize_v_kernel(const T* __restrict__ v, uint8_t* __restrict__ vtc,
+                                                         uint8_t* __restrict__ vts, int nkv) {
     constexpr int NRB = (D + 127) / 128;
-    constexpr int NT = 2 * (D < 128 ? 128 : D);
-    extern __shared__ __align__(16) uint8_t v_smem[];
-    T* tile = reinterpret_cast<T*>(v_smem);
-    const int j = blockIdx.x;                           // token tile
-    const long long grp = blockIdx.y;                   // b * Hkv + g
-    const int ntile = nkv / 128;
-    const T* src = v + ((size_t)grp * nkv + (size_t)j * 128) * D;
-    constexpr int VEC = 8;                              // elements per 128-bit load
-    for (int idx = threadIdx.x; idx < 128 * D / VEC; idx += NT) {
-        const int row = idx / (D / VEC), c = idx % (D / VEC);
-        const uint4 w = reinterpret_cast<const uint4*>(src + (size_t)row * D)[c];
-        *reinterpret_cast<uint4*>(&tile[row * PITCH + c * VEC]) = w;
-    }
-    __syncthreads();
-    const int d = threadIdx.x % (NT / 2);
-    const int half = threadIdx.x / (NT / 2);
-    const size_t atom = (((size_t)grp * ntile + j) * NRB + (d >> 7)) * 2 + half;
-    uint32_t* sf_word = reinterpret_cast<uint32_t*>(vts + atom * 512 + atom_offset((uint32_t)(d & 127)));
-    if (d >= D) {                                       // padding rows (only when D = 64)
-        *sf_word = (d == D) ? 0x38383838u : 0u;
-        return;
-    }
-    uint32_t words[8];
-    uint32_t sfw = 0u;
+    constexpr unsigned CWARPS = D / 32;                    // warps per 64-token half (32 channels each)
+    __shared__ float lut[128];
+    build_rcp_lut(lut);
+    const unsigned lane = threadIdx.x & 31u;
+    const unsigned gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;   // warp within the group
+    const unsigned nhalf = (unsigned)nkv / 64u;
+    if (gw >= nhalf * CWARPS) return;
+    const unsigned grp = blockIdx.y;
+    const unsigned cw = gw % CWARPS;
+    const unsigned hh = gw / CWARPS;                       // 64-token half over the sequence
+    const unsigned cc = lane >> 2, tb = lane & 3u;
+    const unsigned d0 = cw * 32 + cc * 4;                  // first channel of this lane
+    const unsigned tok0 = hh * 64 + tb * 16;               // first token of this lane's block
+    const T* src = v + ((size_t)grp * nkv + tok0) * D + d0;
+    uint2 raw[16];
 #pragma unroll
-    for (int blk = 0; blk < 4; ++blk) {
+    for (int i = 0; i < 16; ++i) raw[i] = *reinterpret_cast<const uint2*>(src + (size_t)i * D);
+    const unsigned j = hh / 2, half = hh % 2;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
         float x[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) x[i] = to_f32<T>(tile[(half * 64 + blk * 16 + i) * PITCH + d]);
-        const uint32_t sf = quant_block16(x, words[2 * blk], words[2 * blk + 1]);
-        sfw |= sf << (8 * blk);
+        for (int i = 0; i < 16; ++i) x[i] = to_f32<T>(reinterpret_cast<const T*>(&raw[i])[k]);
+        uint32_t lo, hi;
+        const uint32_t sf = quant_block16_lut(x, lut, lo, hi);
+        const unsigned d = d0 + k;
+        *reinterpret_cast<uint2*>(vtc + ((size_t)grp * D + d) * (nkv / 2) + tok0 / 2) = make_uint2(lo, hi);
+        uint32_t word = sf << (8u * tb);
+        word |= __shfl_xor_sync(0xFFFFFFFFu, word, 1);
+        word |= __shfl_xor_sync(0xFFFFFFFFu, word, 2);
+        if (tb == 0) {
+            const size_t atom = (((size_t)grp * (nkv / 128) + j) * NRB + (d >> 7)) * 2 + half;
+            *reinterpret_cast<uint32_t*>(vts + atom * 512 + atom_offset(d & 127u)) = word;
+        }
     }
-    uint4* dst = reinterpret_cast<uint4*>(vtc + ((size_t)grp * D + d) * (nkv / 2) + (size_t)j * 64 + half * 32);
-    dst[0] = make_uint4(words[0], words[1], words[2], words[3]);
-    dst[1] = make_uint4(words[4], words[5], words[6], words[7]);
-    *sf_word = sfw;
+    if constexpr (D == 64) {
+        if (cw == 0) {
+            const size_t atom = ((size_t)grp * (nkv / 128) + j) * 2 + half;
+            for (unsigned r = 64 + lane; r < 128; r += 32)
+                *reinterpret_cast<uint32_t*>(vts + atom * 512 + atom_offset(r)) = (r == 64) ? 0x38383838u : 0u;
+        }
+    }
 }
 
 // ------------------------------------------------------------ calibration
@@ -207,22 +228,35 @@ __global__ void calib_finalize_kernel(float* __restrict__ s, float* __restrict__
 template <typename T>
 static cudaError_t launch_rows_t(const void* x, const float* scale, uint8_t* codes, uint8_t* sfs, long long n_groups,
                                  int rows_per_group, int tiles_per_group, int hkv, int D, cudaStream_t st) {
-    const long long padded = (long long)tiles_per_group * 128;
-    const long long total = n_groups * padded * (D / 16);
-    if (total > 0xFFFFFFFFLL - 256) return cudaErrorInvalidConfiguration;
-    const int threads = 256;
-    const unsigned blocks = (unsigned)((total + threads - 1) / threads);
+    if (n_groups > 65535) return cudaErrorInvalidConfiguration;
+    int dev = 0, sms = 148, occ = 1;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    cudaError_t e = cudaSuccess;
+    switch (D) {
+        case 64: e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, quantize_rows_kernel<T, 64>, 256, 0); break;
+        case 128: e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, quantize_rows_kernel<T, 128>, 256, 0); break;
+        default: e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, quantize_rows_kernel<T, 256>, 256, 0); break;
+    }
+    if (e != cudaSuccess || occ < 1) occ = 1;
+    const long long rows_per_step = 256 / (D / 8);
+    const long long steps = ((long long)tiles_per_group * 128 + rows_per_step - 1) / rows_per_step;
+    // one resident wave: every CTA of the grid is on an SM at once
+    long long bx = ((long long)sms * occ) / n_groups;
+    if (bx > steps) bx = steps;
+    if (bx < 1) bx = 1;
+    const dim3 grid((unsigned)bx, (unsigned)n_groups);
     const T* xp = static_cast<const T*>(x);
-    const unsigned tb = (unsigned)total, rg = (unsigned)rows_per_group, pr = (unsigned)padded, hk = (unsigned)hkv;
+    const unsigned rg = (unsigned)rows_per_group, tg = (unsigned)tiles_per_group, hk = (unsigned)hkv;
     switch (D) {
         case 64:
-            quantize_rows_kernel<T, 64><<<blocks, threads, 0, st>>>(xp, scale, codes, sfs, tb, rg, pr, hk);
+            quantize_rows_kernel<T, 64><<<grid, 256, 0, st>>>(xp, scale, codes, sfs, rg, tg, hk);
             break;
         case 128:
-            quantize_rows_kernel<T, 128><<<blocks, threads, 0, st>>>(xp, scale, codes, sfs, tb, rg, pr, hk);
+            quantize_rows_kernel<T, 128><<<grid, 256, 0, st>>>(xp, scale, codes, sfs, rg, tg, hk);
             break;
         case 256:
-            quantize_rows_kernel<T, 256><<<blocks, threads, 0, st>>>(xp, scale, codes, sfs, tb, rg, pr, hk);
+            quantize_rows_kernel<T, 256><<<grid, 256, 0, st>>>(xp, scale, codes, sfs, rg, tg, hk);
             break;
         default:
             return cudaErrorInvalidValue;
@@ -243,21 +277,18 @@ template <typename T>
 static cudaError_t launch_v_t(const void* v, uint8_t* vtc, uint8_t* vts, long long n_groups, int nkv, int D,
                               cudaStream_t st) {
     if (n_groups > 65535) return cudaErrorInvalidConfiguration;
-    const dim3 grid(nkv / 128, (unsigned)n_groups);
+    const long long warps = (long long)(nkv / 64) * (D / 32);
+    const dim3 grid((unsigned)((warps * 32 + 255) / 256), (unsigned)n_groups);
     const T* vp = static_cast<const T*>(v);
-    const size_t smem = (size_t)128 * (D + 8) * sizeof(T);
-    cudaError_t e = cudaSuccess;
     switch (D) {
         case 64:
-            quantize_v_kernel<T, 64><<<grid, 256, smem, st>>>(vp, vtc, vts, nkv);
+            quantize_v_kernel<T, 64><<<grid, 256, 0, st>>>(vp, vtc, vts, nkv);
             break;
         case 128:
-            quantize_v_kernel<T, 128><<<grid, 256, smem, st>>>(vp, vtc, vts, nkv);
+            quantize_v_kernel<T, 128><<<grid, 256, 0, st>>>(vp, vtc, vts, nkv);
             break;
         case 256:
-            e = cudaFuncSetAttribute(quantize_v_kernel<T, 256>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-            if (e != cudaSuccess) return e;
-            quantize_v_kernel<T, 256><<<grid, 512, smem, st>>>(vp, vtc, vts, nkv);
+            quantize_v_kernel<T, 256><<<grid, 256, 0, st>>>(vp, vtc, vts, nkv);
             break;
         default:
             return cudaErrorInvalidValue;
