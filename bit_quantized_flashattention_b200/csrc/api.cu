@@ -191,35 +191,58 @@ hifa4_status hifa4_quantize_kv(const void* k, const void* v, hifa4_dtype dtype, 
     for (const void* q : ptrs)
         if (q == nullptr || !aligned16(q)) return HIFA4_ERR_INVALID_ARG;
     if (s_inv != nullptr && !aligned16(s_inv)) return HIFA4_ERR_INVALID_ARG;
-    if ((long long)B * Hkv > 65535) return HIFA4_ERR_UNSUPPORTED;
-    const bool bf = dtype == HIFA4_BF16;
-    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    const long long n_grp = (long long)B * Hkv;
-    cudaError_t e = launch_quantize_rows(bf, k, s_inv, static_cast<uint8_t*>(out->kc), static_cast<uint8_t*>(out->ks),
-                                         n_grp, Nkv, Nkv / 128, Hkv, D, st);
-    if (e != cudaSuccess) return from_cuda(e);
-    e = launch_quantize_v(bf, v, static_cast<uint8_t*>(out->vtc), static_cast<uint8_t*>(out->vts), n_grp, Nkv, D, st);
-    return from_cuda(e);
+    QuantArgs a{};
+    a.bf16 = dtype == HIFA4_BF16;
+    a.D = D;
+    a.G = 1;
+    a.hkv = Hkv;
+    a.nq = 0;
+    a.nkv = Nkv;
+    a.tiles_q = 0;
+    a.n_groups = (long long)B * Hkv;
+    a.k = k;
+    a.v = v;
+    a.s_inv = s_inv;
+    a.kc = static_cast<uint8_t*>(out->kc);
+    a.ks = static_cast<uint8_t*>(out->ks);
+    a.vtc = static_cast<uint8_t*>(out->vtc);
+    a.vts = static_cast<uint8_t*>(out->vts);
+    return from_cuda(launch_quantize_qkv(a, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 hifa4_status hifa4_quantize_qkv(const void* q, const void* k, const void* v, hifa4_dtype dtype, int B, int Hq, int Hkv,
                                 int Nq, int Nkv, int D, const float* s, const float* s_inv, const hifa4_packed* out,
                                 hifa4_stream_t stream) {
-    if (q == nullptr || out == nullptr) return HIFA4_ERR_INVALID_ARG;
+    if (q == nullptr || k == nullptr || v == nullptr || out == nullptr) return HIFA4_ERR_INVALID_ARG;
     if ((s == nullptr) != (s_inv == nullptr)) return HIFA4_ERR_INVALID_ARG;
     if (dtype != HIFA4_F16 && dtype != HIFA4_BF16) return HIFA4_ERR_INVALID_ARG;
     if (!shape_ok(B, Hq, Hkv, Nq, Nkv, D)) return HIFA4_ERR_UNSUPPORTED;
-    if (!aligned16(q) || out->qc == nullptr || out->qs == nullptr || !aligned16(out->qc) || !aligned16(out->qs) ||
-        (s != nullptr && !aligned16(s)))
-        return HIFA4_ERR_INVALID_ARG;
+    const void* ptrs[9] = {q, k, v, out->qc, out->qs, out->kc, out->ks, out->vtc, out->vts};
+    for (const void* p : ptrs)
+        if (p == nullptr || !aligned16(p)) return HIFA4_ERR_INVALID_ARG;
+    if ((s != nullptr && !aligned16(s)) || (s_inv != nullptr && !aligned16(s_inv))) return HIFA4_ERR_INVALID_ARG;
     const Sizes sz = sizes_of(B, Hq, Hkv, Nq, Nkv, D);
-    const int G = Hq / Hkv;
-    const long long n_grp = (long long)B * Hkv;
-    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    cudaError_t e = launch_quantize_rows(dtype == HIFA4_BF16, q, s, static_cast<uint8_t*>(out->qc),
-                                         static_cast<uint8_t*>(out->qs), n_grp, G * Nq, sz.Tq, Hkv, D, st);
-    if (e != cudaSuccess) return from_cuda(e);
-    return hifa4_quantize_kv(k, v, dtype, B, Hkv, Nkv, D, s_inv, out, stream);
+    QuantArgs a{};
+    a.bf16 = dtype == HIFA4_BF16;
+    a.D = D;
+    a.G = Hq / Hkv;
+    a.hkv = Hkv;
+    a.nq = Nq;
+    a.nkv = Nkv;
+    a.tiles_q = sz.Tq;
+    a.n_groups = (long long)B * Hkv;
+    a.q = q;
+    a.k = k;
+    a.v = v;
+    a.s = s;
+    a.s_inv = s_inv;
+    a.qc = static_cast<uint8_t*>(out->qc);
+    a.qs = static_cast<uint8_t*>(out->qs);
+    a.kc = static_cast<uint8_t*>(out->kc);
+    a.ks = static_cast<uint8_t*>(out->ks);
+    a.vtc = static_cast<uint8_t*>(out->vtc);
+    a.vts = static_cast<uint8_t*>(out->vts);
+    return from_cuda(launch_quantize_qkv(a, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 hifa4_status hifa4_attention_fwd(const hifa4_packed* in, int B, int Hq, int Hkv, int Nq, int Nkv, int D,

@@ -7,12 +7,21 @@
 
 namespace hifa4 {
 
-cudaError_t launch_quantize_rows(bool bf16, const void* x, const float* scale, uint8_t* codes, uint8_t* sfs,
-                                 long long n_groups, int rows_per_group, int tiles_per_group, int hkv, int D,
-                                 cudaStream_t st);
+// One pass over Q (optional), K and V: smooth, quantize, write codes and
+// MMA-ready scales.
+struct QuantArgs {
+    bool bf16;
+    int D, G, hkv, nq, nkv, tiles_q;
+    long long n_groups;           // B * Hkv
+    const void* q;                // null: K and V only
+    const void* k;
+    const void* v;
+    const float* s;
+    const float* s_inv;
+    uint8_t *qc, *qs, *kc, *ks, *vtc, *vts;
+};
 
-cudaError_t launch_quantize_v(bool bf16, const void* v, uint8_t* vtc, uint8_t* vts, long long n_groups, int nkv, int D,
-                              cudaStream_t st);
+cudaError_t launch_quantize_qkv(const QuantArgs& a, cudaStream_t st);
 
 cudaError_t launch_calibrate(bool bf16, const void* q, const void* k, int B, int Hq, int Hkv, int N, int D, float alpha,
                              float* s, float* s_inv, cudaStream_t st);

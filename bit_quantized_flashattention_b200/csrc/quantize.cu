@@ -61,68 +61,98 @@ __device__ __forceinline__ uint32_t quant_block16_lut(const float (&x)[16], cons
 
 // ---------------------------------------------------------------- Q and K
 
-// Rows of Q or K (quantized along D). blockIdx.y is the group: the G*N
+// One row-quantization job (Q or K, quantized along D). A group is the G*N
 // consecutive input rows that share a kv head (G = q heads per kv head for Q,
 // 1 for K), padded to whole 128-row tiles; padding rows only receive zero
-// scale words. Each lane owns one 8-element chunk of a row (so a warp
-// instruction reads 512 contiguous bytes) and walks the group's rows with a
-// block stride; its 8 smoothing factors stay in registers. The two halves of a
-// 16-element block sit in neighbouring lanes (one shuffle for the maximum), and
-// the 4 scale bytes of a 64-element K step are gathered by shuffles into one
-// 32-bit word of the MMA-ready atom.
+// scale words.
+struct RowJob {
+    const void* x;
+    const float* scale;       // smoothing factors [Hkv, D] or null
+    uint8_t* codes;
+    uint8_t* sfs;
+    unsigned rows_per_group;
+    unsigned tiles_per_group;
+    unsigned hkv;
+    unsigned blocks_per_group;  // CTAs sharing one group's rows
+};
+
+struct VJob {
+    const void* v;
+    uint8_t* vtc;
+    uint8_t* vts;
+    int nkv;
+    unsigned warps_per_group;
+};
+
+// Each lane owns one 8-element chunk of a row (a warp instruction reads 512
+// contiguous bytes); a CTA walks a contiguous range of its group's rows, four
+// row steps per iteration so that four loads per lane are in flight. The
+// lane's 8 smoothing factors stay in registers. The two halves of a
+// 16-element block sit in neighbouring lanes (one shuffle for the maximum),
+// and the 4 scale bytes of a 64-element K step are gathered by shuffles into
+// one 32-bit word of the MMA-ready atom.
 template <typename T, int D>
-__global__ void __launch_bounds__(256) quantize_rows_kernel(const T* __restrict__ x, const float* __restrict__ scale,
-                                                            uint8_t* __restrict__ codes, uint8_t* __restrict__ sfs,
-                                                            unsigned rows_per_group, unsigned tiles_per_group,
-                                                            unsigned hkv) {
+__device__ __forceinline__ void quantize_rows_cta(const RowJob& jb, unsigned cta, const float* lut) {
     constexpr unsigned CPR = D / 8;                        // chunks per row
-    constexpr unsigned RPB = 256 / CPR;                    // rows per block step
+    constexpr unsigned RPB = 256 / CPR;                    // rows per CTA step
+    constexpr unsigned UNROLL = 4;
     constexpr unsigned KS = D / 64;
-    __shared__ float lut[128];
-    build_rcp_lut(lut);
-    const unsigned grp = blockIdx.y;
+    const unsigned grp = cta / jb.blocks_per_group;
+    const unsigned part = cta % jb.blocks_per_group;
     const unsigned c = threadIdx.x % CPR;
-    const unsigned padded = tiles_per_group * 128;
+    const unsigned padded = jb.tiles_per_group * 128;
+    const unsigned steps = (padded + RPB - 1) / RPB;
+    const unsigned s0 = (unsigned)(((unsigned long long)steps * part) / jb.blocks_per_group);
+    const unsigned s1 = (unsigned)(((unsigned long long)steps * (part + 1)) / jb.blocks_per_group);
     float sc[8];
-    if (scale != nullptr) {
-        const float4* s4 = reinterpret_cast<const float4*>(scale + (size_t)(grp % hkv) * D + c * 8);
+    if (jb.scale != nullptr) {
+        const float4* s4 = reinterpret_cast<const float4*>(jb.scale + (size_t)(grp % jb.hkv) * D + c * 8);
         const float4 a = __ldg(s4), b = __ldg(s4 + 1);
         sc[0] = a.x; sc[1] = a.y; sc[2] = a.z; sc[3] = a.w;
         sc[4] = b.x; sc[5] = b.y; sc[6] = b.z; sc[7] = b.w;
     }
-    const T* xg = x + (size_t)grp * rows_per_group * D;
-    uint8_t* cg = codes + (size_t)grp * rows_per_group * (D / 2);
-    uint8_t* sg = sfs + (size_t)grp * tiles_per_group * KS * 512;
-    for (unsigned p = blockIdx.x * RPB + threadIdx.x / CPR; p - (threadIdx.x / CPR) < padded;
-         p += gridDim.x * RPB) {
-        const bool in_tile = p < padded;
-        const bool real = p < rows_per_group;
-        float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        if (real) {
-            unpack8<T>(*reinterpret_cast<const uint4*>(xg + (size_t)p * D + c * 8), v);
-            if (scale != nullptr) {
+    const T* xg = static_cast<const T*>(jb.x) + (size_t)grp * jb.rows_per_group * D;
+    uint8_t* cg = jb.codes + (size_t)grp * jb.rows_per_group * (D / 2);
+    uint8_t* sg = jb.sfs + (size_t)grp * jb.tiles_per_group * KS * 512;
+    const unsigned r_in = threadIdx.x / CPR;
+    for (unsigned st = s0; st < s1; st += UNROLL) {
+        uint4 raw[UNROLL];
+#pragma unroll
+        for (unsigned u = 0; u < UNROLL; ++u) {
+            const unsigned pp = (st + u) * RPB + r_in;
+            raw[u] = (st + u < s1 && pp < jb.rows_per_group)
+                         ? *reinterpret_cast<const uint4*>(xg + (size_t)pp * D + c * 8)
+                         : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (unsigned u = 0; u < UNROLL; ++u) {
+            const unsigned p = (st + u) * RPB + r_in;
+            const bool in_range = st + u < s1;             // warp-uniform
+            const bool real = in_range && p < jb.rows_per_group;
+            float v[8];
+            unpack8<T>(raw[u], v);
+            if (jb.scale != nullptr) {
 #pragma unroll
                 for (int i = 0; i < 8; ++i) v[i] = __fmul_rn(v[i], sc[i]);
             }
+            float amax = 0.0f;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
+            amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
+            const uint32_t sf = cvt_e4m3(__fmul_rn(amax, rn_one_sixth()));
+            const float r = lut[sf & 127u];
+            float y[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) y[i] = __fmul_rn(v[i], r);
+            const uint32_t w = cvt_e2m1x8(y[0], y[1], y[2], y[3], y[4], y[5], y[6], y[7]);
+            if (real) *reinterpret_cast<uint32_t*>(cg + (size_t)p * (D / 2) + c * 4) = w;
+            uint32_t word = ((c & 1u) == 0u) ? (sf << (8u * ((c >> 1) & 3u))) : 0u;
+            word |= __shfl_xor_sync(0xFFFFFFFFu, word, 2);
+            word |= __shfl_xor_sync(0xFFFFFFFFu, word, 4);
+            if (in_range && p < padded && (c & 7u) == 0u)
+                *reinterpret_cast<uint32_t*>(sg + ((size_t)(p >> 7) * KS + c / 8) * 512 + atom_offset(p & 127u)) =
+                    real ? word : 0u;
         }
-        float amax = 0.0f;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
-        amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
-        const uint32_t sf = cvt_e4m3(__fmul_rn(amax, rn_one_sixth()));
-        const float r = lut[sf & 127u];
-        float y[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) y[i] = __fmul_rn(v[i], r);
-        const uint32_t w = cvt_e2m1x8(y[0], y[1], y[2], y[3], y[4], y[5], y[6], y[7]);
-        if (real) *reinterpret_cast<uint32_t*>(cg + (size_t)p * (D / 2) + c * 4) = w;
-        // scale word of the 64-element K step: blocks 2k..2k+1 -> byte k
-        uint32_t word = ((c & 1u) == 0u) ? (sf << (8u * ((c >> 1) & 3u))) : 0u;
-        word |= __shfl_xor_sync(0xFFFFFFFFu, word, 2);
-        word |= __shfl_xor_sync(0xFFFFFFFFu, word, 4);
-        if (in_tile && (c & 7u) == 0u)
-            *reinterpret_cast<uint32_t*>(sg + ((size_t)(p >> 7) * KS + c / 8) * 512 + atom_offset(p & 127u)) =
-                real ? word : 0u;
     }
 }
 
@@ -137,23 +167,19 @@ __global__ void __launch_bounds__(256) quantize_rows_kernel(const T* __restrict_
 // warp per half also fills the padding rows of the scale atoms (row 64 = 1.0
 // for the normalizer column of P-Reordering, the rest 0).
 template <typename T, int D>
-__global__ void __launch_bounds__(256) quantize_v_kernel(const T* __restrict__ v, uint8_t* __restrict__ vtc,
-                                                         uint8_t* __restrict__ vts, int nkv) {
+__device__ __forceinline__ void quantize_v_warp(const VJob& jb, unsigned gw_all, const float* lut) {
     constexpr int NRB = (D + 127) / 128;
     constexpr unsigned CWARPS = D / 32;                    // warps per 64-token half (32 channels each)
-    __shared__ float lut[128];
-    build_rcp_lut(lut);
     const unsigned lane = threadIdx.x & 31u;
-    const unsigned gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;   // warp within the group
-    const unsigned nhalf = (unsigned)nkv / 64u;
-    if (gw >= nhalf * CWARPS) return;
-    const unsigned grp = blockIdx.y;
+    const unsigned grp = gw_all / jb.warps_per_group;
+    const unsigned gw = gw_all % jb.warps_per_group;
+    const int nkv = jb.nkv;
     const unsigned cw = gw % CWARPS;
     const unsigned hh = gw / CWARPS;                       // 64-token half over the sequence
     const unsigned cc = lane >> 2, tb = lane & 3u;
-    const unsigned d0 = cw * 32 + cc * 4;                  // first channel of this lane
-    const unsigned tok0 = hh * 64 + tb * 16;               // first token of this lane's block
-    const T* src = v + ((size_t)grp * nkv + tok0) * D + d0;
+    const unsigned d0 = cw * 32 + cc * 4;
+    const unsigned tok0 = hh * 64 + tb * 16;
+    const T* src = static_cast<const T*>(jb.v) + ((size_t)grp * nkv + tok0) * D + d0;
     uint2 raw[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) raw[i] = *reinterpret_cast<const uint2*>(src + (size_t)i * D);
@@ -166,21 +192,39 @@ __global__ void __launch_bounds__(256) quantize_v_kernel(const T* __restrict__ v
         uint32_t lo, hi;
         const uint32_t sf = quant_block16_lut(x, lut, lo, hi);
         const unsigned d = d0 + k;
-        *reinterpret_cast<uint2*>(vtc + ((size_t)grp * D + d) * (nkv / 2) + tok0 / 2) = make_uint2(lo, hi);
+        *reinterpret_cast<uint2*>(jb.vtc + ((size_t)grp * D + d) * (nkv / 2) + tok0 / 2) = make_uint2(lo, hi);
         uint32_t word = sf << (8u * tb);
         word |= __shfl_xor_sync(0xFFFFFFFFu, word, 1);
         word |= __shfl_xor_sync(0xFFFFFFFFu, word, 2);
         if (tb == 0) {
             const size_t atom = (((size_t)grp * (nkv / 128) + j) * NRB + (d >> 7)) * 2 + half;
-            *reinterpret_cast<uint32_t*>(vts + atom * 512 + atom_offset(d & 127u)) = word;
+            *reinterpret_cast<uint32_t*>(jb.vts + atom * 512 + atom_offset(d & 127u)) = word;
         }
     }
     if constexpr (D == 64) {
         if (cw == 0) {
             const size_t atom = ((size_t)grp * (nkv / 128) + j) * 2 + half;
             for (unsigned r = 64 + lane; r < 128; r += 32)
-                *reinterpret_cast<uint32_t*>(vts + atom * 512 + atom_offset(r)) = (r == 64) ? 0x38383838u : 0u;
+                *reinterpret_cast<uint32_t*>(jb.vts + atom * 512 + atom_offset(r)) = (r == 64) ? 0x38383838u : 0u;
         }
+    }
+}
+
+// One launch for the whole pass: CTAs [0, nq) quantize Q rows, [nq, nq + nk)
+// K rows, the rest V (8 warps per CTA).
+template <typename T, int D>
+__global__ void __launch_bounds__(256) quantize_qkv_kernel(RowJob q, RowJob k, VJob v, unsigned nq, unsigned nk,
+                                                           unsigned v_warps) {
+    __shared__ float lut[128];
+    build_rcp_lut(lut);
+    const unsigned b = blockIdx.x;
+    if (b < nq) {
+        quantize_rows_cta<T, D>(q, b, lut);
+    } else if (b < nq + nk) {
+        quantize_rows_cta<T, D>(k, b - nq, lut);
+    } else {
+        const unsigned gw = (b - nq - nk) * 8 + (threadIdx.x >> 5);
+        if (gw < v_warps) quantize_v_warp<T, D>(v, gw, lut);
     }
 }
 
@@ -225,81 +269,49 @@ __global__ void calib_finalize_kernel(float* __restrict__ s, float* __restrict__
 
 // ------------------------------------------------------------ launchers
 
-template <typename T>
-static cudaError_t launch_rows_t(const void* x, const float* scale, uint8_t* codes, uint8_t* sfs, long long n_groups,
-                                 int rows_per_group, int tiles_per_group, int hkv, int D, cudaStream_t st) {
-    if (n_groups > 65535) return cudaErrorInvalidConfiguration;
+template <typename T, int D>
+static cudaError_t launch_qkv_t(const QuantArgs& a, cudaStream_t st) {
     int dev = 0, sms = 148, occ = 1;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    cudaError_t e = cudaSuccess;
-    switch (D) {
-        case 64: e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, quantize_rows_kernel<T, 64>, 256, 0); break;
-        case 128: e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, quantize_rows_kernel<T, 128>, 256, 0); break;
-        default: e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, quantize_rows_kernel<T, 256>, 256, 0); break;
-    }
-    if (e != cudaSuccess || occ < 1) occ = 1;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, quantize_qkv_kernel<T, D>, 256, 0) != cudaSuccess || occ < 1)
+        occ = 1;
+    (void)occ;
+    (void)sms;
+    const long long n_grp = a.n_groups;
+    // small CTAs (at most 8 row steps of 256/(D/8) rows each): many CTAs per SM
+    // overlap one CTA's loads with another's arithmetic
     const long long rows_per_step = 256 / (D / 8);
-    const long long steps = ((long long)tiles_per_group * 128 + rows_per_step - 1) / rows_per_step;
-    // one resident wave: every CTA of the grid is on an SM at once
-    long long bx = ((long long)sms * occ) / n_groups;
-    if (bx > steps) bx = steps;
-    if (bx < 1) bx = 1;
-    const dim3 grid((unsigned)bx, (unsigned)n_groups);
-    const T* xp = static_cast<const T*>(x);
-    const unsigned rg = (unsigned)rows_per_group, tg = (unsigned)tiles_per_group, hk = (unsigned)hkv;
-    switch (D) {
-        case 64:
-            quantize_rows_kernel<T, 64><<<grid, 256, 0, st>>>(xp, scale, codes, sfs, rg, tg, hk);
-            break;
-        case 128:
-            quantize_rows_kernel<T, 128><<<grid, 256, 0, st>>>(xp, scale, codes, sfs, rg, tg, hk);
-            break;
-        case 256:
-            quantize_rows_kernel<T, 256><<<grid, 256, 0, st>>>(xp, scale, codes, sfs, rg, tg, hk);
-            break;
-        default:
-            return cudaErrorInvalidValue;
-    }
+    auto per_group = [&](long long padded_rows) -> long long {
+        if (padded_rows == 0) return 0;
+        const long long steps = (padded_rows + rows_per_step - 1) / rows_per_step;
+        return (steps + 7) / 8;
+    };
+    const long long rows_q = a.q != nullptr ? (long long)a.tiles_q * 128 : 0;
+    const long long rows_k = a.nkv;
+    const long long v_warps = n_grp * (a.nkv / 64) * (D / 32);
+    const long long v_ctas = (v_warps + 7) / 8;
+    RowJob jq{a.q, a.s, a.qc, a.qs, (unsigned)(a.G * a.nq), (unsigned)a.tiles_q, (unsigned)a.hkv,
+              (unsigned)per_group(rows_q)};
+    RowJob jk{a.k, a.s_inv, a.kc, a.ks, (unsigned)a.nkv, (unsigned)(a.nkv / 128), (unsigned)a.hkv,
+              (unsigned)per_group(rows_k)};
+    VJob jv{a.v, a.vtc, a.vts, a.nkv, (unsigned)((a.nkv / 64) * (D / 32))};
+    const long long nq = a.q != nullptr ? n_grp * jq.blocks_per_group : 0;
+    const long long nk = n_grp * jk.blocks_per_group;
+    const long long total = nq + nk + v_ctas;
+    if (total > 0x7FFFFFFFLL) return cudaErrorInvalidConfiguration;
+    quantize_qkv_kernel<T, D><<<(unsigned)total, 256, 0, st>>>(jq, jk, jv, (unsigned)nq, (unsigned)nk,
+                                                                (unsigned)v_warps);
     return cudaGetLastError();
 }
 
-cudaError_t launch_quantize_rows(bool bf16, const void* x, const float* scale, uint8_t* codes, uint8_t* sfs,
-                                 long long n_groups, int rows_per_group, int tiles_per_group, int hkv, int D,
-                                 cudaStream_t st) {
-    if (bf16)
-        return launch_rows_t<__nv_bfloat16>(x, scale, codes, sfs, n_groups, rows_per_group, tiles_per_group, hkv, D,
-                                            st);
-    return launch_rows_t<__half>(x, scale, codes, sfs, n_groups, rows_per_group, tiles_per_group, hkv, D, st);
-}
-
-template <typename T>
-static cudaError_t launch_v_t(const void* v, uint8_t* vtc, uint8_t* vts, long long n_groups, int nkv, int D,
-                              cudaStream_t st) {
-    if (n_groups > 65535) return cudaErrorInvalidConfiguration;
-    const long long warps = (long long)(nkv / 64) * (D / 32);
-    const dim3 grid((unsigned)((warps * 32 + 255) / 256), (unsigned)n_groups);
-    const T* vp = static_cast<const T*>(v);
-    switch (D) {
-        case 64:
-            quantize_v_kernel<T, 64><<<grid, 256, 0, st>>>(vp, vtc, vts, nkv);
-            break;
-        case 128:
-            quantize_v_kernel<T, 128><<<grid, 256, 0, st>>>(vp, vtc, vts, nkv);
-            break;
-        case 256:
-            quantize_v_kernel<T, 256><<<grid, 256, 0, st>>>(vp, vtc, vts, nkv);
-            break;
-        default:
-            return cudaErrorInvalidValue;
+cudaError_t launch_quantize_qkv(const QuantArgs& a, cudaStream_t st) {
+    switch (a.D) {
+        case 64: return a.bf16 ? launch_qkv_t<__nv_bfloat16, 64>(a, st) : launch_qkv_t<__half, 64>(a, st);
+        case 128: return a.bf16 ? launch_qkv_t<__nv_bfloat16, 128>(a, st) : launch_qkv_t<__half, 128>(a, st);
+        case 256: return a.bf16 ? launch_qkv_t<__nv_bfloat16, 256>(a, st) : launch_qkv_t<__half, 256>(a, st);
+        default: return cudaErrorInvalidValue;
     }
-    return cudaGetLastError();
-}
-
-cudaError_t launch_quantize_v(bool bf16, const void* v, uint8_t* vtc, uint8_t* vts, long long n_groups, int nkv, int D,
-                              cudaStream_t st) {
-    if (bf16) return launch_v_t<__nv_bfloat16>(v, vtc, vts, n_groups, nkv, D, st);
-    return launch_v_t<__half>(v, vtc, vts, n_groups, nkv, D, st);
 }
 
 template <typename T>
