@@ -10,10 +10,11 @@
 // head after head (GQA), so a tile may mix heads when Nq is small. Warp roles:
 //   warp 0      TMA / bulk-copy producer: Q_hat tiles once, then K_hat and
 //               V_hat^T tiles (128 keys) with their scale atoms, 3-stage rings
-//   warp 1      TMEM owner; one thread issues S = Q_hat K_hat^T (and moves the
-//               Q and K scale atoms shared->TMEM with tcgen05.cp)
-//   warp 2      one thread issues O += P_hat V_hat (P and V scale atoms); the
-//               two issuers touch disjoint TMEM and wait independently
+//   warp 1      TMEM owner; issues S = Q_hat K_hat^T (and moves the Q and K
+//               scale atoms shared->TMEM with tcgen05.cp)
+//   warp 2      issues O += P_hat V_hat (P and V scale atoms); the two issuers
+//               touch disjoint TMEM and wait independently; in both the whole
+//               warp runs the loop and lane 0 issues the tcgen05 instructions
 //   warps 4..   one softmax warpgroup per query tile, thread t owns row t:
 //               block maxima of S, running max, P = 2^(S*c - RN(m*c)),
 //               P quantized per 16 keys to E2M1 + E4M3 in registers, O rescaled
@@ -286,12 +287,29 @@ __global__ void __launch_bounds__(Cfg<D, PREORDER>::THREADS, 1)
         // ----------------------------------------------------- S MMA issuer
         // S = Q_hat(qt) K_hat(j)^T in the order (j=0,A) (0,B) (1,A) (1,B) ... through
         // the one S buffer; each needs its K tile and the previous S consumed.
-        if (lane == 0) {
-            const uint32_t idesc_s = idesc_fp4_block16(128);
-            auto sf_desc = [&](uint32_t off) { return smem_desc(smem_u32(smem + off), 0u, 128u, 0u); };
-            bool ok = mbar_wait(&bars->q_full, 0, ctl);
-            if (ok) {
-                tc_fence_after();
+        // The whole warp runs the loop, so its values stay warp-uniform, and
+        // lane 0 issues every tcgen05 instruction (a commit covers only the
+        // issuing thread's operations). The K scales of the next tile go to
+        // TMEM as soon as the current tile's MMAs are issued: only the MMAs
+        // sit between a freed S buffer and the next S.
+        const uint32_t idesc_s = idesc_fp4_block16(128);
+        const uint32_t sbase = smem_u32(smem);
+        auto sf_desc = [&](uint32_t off) { return smem_desc(sbase + off, 0u, 128u, 0u); };
+        auto copy_sfk = [&](int st) {
+#pragma unroll
+            for (int s = 0; s < C::KS; ++s)
+                tmem_cp_scale_atom(tmem + C::COL_SFK + 4 * s, sf_desc(C::OFF_SFK + st * C::SFQK_BYTES + 512 * s));
+        };
+        uint64_t qdesc[NQT][C::KS];
+#pragma unroll
+        for (int qt = 0; qt < NQT; ++qt)
+#pragma unroll
+            for (int s = 0; s < C::KS; ++s)
+                qdesc[qt][s] = smem_desc(sbase + C::OFF_Q + qt * C::Q_BYTES + 32u * s, 16u, C::QK_SBO, C::QK_SWZ);
+        bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(&bars->q_full, 0, ctl));
+        if (ok) {
+            tc_fence_after();
+            if (lane == 0) {
                 for (int qt = 0; qt < n_qt; ++qt) {
 #pragma unroll
                     for (int s = 0; s < C::KS; ++s)
@@ -299,66 +317,91 @@ __global__ void __launch_bounds__(Cfg<D, PREORDER>::THREADS, 1)
                                            sf_desc(C::OFF_SFQ + qt * C::SFQK_BYTES + 512 * s));
                 }
             }
-            int prev_qt = -1, prev_j = 0;
-            for (int j = 0; j < n_tiles_max && ok; ++j) {
-                const int st = j % kStages;
-                if (!mbar_wait(&bars->k_full[st], (j / kStages) & 1, ctl)) { ok = false; break; }
-                bool first = true;
+            __syncwarp();
+        }
+        if (ok && n_tiles_max > 0) {
+            ok = __all_sync(0xFFFFFFFFu, mbar_wait(&bars->k_full[0], 0, ctl));
+            if (ok) {
+                tc_fence_after();
+                if (lane == 0) copy_sfk(0);
+                __syncwarp();
+            }
+        }
+        int prev_qt = -1, prev_j = 0;
+        for (int j = 0; j < n_tiles_max && ok; ++j) {
+            const int st = j % kStages;
+            const uint32_t kaddr = sbase + C::OFF_K + st * C::K_BYTES;
 #pragma unroll
-                for (int qt = 0; qt < NQT; ++qt) {
-                    if (j >= (qt == 0 ? n_tiles0 : n_tiles1)) continue;
-                    if (prev_qt >= 0 && !mbar_wait(&bars->s_free[prev_qt], prev_j & 1, ctl)) { ok = false; break; }
-                    tc_fence_after();
-                    if (first) {
-#pragma unroll
-                        for (int s = 0; s < C::KS; ++s)
-                            tmem_cp_scale_atom(tmem + C::COL_SFK + 4 * s,
-                                               sf_desc(C::OFF_SFK + st * C::SFQK_BYTES + 512 * s));
-                        first = false;
-                    }
-                    const uint32_t kbuf = C::OFF_K + st * C::K_BYTES;
+            for (int qt = 0; qt < NQT; ++qt) {
+                if (j >= (qt == 0 ? n_tiles0 : n_tiles1)) continue;
+                if (prev_qt >= 0 && !__all_sync(0xFFFFFFFFu, mbar_wait(&bars->s_free[prev_qt], prev_j & 1, ctl))) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                if (lane == 0) {
 #pragma unroll
                     for (int s = 0; s < C::KS; ++s) {
-                        const uint64_t a =
-                            smem_desc(smem_u32(smem + C::OFF_Q + qt * C::Q_BYTES) + 32u * s, 16u, C::QK_SBO, C::QK_SWZ);
-                        const uint64_t b = smem_desc(smem_u32(smem + kbuf) + 32u * s, 16u, C::QK_SBO, C::QK_SWZ);
-                        mma_fp4_block16(tmem + C::COL_S, a, b, idesc_s, tmem + C::COL_SFQ + qt * 4 * C::KS + 4 * s,
-                                        tmem + C::COL_SFK + 4 * s, s > 0 ? 1u : 0u);
+                        const uint64_t b = smem_desc(kaddr + 32u * s, 16u, C::QK_SBO, C::QK_SWZ);
+                        mma_fp4_block16(tmem + C::COL_S, qdesc[qt][s], b, idesc_s,
+                                        tmem + C::COL_SFQ + qt * 4 * C::KS + 4 * s, tmem + C::COL_SFK + 4 * s,
+                                        s > 0 ? 1u : 0u);
                     }
                     tc_commit(&bars->s_full[qt]);
-                    prev_qt = qt;
-                    prev_j = j;
                 }
-                if (ok) tc_commit(&bars->k_empty[st]);
+                __syncwarp();
+                prev_qt = qt;
+                prev_j = j;
             }
-            // wait until every MMA / copy issued above has finished
-            tc_commit(&bars->drain[0]);
-            mbar_wait_drain(&bars->drain[0], 0, p.wait_limit_ns);
+            if (!ok) break;
+            if (lane == 0) tc_commit(&bars->k_empty[st]);
+            __syncwarp();
+            // K scales of the next tile (they replace this tile's in TMEM only
+            // after its MMAs: one thread's tcgen05 operations run in order)
+            if (j + 1 < n_tiles_max) {
+                const int st1 = (j + 1) % kStages;
+                if (!__all_sync(0xFFFFFFFFu, mbar_wait(&bars->k_full[st1], ((j + 1) / kStages) & 1, ctl))) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                if (lane == 0) copy_sfk(st1);
+                __syncwarp();
+            }
         }
+        // wait until every MMA / copy issued above has finished
+        if (lane == 0) tc_commit(&bars->drain[0]);
+        __syncwarp();
+        mbar_wait_drain(&bars->drain[0], 0, p.wait_limit_ns);
     } else if (warp == 2) {
         // ---------------------------------------------------- PV MMA issuer
-        // O(qt) += P_hat(qt, j) V_hat(j) in the order (0,A) (0,B) (1,A) (1,B) ...
-        if (lane == 0) {
-            auto sf_desc = [&](uint32_t off) { return smem_desc(smem_u32(smem + off), 0u, 128u, 0u); };
-            bool ok = true;
-            if constexpr (PREORDER && D >= 128) {
+        // O(qt) += P_hat(qt, j) V_hat(j) in the order (0,A) (0,B) (1,A) (1,B) ...;
+        // the whole warp runs the loop, lane 0 issues.
+        const uint32_t sbase = smem_u32(smem);
+        auto sf_desc = [&](uint32_t off) { return smem_desc(sbase + off, 0u, 128u, 0u); };
+        bool ok = true;
+        if constexpr (PREORDER && D >= 128) {
+            if (lane == 0) {
 #pragma unroll
                 for (int s = 0; s < 2; ++s)
                     tmem_cp_scale_atom(tmem + C::COL_SFV + s * C::SFV_PER_KS + 4 * C::NRB, sf_desc(C::OFF_ONES));
             }
-            for (int j = 0; j < n_tiles_max && ok; ++j) {
-                const int st = j % kStages;
-                if (!mbar_wait(&bars->v_full[st], (j / kStages) & 1, ctl)) { ok = false; break; }
-                const uint32_t vbuf = C::OFF_V + st * C::V_STRIDE;
-                const uint32_t sfv = C::OFF_SFV + st * C::SFV_BYTES;
-                bool first = true;
+            __syncwarp();
+        }
+        for (int j = 0; j < n_tiles_max && ok; ++j) {
+            const int st = j % kStages;
+            if (!__all_sync(0xFFFFFFFFu, mbar_wait(&bars->v_full[st], (j / kStages) & 1, ctl))) { ok = false; break; }
+            const uint32_t vaddr = sbase + C::OFF_V + st * C::V_STRIDE;
+            const uint32_t sfv = C::OFF_SFV + st * C::SFV_BYTES;
+            bool first = true;
 #pragma unroll
-                for (int qt = 0; qt < NQT; ++qt) {
-                    if (j >= (qt == 0 ? n_tiles0 : n_tiles1)) continue;
-                    if (!mbar_wait(&bars->p_full[qt][j & 1], (j >> 1) & 1, ctl)) { ok = false; break; }
-                    tc_fence_after();
-                    const uint32_t pbuf = C::OFF_P + (qt * 2 + (j & 1)) * C::P_BYTES;
-                    const uint32_t sfp = C::OFF_SFP + (qt * 2 + (j & 1)) * C::SFP_BYTES;
+            for (int qt = 0; qt < NQT; ++qt) {
+                if (j >= (qt == 0 ? n_tiles0 : n_tiles1)) continue;
+                if (!__all_sync(0xFFFFFFFFu, mbar_wait(&bars->p_full[qt][j & 1], (j >> 1) & 1, ctl))) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t paddr = sbase + C::OFF_P + (qt * 2 + (j & 1)) * C::P_BYTES;
+                const uint32_t sfp = C::OFF_SFP + (qt * 2 + (j & 1)) * C::SFP_BYTES;
+                if (lane == 0) {
 #pragma unroll
                     for (int s = 0; s < 2; ++s) {
                         tmem_cp_scale_atom(tmem + C::COL_SFP + qt * 8 + 4 * s, sf_desc(sfp + 512 * s));
@@ -369,31 +412,35 @@ __global__ void __launch_bounds__(Cfg<D, PREORDER>::THREADS, 1)
                                                    sf_desc(sfv + (rb * 2 + s) * 512));
                         }
                     }
-                    first = false;
                     const uint32_t o = tmem + C::COL_O + qt * C::NO;
 #pragma unroll
                     for (int s = 0; s < 2; ++s) {
-                        const uint64_t a = smem_desc(smem_u32(smem + pbuf) + 32u * s, 16u, 512u, 4u);
+                        const uint64_t a = smem_desc(paddr + 32u * s, 16u, 512u, 4u);
                         const uint32_t acc = (j > 0 || s > 0) ? 1u : 0u;
                         const uint32_t sfa = tmem + C::COL_SFP + qt * 8 + 4 * s;
                         const uint32_t sfb = tmem + C::COL_SFV + s * C::SFV_PER_KS;
                         if constexpr (D == 256 && PREORDER) {
-                            const uint64_t b0 = smem_desc(smem_u32(smem + vbuf) + 32u * s, 16u, 512u, 4u);
-                            const uint64_t b1 = smem_desc(smem_u32(smem + vbuf + 128 * 64) + 32u * s, 16u, 512u, 4u);
+                            const uint64_t b0 = smem_desc(vaddr + 32u * s, 16u, 512u, 4u);
+                            const uint64_t b1 = smem_desc(vaddr + 128 * 64 + 32u * s, 16u, 512u, 4u);
                             mma_fp4_block16(o, a, b0, idesc_fp4_block16(128), sfa, sfb, acc);
                             mma_fp4_block16(o + 128, a, b1, idesc_fp4_block16(144), sfa, sfb + 4, acc);
                         } else {
-                            const uint64_t b = smem_desc(smem_u32(smem + vbuf) + 32u * s, 16u, 512u, 4u);
+                            const uint64_t b = smem_desc(vaddr + 32u * s, 16u, 512u, 4u);
                             mma_fp4_block16(o, a, b, idesc_fp4_block16(C::NO), sfa, sfb, acc);
                         }
                     }
                     tc_commit(&bars->o_done[qt]);
                 }
-                if (ok) tc_commit(&bars->v_empty[st]);
+                __syncwarp();
+                first = false;
             }
-            tc_commit(&bars->drain[1]);
-            mbar_wait_drain(&bars->drain[1], 0, p.wait_limit_ns);
+            if (!ok) break;
+            if (lane == 0) tc_commit(&bars->v_empty[st]);
+            __syncwarp();
         }
+        if (lane == 0) tc_commit(&bars->drain[1]);
+        __syncwarp();
+        mbar_wait_drain(&bars->drain[1], 0, p.wait_limit_ns);
     } else if (warp >= kSmWarp0) {
         // ------------------------------------------------------------ softmax
         const int qt = (warp - kSmWarp0) >> 2;             // query tile of this warpgroup
