@@ -103,6 +103,18 @@ def profiled_traffic(cfg):
         return None
 
 
+def max_over_ranks(x: float, device) -> float:
+    """Maximum of x over the ranks of the default process group (x itself on one
+    rank). Every rank calls it at the same points, error checks included."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def dist_env():
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -268,9 +280,9 @@ def run_ours(args):
     for _ in range(max(args.warmup, 3)):
         step()
     torch.cuda.synchronize()
-    st = H.get_status(wsp)
+    st = max_over_ranks(H.get_status(wsp), dev)
     if st != 0:
-        raise RuntimeError(f"kernel status {st} during warm-up")
+        raise RuntimeError(f"kernel status {int(st)} during warm-up (max over ranks)")
 
     # The timed loop replays each of the step's two launches from a CUDA graph
     # (captured after the warm-up calls): the device timeline then holds the
@@ -304,14 +316,10 @@ def run_ours(args):
     step_ms = [a.elapsed_time(c) for a, _, c in ev]
     attn_ms = [b.elapsed_time(c) for _, b, c in ev]
     quant_ms = [a.elapsed_time(b) for a, b, _ in ev]
-    total_ms = float(sum(step_ms))
-    if ws > 1:
-        t = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
-    st = H.get_status(wsp)
+    total_ms = max_over_ranks(float(sum(step_ms)), dev)
+    st = max_over_ranks(H.get_status(wsp), dev)
     if st != 0:
-        raise RuntimeError(f"kernel status {st} in the timed region")
+        raise RuntimeError(f"kernel status {int(st)} in the timed region (max over ranks)")
 
     flops = cfg.flops()
     value = ws * flops * n / (total_ms * 1e-3) / 1e12
@@ -373,16 +381,10 @@ def run_ours(args):
     s_out.wait_stream(s_cp)
     t_end.record(s_out)
     torch.cuda.synchronize()
-    for w_ in dws:
-        st = H.get_status(w_)
-        if st != 0:
-            raise RuntimeError(f"kernel status {st} in the end-to-end loop")
-    e2e_ms = [t_beg.elapsed_time(t_end)]
-    e2e_total = float(sum(e2e_ms))
-    if ws > 1:
-        t = torch.tensor([e2e_total], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_total = float(t.item())
+    st = max_over_ranks(max(H.get_status(w_) for w_ in dws), dev)
+    if st != 0:
+        raise RuntimeError(f"kernel status {int(st)} in the end-to-end loop (max over ranks)")
+    e2e_total = max_over_ranks(t_beg.elapsed_time(t_end), dev)
     h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv))
     d2h = ho[0].numel() * ho[0].element_size() + hl[0].numel() * hl[0].element_size()
 
