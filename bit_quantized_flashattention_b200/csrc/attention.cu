@@ -248,6 +248,11 @@ __global__ void __launch_bounds__(Cfg<D, PREORDER>::THREADS, 1)
 
     if (warp == 0) {
         // ---------------------------------------------------------- producer
+        // The set-up above overlaps the end of the previous kernel in the
+        // stream (programmatic dependent launch); the packed operands are read
+        // only after it has completed. Every other read of those operands
+        // goes through this warp's copies.
+        grid_dependency_wait();
         if (lane == 0 && !p.stall_loads) {
             int issued = 0;
             bool ok = true;
@@ -616,8 +621,17 @@ static cudaError_t launch_one(const CUtensorMap* q, const CUtensorMap* k, const 
     auto kern = attn_fwd_kernel<D, PRE, CAUSAL, OUT, DUMP>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    kern<<<p.n_work, C::THREADS, C::SMEM_BYTES, st>>>(*q, *k, *v, p);
-    return cudaGetLastError();
+    cudaLaunchConfig_t lc{};
+    lc.gridDim = dim3((unsigned)p.n_work);
+    lc.blockDim = dim3(C::THREADS);
+    lc.dynamicSmemBytes = C::SMEM_BYTES;
+    lc.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    lc.attrs = attr;
+    lc.numAttrs = 1;
+    return cudaLaunchKernelEx(&lc, kern, *q, *k, *v, p);
 }
 
 template <int D, bool PRE, bool CAUSAL, int OUT>

@@ -216,6 +216,9 @@ template <typename T, int D>
 __global__ void __launch_bounds__(256) quantize_qkv_kernel(RowJob q, RowJob k, VJob v, unsigned nq, unsigned nk,
                                                            unsigned v_warps) {
     __shared__ float lut[128];
+    // the next kernel (attention) may be scheduled as these CTAs retire; it
+    // waits for this grid's completion before reading the packed operands
+    launch_dependents();
     build_rcp_lut(lut);
     const unsigned b = blockIdx.x;
     if (b < nq) {
