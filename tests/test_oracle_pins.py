@@ -355,3 +355,78 @@ def test_smooth_qk_reduces_score_error_on_outlier_channels():
     # same scores up to quantization error either way; smoothing lowers that error
     assert errs["on"] < errs["off"]
     assert errs["on"] < 0.1 * np.sqrt(np.mean(exact ** 2))
+
+
+# ------------------------------------------------ Smooth-QK is an equivalence
+
+def _exactly_smoothable(rng, B, Hq, Hkv, N, D):
+    """Q = g * 2^-e, K = h * 2^e with g, h on the E2M1 grid, e per (kv head,
+    channel), and a +-6 in every 16-element block of every row. Calibration then
+    gives s = 2^e exactly, the smoothed rows are g and h, and 4-bit quantization
+    of g and h is lossless (every block's scale is 1)."""
+    G = Hq // Hkv
+    grid = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
+    e = rng.integers(-3, 4, (Hkv, D))
+
+    def rows(H, n, group):
+        x = rng.choice(grid, (B, H, n, D)) * rng.choice([-1.0, 1.0], (B, H, n, D))
+        for blk in range(D // 16):
+            x[:, :, np.arange(n), blk * 16 + np.arange(n) % 16] = 6.0 * rng.choice([-1.0, 1.0], (B, H, n))
+        return x
+
+    g, h = rows(Hq, N, G), rows(Hkv, N, 1)
+    eq = np.repeat(e, G, axis=0)[None, :, None, :]
+    q = (g * 2.0 ** -eq).astype(np.float32)
+    k = (h * 2.0 ** e[None, :, None, :]).astype(np.float32)
+    return q, k, e
+
+
+@pytest.mark.parametrize("shape", [(2, 4, 2, 32, 64), (1, 8, 2, 48, 128), (1, 2, 1, 16, 256)])
+def test_smooth_qk_leaves_qk_unchanged_exactly(shape):
+    """HiFA4 abstract: Smooth-QK is an equivalent per-channel rescaling (Q*s,
+    K/s), so QK^T is unchanged in exact arithmetic. On inputs where smoothing
+    makes quantization lossless, the oracle's whole smoothing path (calibration,
+    Q*s and K*s_inv per kv head and channel, quantization, QK^T) must give the
+    exact unsmoothed scores bit for bit; without smoothing the same inputs are
+    quantized lossily, so the check has teeth."""
+    B, Hq, Hkv, N, D = shape
+    G = Hq // Hkv
+    rng = np.random.default_rng(31)
+    q, k, e = _exactly_smoothable(rng, B, Hq, Hkv, N, D)
+    s, si = oracle.calibrate(q, k, 0.5)
+    assert np.array_equal(s, (2.0 ** e).astype(np.float32))
+    v = np.zeros_like(k)
+    on = oracle.quantize_qkv(q, k, v, s, si)
+    off = oracle.quantize_qkv(q, k, v)
+    exact = np.einsum("bhid,bhjd->bhij", q.astype(np.float64), np.repeat(k.astype(np.float64), G, axis=1))
+    n_off_exact = 0
+    for b in range(B):
+        for hh in range(Hq):
+            for i in (0, N // 2, N - 1):
+                row = (b * Hq + hh) * N + i
+                want = exact[b, hh, i].astype(np.float32)
+                assert np.array_equal(oracle.qk_row(on, Hq, Hkv, N, N, D, row), want), (b, hh, i)
+                n_off_exact += np.array_equal(oracle.qk_row(off, Hq, Hkv, N, N, D, row), want)
+    assert n_off_exact == 0
+
+
+def test_smooth_qk_factors_are_reciprocal_pairs_on_outlier_tensors():
+    """On the tiny config's outlier tensors and on a GQA shape the calibration
+    returns s_inv = RN(1/s), so (Q*s)(K*s_inv)^T equals QK^T up to one rounding
+    of s*s_inv per channel (relative 2^-24), far below the 4-bit error."""
+    cfg = W.get(1)
+    q1, k1, _ = W.full(cfg)
+    rng = np.random.default_rng(32)
+    q2 = rng.standard_normal((2, 8, 64, 128)).astype(np.float32)
+    k2 = (rng.standard_normal((2, 2, 64, 128)) * rng.lognormal(0, 1, (1, 2, 1, 128))).astype(np.float32)
+    for q, k in ((q1, k1), (q2, k2)):
+        s, si = oracle.calibrate(q, k)
+        prod = s.astype(np.float64) * si.astype(np.float64)
+        assert np.all(np.abs(prod - 1.0) <= 2.0 ** -24)
+        assert np.all(si == (1.0 / s.astype(np.float64)).astype(np.float32))
+        G = q.shape[1] // k.shape[1]
+        sq = np.repeat(s.astype(np.float64), G, axis=0)[None, :, None, :]
+        kk = np.repeat(k.astype(np.float64), G, axis=1)
+        ref = np.einsum("bhid,bhjd->bhij", q.astype(np.float64), kk)
+        sm = np.einsum("bhid,bhjd->bhij", q * sq, kk * np.repeat(si.astype(np.float64), G, axis=0)[None, :, None, :])
+        assert np.abs(sm - ref).max() <= 1e-6 * np.abs(ref).max()
