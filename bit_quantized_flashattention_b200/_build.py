@@ -9,7 +9,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libhifa4.so")
 SOURCES = ["api.cu", "quantize.cu", "attention.cu", "noalloc.cu"]
-HEADERS = ["hifa4_device.cuh", "hifa4_kernels.h", os.path.join("..", "..", "include", "hifa4.h")]
+HEADERS = ["hifa4_device.cuh", "hifa4_kernels.h", "api_internal.h", os.path.join("..", "..", "include", "hifa4.h")]
 
 
 def nvcc() -> str:

@@ -10,6 +10,7 @@
 #include <cstring>
 
 #include "../../include/hifa4.h"
+#include "api_internal.h"
 #include "hifa4_kernels.h"
 
 using namespace hifa4;
@@ -79,36 +80,51 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t inner_bytes, uint64_t r
 
 thread_local cudaError_t g_last_cuda_error = cudaSuccess;
 
-hifa4_status from_cuda(cudaError_t e) {
+}  // namespace
+
+hifa4_status hifa4::from_cuda(cudaError_t e) {
     if (e == cudaSuccess) return HIFA4_OK;
     g_last_cuda_error = e;
     return HIFA4_ERR_CUDA;
 }
 
-hifa4_status attention_impl(const hifa4_packed* in, int B, int Hq, int Hkv, int Nq, int Nkv, int D, float sm_scale,
-                            unsigned flags, hifa4_norm_mode norm, void* o, hifa4_dtype o_dtype, float* lse,
-                            uint8_t* p_codes, uint8_t* p_sf, bool dump, void* workspace, hifa4_stream_t stream) {
-    if (in == nullptr || o == nullptr || workspace == nullptr) return HIFA4_ERR_INVALID_ARG;
+hifa4_status hifa4::check_attention_args(const hifa4_packed* in, int B, int Hq, int Hkv, int Nq, int Nkv, int D,
+                                         float sm_scale, unsigned flags, hifa4_norm_mode norm, const void* o,
+                                         hifa4_dtype o_dtype, const float* lse) {
+    if (in == nullptr || o == nullptr) return HIFA4_ERR_INVALID_ARG;
     if (!shape_ok(B, Hq, Hkv, Nq, Nkv, D)) return HIFA4_ERR_UNSUPPORTED;
     if (!(sm_scale > 0.0f) || !std::isfinite(sm_scale)) return HIFA4_ERR_INVALID_ARG;
     if ((flags & ~(unsigned)HIFA4_CAUSAL) != 0) return HIFA4_ERR_INVALID_ARG;
-    const bool causal = (flags & HIFA4_CAUSAL) != 0;
-    if (causal && Nq > Nkv) return HIFA4_ERR_UNSUPPORTED;
+    if ((flags & HIFA4_CAUSAL) != 0 && Nq > Nkv) return HIFA4_ERR_UNSUPPORTED;
     if (norm != HIFA4_NORM_P_REORDER && norm != HIFA4_NORM_HIGH_PRECISION_L) return HIFA4_ERR_INVALID_ARG;
     if (o_dtype != HIFA4_F16 && o_dtype != HIFA4_BF16 && o_dtype != HIFA4_F32) return HIFA4_ERR_INVALID_ARG;
     const void* ptrs[6] = {in->qc, in->qs, in->kc, in->ks, in->vtc, in->vts};
     for (const void* q : ptrs)
         if (q == nullptr || !aligned16(q)) return HIFA4_ERR_INVALID_ARG;
-    if (!aligned16(o) || !aligned16(workspace) || (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u)))
-        return HIFA4_ERR_INVALID_ARG;
-    if (dump && (p_codes == nullptr || p_sf == nullptr || !aligned16(p_codes) || !aligned16(p_sf)))
-        return HIFA4_ERR_INVALID_ARG;
+    if (!aligned16(o) || (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u))) return HIFA4_ERR_INVALID_ARG;
     const long long rows_q = (long long)B * Hq * Nq, rows_k = (long long)B * Hkv * Nkv, rows_v = (long long)B * Hkv * D;
     if (rows_q > INT32_MAX || rows_k > INT32_MAX || rows_v > INT32_MAX) return HIFA4_ERR_UNSUPPORTED;
     const Sizes sz = sizes_of(B, Hq, Hkv, Nq, Nkv, D);
     const int nqt = D == 256 ? 1 : 2;              // query tiles per CTA (see attention.cu)
+    if ((long long)B * Hkv * ((sz.Tq + nqt - 1) / nqt) > INT32_MAX) return HIFA4_ERR_UNSUPPORTED;
+    return HIFA4_OK;
+}
+
+namespace {
+
+hifa4_status attention_impl(const hifa4_packed* in, int B, int Hq, int Hkv, int Nq, int Nkv, int D, float sm_scale,
+                            unsigned flags, hifa4_norm_mode norm, void* o, hifa4_dtype o_dtype, float* lse,
+                            uint8_t* p_codes, uint8_t* p_sf, bool dump, void* workspace, hifa4_stream_t stream) {
+    const hifa4_status chk = check_attention_args(in, B, Hq, Hkv, Nq, Nkv, D, sm_scale, flags, norm, o, o_dtype, lse);
+    if (chk != HIFA4_OK) return chk;
+    if (workspace == nullptr || !aligned16(workspace)) return HIFA4_ERR_INVALID_ARG;
+    if (dump && (p_codes == nullptr || p_sf == nullptr || !aligned16(p_codes) || !aligned16(p_sf)))
+        return HIFA4_ERR_INVALID_ARG;
+    const bool causal = (flags & HIFA4_CAUSAL) != 0;
+    const long long rows_q = (long long)B * Hq * Nq, rows_k = (long long)B * Hkv * Nkv, rows_v = (long long)B * Hkv * D;
+    const Sizes sz = sizes_of(B, Hq, Hkv, Nq, Nkv, D);
+    const int nqt = D == 256 ? 1 : 2;              // query tiles per CTA (see attention.cu)
     const long long n_work = (long long)B * Hkv * ((sz.Tq + nqt - 1) / nqt);
-    if (n_work > INT32_MAX) return HIFA4_ERR_UNSUPPORTED;
 
     const CUtensorMapSwizzle swz_qk =
         D == 64 ? CU_TENSOR_MAP_SWIZZLE_32B : (D == 128 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B);
@@ -166,7 +182,7 @@ size_t hifa4_packed_bytes(int B, int Hq, int Hkv, int Nq, int Nkv, int D, size_t
 
 size_t hifa4_workspace_bytes(int B, int Hq, int Hkv, int Nq, int Nkv, int D) {
     (void)B; (void)Hq; (void)Hkv; (void)Nq; (void)Nkv; (void)D;
-    return 256;
+    return 256;                                    // the status word, padded to 256 bytes
 }
 
 hifa4_status hifa4_calibrate_smooth(const void* q, const void* k, hifa4_dtype dtype, int B, int Hq, int Hkv, int N,
