@@ -92,9 +92,9 @@ typedef struct {
  * to out[6] (may be NULL). Returns their sum, or 0 for an unsupported shape. */
 size_t hifa4_packed_bytes(int B, int Hq, int Hkv, int Nq, int Nkv, int D, size_t out[6]);
 
-/* Bytes of the device workspace hifa4_attention_fwd needs: a status word and
- * a work counter. The caller zeroes it once after allocating; the kernels
- * leave the counter at zero when they finish. */
+/* Bytes of the device workspace hifa4_attention_fwd needs: one status word
+ * (padded to 256 bytes). The caller zeroes it once after allocating; a kernel
+ * writes it only when a bounded wait expires, and hifa4_get_status clears it. */
 size_t hifa4_workspace_bytes(int B, int Hq, int Hkv, int Nq, int Nkv, int D);
 
 /* Smooth-QK calibration (HiFA4 abstract: "calibration-static per-channel
@@ -169,10 +169,13 @@ hifa4_status hifa4_attention_fwd_debug(const hifa4_packed* in, int B, int Hq, in
  * paper has no counterpart of this call; it is an integration aid.)
  * Arguments, layouts and results are those of hifa4_attention_fwd.
  *  - The first call on each device looks up the array's device address
- *    (cudaGetSymbolAddress, no allocation) with that device current; make that
- *    first call before any stream capture.
- *  - Every call clears the part of the array it uses (the status word and the
- *    work counter) on `stream` before launching.
+ *    (cudaGetSymbolAddress, no allocation) with that device current, and so
+ *    does the first call after the device's context was re-created (for
+ *    example by cudaDeviceReset); make such a call before any stream capture.
+ *    Devices with an ordinal of 64 or more return HIFA4_ERR_UNSUPPORTED.
+ *  - Arguments are checked as for hifa4_attention_fwd before anything is
+ *    queued; then every call clears the part of the array it uses (the status
+ *    word) on `stream` and launches.
  *  - Problems whose hifa4_workspace_bytes exceeds 4096 return
  *    HIFA4_ERR_UNSUPPORTED without launching.
  *  - All calls on a device share the one array: calls that overlap on the GPU

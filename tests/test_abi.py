@@ -92,3 +92,21 @@ def test_host_validation_rejects_before_launch(lib):
                                       None) == L.ERR_INVALID_ARG
     assert lib.hifa4_status_string(4) == b"bounded wait expired inside a kernel"
     assert lib.hifa4_version() >= 100
+
+
+def test_noalloc_checks_arguments_before_any_cuda_call(lib):
+    """The no-allocation entry point rejects bad arguments on the host before it
+    looks up its scratch array or queues the memset (on a machine without a GPU
+    a CUDA call would fail, so these statuses prove the order)."""
+    from bit_quantized_flashattention_b200 import _lib as L
+    fake = ctypes.c_void_p(1 << 20)
+    pk = L.Packed(*([fake] * 6))
+
+    def call(Nkv=128, scale=0.1, flags=0, o=fake):
+        return lib.hifa4_attention_fwd_noalloc(ctypes.byref(pk), 1, 2, 1, 128, Nkv, 128, ctypes.c_float(scale), flags,
+                                               0, o, L.F32, None, None)
+
+    assert call(Nkv=100) == L.ERR_UNSUPPORTED
+    assert call(scale=0.0) == L.ERR_INVALID_ARG
+    assert call(flags=8) == L.ERR_INVALID_ARG
+    assert call(o=None) == L.ERR_INVALID_ARG

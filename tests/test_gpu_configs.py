@@ -1,6 +1,9 @@
 """Parity on the five full-size workloads, in the launch configuration the
-benchmark times (same kernels, same shapes), against the CPU oracle on
-sampled (batch, kv head) groups and sampled query rows.
+benchmark times (same kernels, same shapes), against the CPU oracle.
+
+Configs 1 and 2 are compared on every (batch, kv head) group and every query
+row; configs 3 to 5 on sampled groups and sampled query rows. The P_hat codes
+the PV GEMM consumed are dumped and compared on every config.
 
 Bars as in test_gpu_parity.py: calibration factors and quantized operands
 bit-exact; P_hat code mismatch <= 1e-4; O (fp32 output) max abs <= 5e-3 and
@@ -30,7 +33,12 @@ def H():
     return H
 
 
+ALL_ROWS = (1, 2)          # configs compared on every group and row
+
+
 def _sample_groups(cfg, rng):
+    if cfg.index in ALL_ROWS:
+        return [(b, g) for b in range(cfg.B) for g in range(cfg.Hkv)]
     grps = [(0, 0), (cfg.B - 1, cfg.Hkv - 1)]
     if cfg.B * cfg.Hkv > 2:
         grps.append((int(rng.integers(cfg.B)), int(rng.integers(cfg.Hkv))))
@@ -38,6 +46,8 @@ def _sample_groups(cfg, rng):
 
 
 def _sample_rows(cfg, rng):
+    if cfg.index in ALL_ROWS:
+        return np.arange(cfg.Nq)
     i = np.unique(np.concatenate([np.arange(min(4, cfg.Nq)), cfg.Nq - 1 - np.arange(min(4, cfg.Nq)),
                                   rng.integers(0, cfg.Nq, ROWS_PER_HEAD)]))
     return np.sort(i)
@@ -56,14 +66,10 @@ def test_config_parity(H, index):
         ref_s, ref_si = oracle.calibrate(cq, ck, cfg.alpha)
         assert np.array_equal(s.cpu().numpy(), ref_s) and np.array_equal(s_inv.cpu().numpy(), ref_si)
     pk = H.quantize_qkv(q, k, v, s, s_inv)
-    dump = cfg.B * cfg.Hq * cfg.Nq * cfg.Nkv // 2 <= (1 << 30)
+    dump = True                # the P_hat dump fits on a B200 for every config (8.6 GB at config 4)
     results = {}
     for norm in cfg.modes:
-        if dump:
-            o, lse, pc, ps = H.attention_fwd_debug(pk, causal=cfg.causal, norm=norm)
-        else:
-            o, lse = H.attention_fwd(pk, causal=cfg.causal, norm=norm, out_dtype=torch.float32)
-            pc = ps = None
+        o, lse, pc, ps = H.attention_fwd_debug(pk, causal=cfg.causal, norm=norm)
         o_bf16, _ = H.attention_fwd(pk, causal=cfg.causal, norm=norm, out_dtype=torch.bfloat16)
         torch.cuda.synchronize()
         results[norm] = (o, lse, pc, ps, o_bf16)
@@ -108,5 +114,5 @@ def test_config_parity(H, index):
                 nib_r = np.stack([ref["p_codes"] & 15, ref["p_codes"] >> 4], -1)
                 n_codes += nib_g.size
                 n_mism += int((nib_g != nib_r).sum())
-    if dump:
-        assert n_mism <= P_MISMATCH * n_codes, (n_mism, n_codes)
+    print(f"config {index}: P_hat code mismatch {n_mism} of {n_codes} ({n_mism / max(n_codes, 1):.2e})")
+    assert n_mism <= P_MISMATCH * n_codes, (n_mism, n_codes)

@@ -218,3 +218,32 @@ def test_timeout_path_reports_status(H):
     o, _ = H.attention_fwd(pk, causal=True, workspace=ws, out_dtype=torch.float32)
     assert H.get_status(ws) == 0
     assert torch.isfinite(o).all()
+
+
+@pytest.mark.parametrize("shape,dtype,smooth", [
+    ((2, 2, 384, 128), "bf16", True),
+    ((1, 3, 256, 64), "fp16", False),
+    ((1, 2, 512, 256), "bf16", True),
+])
+def test_quantize_kv_matches_oracle(H, shape, dtype, smooth):
+    """hifa4_quantize_kv (K and V only, as when a KV cache is appended): codes
+    and MMA-ready scales bit-exact against the oracle, with and without the
+    Smooth-QK factor on K."""
+    B, Hkv, N, D = shape
+    rng = np.random.default_rng(17)
+    q = W.round_to_dtype(_rand(rng, (B, Hkv, N, D)), dtype)
+    k = W.round_to_dtype(_rand(rng, (B, Hkv, N, D)) * rng.lognormal(0, 1, (1, Hkv, 1, D)).astype(np.float32), dtype)
+    v = W.round_to_dtype(_rand(rng, (B, Hkv, N, D)), dtype)
+    s = si = None
+    if smooth:
+        s, si = oracle.calibrate(q, k)
+    dsi = None if si is None else torch.from_numpy(si).cuda()
+    pk = H.quantize_kv(U.to_device(k, dtype), U.to_device(v, dtype), dsi)
+    torch.cuda.synchronize()
+    kc, ks = oracle.quantize_rows(k, si, 1)
+    vtc, vts = oracle.quantize_v(v)
+    _, ks_g, vts_g = U.canonical_scales(pk, B, Hkv, Hkv, 16, N, D)
+    assert np.array_equal(pk.kc.cpu().numpy().reshape(kc.shape), kc)
+    assert np.array_equal(ks_g, ks)
+    assert np.array_equal(pk.vtc.cpu().numpy().reshape(vtc.shape), vtc)
+    assert np.array_equal(vts_g, vts)
