@@ -75,7 +75,7 @@ def lib():
         L.ora_quantize_v.restype = None
         L.ora_qk_row.argtypes = [u8p, u8p, u8p, u8p, ci, ci, ci, ci, ci, cll, f32p]
         L.ora_qk_row.restype = None
-        L.ora_attention_rows.argtypes = [vp] * 9 + [ci] * 6 + [cf, ci, ci, ci, i64p, cll] + [vp] * 7 + [ci]
+        L.ora_attention_rows.argtypes = [vp] * 9 + [ci] * 6 + [cf, ci, ci, ci, ci, i64p, cll] + [vp] * 7 + [ci]
         L.ora_attention_rows.restype = ci
         _lib = L
     return _lib
@@ -173,12 +173,15 @@ def default_sm_scale(D: int) -> float:
 
 
 def attention_rows(shape, rows, *, packed=None, fp32=None, sm_scale=None, causal=False,
-                   norm_mode=P_REORDER, want_eps=False, want_p=False, n_threads=0):
+                   norm_mode=P_REORDER, want_eps=False, want_p=False, n_threads=0, n_splits=1):
     """Run the oracle on selected query rows.
 
     shape: (B, Hq, Hkv, Nq, Nkv, D). rows: flat ids (b*Hq + h)*Nq + i.
     packed: dict of canonical quantized operands (4-bit path), or
     fp32: (q, k, v) float32 operands (quantization off).
+    n_splits: kv split count (contiguous ranges of 128-key tiles, each with its
+    own online softmax, merged by log-sum-exp weights); 1 = one pass.
+    l_hat / l_hp are reported in the frame of the merged max.
     Returns dict with O [n,D] f64, lse [n], l_hat [n], l_hp [n] and optionally
     eps [n, Nkv/128], p_codes [n, Nkv/2], p_sf [n, Nkv/16].
     """
@@ -206,7 +209,7 @@ def attention_rows(shape, rows, *, packed=None, fp32=None, sm_scale=None, causal
         quant = 0
         keep = (qf, kf, vf)
     rc = lib().ora_attention_rows(*args, B, Hq, Hkv, Nq, Nkv, D, float(sm_scale), int(bool(causal)),
-                                  int(norm_mode), quant, rows, n, _ptr(O), _ptr(lse), _ptr(lh), _ptr(lp),
+                                  int(norm_mode), quant, int(n_splits), rows, n, _ptr(O), _ptr(lse), _ptr(lh), _ptr(lp),
                                   _ptr(eps), _ptr(pc), _ptr(ps), int(n_threads))
     del keep
     if rc != 0:

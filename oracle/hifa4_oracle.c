@@ -33,6 +33,13 @@
  *              P is quantized per 16 keys of its row with the element rule
  *   causal     key j is visible to query i iff j <= i + Nkv - Nq
  *   output     O = O_acc / l, LSE = mc*ln 2 + ln l (natural log)
+ *   split kv   (inference option, flash-decoding) the kv tiles are cut into
+ *              n_splits contiguous ranges [floor(s*T/n), floor((s+1)*T/n)); each
+ *              range runs the online softmax above from its own start (its own
+ *              running max, so its P_hat is relative to the range's max), and
+ *              the ranges are merged with their log-sum-exp weights:
+ *              O = sum_s 2^(mc_s - M) O_acc_s / sum_s 2^(mc_s - M) l_s,
+ *              M = max mc_s over ranges with mass; n_splits = 1 is the plain pass
  * Every quantization decision is taken in fp32, the precision the GPU takes
  * it in. Sums and the online-softmax state are kept in fp64, which is exact for
  * the per-tile sums (all decoded operands are multiples of 2^-10 bounded by
@@ -252,6 +259,7 @@ void ora_qk_row(const uint8_t* qc, const uint8_t* qs, const uint8_t* kc, const u
 /* ------------------------------------------------------- attention */
 
 /* norm_mode: 0 = P-Reordering (l from P_hat), 1 = high-precision l (from P).
+ * n_splits >= 1: kv split count (see the header; 1 = one pass).
  * quant: 1 = 4-bit path on the packed operands; 0 = the same online softmax
  * on the fp32 operands qf/kf/vf ([B,H,N,D], already smoothed) with P unquantized.
  * rows: flat query-row ids (b*Hq + h)*Nq + i. Outputs are per requested row.
@@ -263,11 +271,11 @@ int ora_attention_rows(const uint8_t* qc, const uint8_t* qs, const uint8_t* kc, 
                        const uint8_t* vtc, const uint8_t* vts,
                        const float* qf, const float* kf, const float* vf,
                        int B, int Hq, int Hkv, int Nq, int Nkv, int D,
-                       float sm_scale, int causal, int norm_mode, int quant,
+                       float sm_scale, int causal, int norm_mode, int quant, int n_splits,
                        const long long* rows, long long n_rows,
                        double* O, double* lse, double* l_hat_out, double* l_hp_out,
                        double* eps_tile, uint8_t* p_codes, uint8_t* p_sf, int n_threads) {
-    if (D > 256 || D % 16 || Nkv % TILE_KV || Hq % Hkv) return -1;
+    if (D > 256 || D % 16 || Nkv % TILE_KV || Hq % Hkv || n_splits < 1) return -1;
     (void)B;
     int G = Hq / Hkv;
     int n_tiles = Nkv / TILE_KV;
@@ -293,17 +301,23 @@ int ora_attention_rows(const uint8_t* qc, const uint8_t* qs, const uint8_t* kc, 
         } else {
             for (int d = 0; d < D; ++d) qd[d] = qf[(size_t)row * D + d];
         }
-        double oacc[256];
-        for (int d = 0; d < D; ++d) oacc[d] = 0.0;
-        double l_hat = 0.0, l_hp = 0.0;
-        float m = -INFINITY, mc = 0.0f;
+        double Oacc[256], L_out = 0.0, Lhat_out = 0.0, Lhp_out = 0.0;
+        float M = -INFINITY;                       /* largest mc over the splits with mass */
+        for (int d = 0; d < D; ++d) Oacc[d] = 0.0;
         float S[TILE_KV], P[TILE_KV];
         double Ph[TILE_KV];
         if (eps_tile) for (int t = 0; t < n_tiles; ++t) eps_tile[r * n_tiles + t] = NAN;
         if (p_codes) memset(p_codes + (size_t)r * (Nkv / 2), 0, (size_t)Nkv / 2);
         if (p_sf) memset(p_sf + (size_t)r * (Nkv / 16), 0, (size_t)Nkv / 16);
 
-        for (int t = 0; t < n_tiles && (long long)t * TILE_KV <= last; ++t) {
+        for (int sp = 0; sp < n_splits; ++sp) {
+        const int t_begin = (int)(((long long)sp * n_tiles) / n_splits);
+        const int t_end = (int)(((long long)(sp + 1) * n_tiles) / n_splits);
+        double oacc[256];
+        for (int d = 0; d < D; ++d) oacc[d] = 0.0;
+        double l_hat = 0.0, l_hp = 0.0;
+        float m = -INFINITY, mc = 0.0f;
+        for (int t = t_begin; t < t_end && (long long)t * TILE_KV <= last; ++t) {
             /* scores of this tile, masked keys at -inf */
             float rowmax = -INFINITY;
             for (int j = 0; j < TILE_KV; ++j) {
@@ -366,11 +380,29 @@ int ora_attention_rows(const uint8_t* qc, const uint8_t* qs, const uint8_t* kc, 
             m = m_new;
             mc = mc_new;
         }
+        /* merge this split into the running result, in the frame of the
+         * largest mc seen so far (with one split: weight 1, the plain pass) */
         double l = norm_mode == 0 ? l_hat : l_hp;
-        for (int d = 0; d < D; ++d) O[(size_t)r * D + d] = l > 0.0 ? oacc[d] / l : 0.0;
-        lse[r] = l > 0.0 ? (double)mc * 0.69314718055994530942 + log(l) : -INFINITY;
-        if (l_hat_out) l_hat_out[r] = l_hat;
-        if (l_hp_out) l_hp_out[r] = l_hp;
+        if (l > 0.0) {
+            double w_old = 1.0, w_new = 1.0;
+            if (M == -INFINITY) {
+                M = mc;
+            } else if (mc > M) {
+                w_old = exp2((double)M - (double)mc);
+                M = mc;
+            } else {
+                w_new = exp2((double)mc - (double)M);
+            }
+            for (int d = 0; d < D; ++d) Oacc[d] = w_old * Oacc[d] + w_new * oacc[d];
+            L_out = w_old * L_out + w_new * l;
+            Lhat_out = w_old * Lhat_out + w_new * l_hat;
+            Lhp_out = w_old * Lhp_out + w_new * l_hp;
+        }
+        }
+        for (int d = 0; d < D; ++d) O[(size_t)r * D + d] = L_out > 0.0 ? Oacc[d] / L_out : 0.0;
+        lse[r] = L_out > 0.0 ? (double)M * 0.69314718055994530942 + log(L_out) : -INFINITY;
+        if (l_hat_out) l_hat_out[r] = Lhat_out;
+        if (l_hp_out) l_hp_out[r] = Lhp_out;
     }
     return 0;
 }

@@ -430,3 +430,64 @@ def test_smooth_qk_factors_are_reciprocal_pairs_on_outlier_tensors():
         ref = np.einsum("bhid,bhjd->bhij", q.astype(np.float64), kk)
         sm = np.einsum("bhid,bhjd->bhij", q * sq, kk * np.repeat(si.astype(np.float64), G, axis=0)[None, :, None, :])
         assert np.abs(sm - ref).max() <= 1e-6 * np.abs(ref).max()
+
+
+# ----------------------------------------------------- split kv (decoding)
+
+@pytest.mark.parametrize("shape,causal,n_splits", [
+    ((1, 2, 1, 16, 512, 64), False, 4),
+    ((2, 4, 2, 64, 640, 128), True, 4),       # 5 tiles over 4 splits: ragged ranges, bottom-right causal
+    ((1, 2, 2, 32, 384, 128), False, 2),
+    ((1, 1, 1, 128, 512, 256), True, 3),
+])
+def test_split_kv_quant_off_matches_bruteforce(shape, causal, n_splits):
+    """With quantization off, cutting the kv tiles into ranges with their own
+    online softmax and merging by log-sum-exp weights is exactly softmax
+    attention, so it must match the brute-force fp64 result."""
+    B, Hq, Hkv, Nq, Nkv, D = shape
+    rng = np.random.default_rng(33)
+    q = (rng.standard_normal((B, Hq, Nq, D)) * 1.5).astype(np.float32)
+    k = (rng.standard_normal((B, Hkv, Nkv, D)) * 1.5).astype(np.float32)
+    v = rng.standard_normal((B, Hkv, Nkv, D)).astype(np.float32)
+    sm = oracle.default_sm_scale(D)
+    for mode in (oracle.P_REORDER, oracle.HIGH_PRECISION_L):
+        out = oracle.attention_rows(shape, oracle.all_rows(B, Hq, Nq), fp32=(q, k, v), sm_scale=sm, causal=causal,
+                                    norm_mode=mode, n_splits=n_splits)
+        O_ref, lse_ref = _bruteforce(q, k, v, causal, sm)
+        assert np.abs(out["O"] - O_ref.reshape(-1, D)).max() <= 1e-5
+        assert np.abs(out["lse"] - lse_ref.ravel()).max() <= 1e-5
+
+
+def test_split_kv_p_reorder_constant_v_rows_equal_vhat():
+    """P-Reordering with kv splits: every split's numerator and normalizer come
+    from the same P_hat, and the merge weights are shared, so with V = 1 every
+    row is exactly V_hat again."""
+    cfg, q, k = _c2_like(Nq=64, Nkv=512, causal=False, seed=34)
+    v = np.ones_like(k)
+    pk = oracle.quantize_qkv(q, k, v)
+    out = oracle.attention_rows((1, 2, 1, 64, 512, 128), oracle.all_rows(1, 2, 64), packed=pk,
+                                norm_mode=oracle.P_REORDER, n_splits=4)
+    assert np.abs(out["O"] / 1.03125 - 1).max() <= 1e-12
+
+
+def test_split_kv_p_hat_is_relative_to_the_split_max():
+    """Each split starts its own running max: a large score in tile 0 shrinks
+    the P of tile 2 in one pass, but not when tile 2 starts the second of two
+    splits, where its own maximum quantizes to P = 1 (code 7, scale 0x23)."""
+    D = 64
+    q = np.zeros((1, 1, 1, D), np.float32)
+    q[..., 0] = 1.0
+    k = np.zeros((1, 1, 512, D), np.float32)
+    k[0, 0, :, 0] = 0.01
+    k[0, 0, 3, 0] = 60.0                       # tile 0, dominant
+    k[0, 0, 300, 0] = 2.0                      # tile 2's maximum
+    v = np.ones_like(k)
+    pk = oracle.quantize_qkv(q, k, v)
+    one = oracle.attention_rows((1, 1, 1, 1, 512, D), [0], packed=pk, want_p=True)
+    two = oracle.attention_rows((1, 1, 1, 1, 512, D), [0], packed=pk, want_p=True, n_splits=2)
+    key = 300
+    nib = lambda c: (c[key // 2] >> 4) if key % 2 else (c[key // 2] & 15)
+    assert nib(two["p_codes"][0]) == 7 and two["p_sf"][0][key // 16] == 0x23
+    assert nib(one["p_codes"][0]) == 0                    # 2^((2 - 60) c) flushes to zero in one pass
+    # tiles 0 and 1 (the first split) are the same either way
+    assert np.array_equal(one["p_codes"][0][:128], two["p_codes"][0][:128])
