@@ -274,7 +274,7 @@ def run_ours(args):
 
     def step():
         H.quantize_qkv(q, k, v, s, s_inv, out=packed)
-        H.attention_fwd(packed, causal=cfg.causal, norm=norm, out=o, lse=lse, workspace=wsp)
+        H.attention_fwd(packed, causal=cfg.causal, norm=norm, out=o, lse=lse, workspace=wsp, split_kv=True)
 
     launches_per_step = 2          # quantize_qkv_kernel (Q, K and V), attn_fwd_kernel
     for _ in range(max(args.warmup, 3)):
@@ -295,7 +295,7 @@ def run_ours(args):
     with torch.cuda.graph(g_quant):
         H.quantize_qkv(q, k, v, s, s_inv, out=packed)
     with torch.cuda.graph(g_attn):
-        H.attention_fwd(packed, causal=cfg.causal, norm=norm, out=o, lse=lse, workspace=wsp)
+        H.attention_fwd(packed, causal=cfg.causal, norm=norm, out=o, lse=lse, workspace=wsp, split_kv=True)
     for g in (g_step, g_quant, g_attn):
         g.replay()
     torch.cuda.synchronize()
@@ -373,7 +373,7 @@ def run_ours(args):
                 s_cp.wait_event(ev_out[b])         # step i-2's results have left this output buffer
             H.quantize_qkv(dq[b], dk[b], dv[b], s, s_inv, out=dpk[b], stream=s_cp)
             H.attention_fwd(dpk[b], causal=cfg.causal, norm=norm, out=do[b], lse=dl[b], workspace=dws[b],
-                            stream=s_cp)
+                            stream=s_cp, split_kv=True)
             ev_cp[b].record(s_cp)
         with torch.cuda.stream(s_out):
             s_out.wait_event(ev_cp[b])

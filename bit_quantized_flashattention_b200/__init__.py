@@ -7,7 +7,7 @@ quantized probabilities that feed PV. The computation lives in libhifa4.so
 (C ABI, include/hifa4.h); this package is the PyTorch-facing binding.
 """
 from ._lib import HiFA4Error, load  # noqa: F401
-from .api import (PackedQKV, alloc_packed, alloc_workspace, attention_fwd,  # noqa: F401
+from .api import (PackedQKV, alloc_packed, alloc_workspace, attention_fwd, attention_splits,  # noqa: F401
                   attention_fwd_debug, attention_fwd_noalloc, calibrate_smooth, debug_set_wait_limit, get_status,
                   packed_bytes, quantize_kv, quantize_qkv, workspace_bytes)
 

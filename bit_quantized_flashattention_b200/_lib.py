@@ -11,11 +11,12 @@ OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT = 0, 1, 2, 3, 4
 NORM_P_REORDER, NORM_HIGH_PRECISION_L = 0, 1
 F16, BF16, F32 = 0, 1, 2
 CAUSAL = 1
+SPLIT_KV = 2
 
 EXPORTS = ["hifa4_packed_bytes", "hifa4_workspace_bytes", "hifa4_calibrate_smooth", "hifa4_quantize_qkv",
            "hifa4_quantize_kv", "hifa4_attention_fwd", "hifa4_attention_fwd_debug", "hifa4_get_status",
            "hifa4_debug_set_wait_limit", "hifa4_status_string", "hifa4_version", "hifa4_attention_fwd_noalloc",
-           "hifa4_last_cuda_error"]
+           "hifa4_last_cuda_error", "hifa4_attention_splits"]
 
 
 class Packed(ctypes.Structure):
@@ -44,6 +45,8 @@ def load():
     pk = ctypes.POINTER(Packed)
     L.hifa4_packed_bytes.argtypes = [ci] * 6 + [ctypes.POINTER(sz)]
     L.hifa4_packed_bytes.restype = sz
+    L.hifa4_attention_splits.argtypes = [ci] * 6 + [cu]
+    L.hifa4_attention_splits.restype = ci
     L.hifa4_workspace_bytes.argtypes = [ci] * 6
     L.hifa4_workspace_bytes.restype = sz
     L.hifa4_calibrate_smooth.argtypes = [vp, vp, ci, ci, ci, ci, ci, ci, cf, vp, vp, vp]

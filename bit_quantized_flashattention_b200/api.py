@@ -133,7 +133,13 @@ def quantize_kv(k, v, s_inv=None, out: PackedQKV | None = None, Hq: int | None =
     return out
 
 
-def _attn_args(packed, sm_scale, causal, norm, out_dtype, out, lse, workspace, want_lse=True):
+def attention_splits(B, Hq, Hkv, Nq, Nkv, D, causal=False, split_kv=False) -> int:
+    """Number of kv ranges the attention calls use for this shape (1 = one pass)."""
+    flags = (L.CAUSAL if causal else 0) | (L.SPLIT_KV if split_kv else 0)
+    return int(L.load().hifa4_attention_splits(B, Hq, Hkv, Nq, Nkv, D, flags))
+
+
+def _attn_args(packed, sm_scale, causal, norm, out_dtype, out, lse, workspace, want_lse=True, split_kv=False):
     B, Hq, Hkv, Nq, Nkv, D = packed.shape
     dev = packed.qc.device
     if sm_scale is None:
@@ -144,16 +150,17 @@ def _attn_args(packed, sm_scale, causal, norm, out_dtype, out, lse, workspace, w
         lse = torch.empty(B, Hq, Nq, dtype=torch.float32, device=dev)
     if workspace is None:
         workspace = alloc_workspace(B, Hq, Hkv, Nq, Nkv, D, dev)
-    flags = L.CAUSAL if causal else 0
+    flags = (L.CAUSAL if causal else 0) | (L.SPLIT_KV if split_kv else 0)
     return sm_scale, flags, _NORM[norm], out, lse, workspace
 
 
 def attention_fwd(packed: PackedQKV, sm_scale: float | None = None, causal: bool = False,
                   norm="p_reorder", out_dtype=torch.bfloat16, out=None, lse=None, workspace=None,
-                  stream=None, want_lse: bool = True):
-    """4-bit attention forward. Returns (O [B,Hq,Nq,D], LSE [B,Hq,Nq] fp32 or None)."""
+                  stream=None, want_lse: bool = True, split_kv: bool = False):
+    """4-bit attention forward. Returns (O [B,Hq,Nq,D], LSE [B,Hq,Nq] fp32 or None).
+    split_kv: allow the split-kv decode mode (see attention_splits)."""
     sm_scale, flags, nm, out, lse, workspace = _attn_args(packed, sm_scale, causal, norm, out_dtype, out, lse,
-                                                          workspace, want_lse)
+                                                          workspace, want_lse, split_kv)
     st = packed.struct()
     B, Hq, Hkv, Nq, Nkv, D = packed.shape
     L.check(L.load().hifa4_attention_fwd(ctypes.byref(st), B, Hq, Hkv, Nq, Nkv, D, float(sm_scale), flags, nm,
@@ -163,7 +170,8 @@ def attention_fwd(packed: PackedQKV, sm_scale: float | None = None, causal: bool
 
 
 def attention_fwd_noalloc(packed: PackedQKV, sm_scale: float | None = None, causal: bool = False,
-                          norm="p_reorder", out_dtype=torch.bfloat16, out=None, lse=None, stream=None):
+                          norm="p_reorder", out_dtype=torch.bfloat16, out=None, lse=None, stream=None,
+                          split_kv: bool = False):
     """attention_fwd for callers that cannot allocate device memory: the library
     uses its own fixed scratch (see hifa4_attention_fwd_noalloc in hifa4.h).
     ``out``/``lse`` are still the caller's buffers (allocated here when None)."""
@@ -177,16 +185,17 @@ def attention_fwd_noalloc(packed: PackedQKV, sm_scale: float | None = None, caus
         lse = torch.empty(B, Hq, Nq, dtype=torch.float32, device=dev)
     st = packed.struct()
     L.check(L.load().hifa4_attention_fwd_noalloc(ctypes.byref(st), B, Hq, Hkv, Nq, Nkv, D, float(sm_scale),
-                                                 L.CAUSAL if causal else 0, _NORM[norm], _ptr(out), _DT[out.dtype],
+                                                 (L.CAUSAL if causal else 0) | (L.SPLIT_KV if split_kv else 0),
+                                                 _NORM[norm], _ptr(out), _DT[out.dtype],
                                                  _ptr(lse), _stream(stream)), "attention_fwd_noalloc")
     return out, lse
 
 
 def attention_fwd_debug(packed: PackedQKV, sm_scale: float | None = None, causal: bool = False,
-                        norm="p_reorder", out_dtype=torch.float32, workspace=None, stream=None):
+                        norm="p_reorder", out_dtype=torch.float32, workspace=None, stream=None, split_kv: bool = False):
     """attention_fwd plus the P_hat the PV GEMM consumed: (O, LSE, p_codes, p_scales)."""
     sm_scale, flags, nm, out, lse, workspace = _attn_args(packed, sm_scale, causal, norm, out_dtype, None, None,
-                                                          workspace)
+                                                          workspace, True, split_kv)
     B, Hq, Hkv, Nq, Nkv, D = packed.shape
     pc = torch.zeros(B, Hq, Nq, Nkv // 2, dtype=torch.uint8, device=out.device)
     ps = torch.zeros(B, Hq, Nq, Nkv // 16, dtype=torch.uint8, device=out.device)

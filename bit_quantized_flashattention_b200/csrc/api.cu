@@ -80,6 +80,13 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t inner_bytes, uint64_t r
 
 thread_local cudaError_t g_last_cuda_error = cudaSuccess;
 
+// The kernels' split-kv decode mode applies: asked for, D <= 128, a group's
+// query rows fit in half a tile, and every one of the kv ranges gets a tile.
+bool decode_mode(int Hq, int Hkv, int Nq, int Nkv, int D, unsigned flags) {
+    return (flags & HIFA4_SPLIT_KV) != 0 && D <= 128 && (long long)(Hq / Hkv) * Nq <= 64 &&
+           Nkv / 128 >= kDecodeSplits;
+}
+
 }  // namespace
 
 hifa4_status hifa4::from_cuda(cudaError_t e) {
@@ -94,7 +101,7 @@ hifa4_status hifa4::check_attention_args(const hifa4_packed* in, int B, int Hq, 
     if (in == nullptr || o == nullptr) return HIFA4_ERR_INVALID_ARG;
     if (!shape_ok(B, Hq, Hkv, Nq, Nkv, D)) return HIFA4_ERR_UNSUPPORTED;
     if (!(sm_scale > 0.0f) || !std::isfinite(sm_scale)) return HIFA4_ERR_INVALID_ARG;
-    if ((flags & ~(unsigned)HIFA4_CAUSAL) != 0) return HIFA4_ERR_INVALID_ARG;
+    if ((flags & ~(unsigned)(HIFA4_CAUSAL | HIFA4_SPLIT_KV)) != 0) return HIFA4_ERR_INVALID_ARG;
     if ((flags & HIFA4_CAUSAL) != 0 && Nq > Nkv) return HIFA4_ERR_UNSUPPORTED;
     if (norm != HIFA4_NORM_P_REORDER && norm != HIFA4_NORM_HIGH_PRECISION_L) return HIFA4_ERR_INVALID_ARG;
     if (o_dtype != HIFA4_F16 && o_dtype != HIFA4_BF16 && o_dtype != HIFA4_F32) return HIFA4_ERR_INVALID_ARG;
@@ -124,7 +131,8 @@ hifa4_status attention_impl(const hifa4_packed* in, int B, int Hq, int Hkv, int 
     const long long rows_q = (long long)B * Hq * Nq, rows_k = (long long)B * Hkv * Nkv, rows_v = (long long)B * Hkv * D;
     const Sizes sz = sizes_of(B, Hq, Hkv, Nq, Nkv, D);
     const int nqt = D == 256 ? 1 : 2;              // query tiles per CTA (see attention.cu)
-    const long long n_work = (long long)B * Hkv * ((sz.Tq + nqt - 1) / nqt);
+    const bool dec = decode_mode(Hq, Hkv, Nq, Nkv, D, flags);
+    const long long n_work = (long long)B * Hkv * (dec ? 1 : (sz.Tq + nqt - 1) / nqt);
 
     const CUtensorMapSwizzle swz_qk =
         D == 64 ? CU_TENSOR_MAP_SWIZZLE_32B : (D == 128 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B);
@@ -152,13 +160,13 @@ hifa4_status attention_impl(const hifa4_packed* in, int B, int Hq, int Hkv, int 
     p.Tq = sz.Tq;
     p.n_kv_tiles = Nkv / 128;
     p.n_work = (int)n_work;
-    p.heavy_first = (causal && Nq % (128 * nqt) == 0) ? 1 : 0;
+    p.heavy_first = (!dec && causal && Nq % (128 * nqt) == 0) ? 1 : 0;
     p.c = (float)((double)sm_scale * 1.4426950408889634074);
     const long long lim = g_wait_limit_ns.load();
     p.wait_limit_ns = lim > 0 ? (unsigned long long)lim : kDefaultWaitNs;
     p.stall_loads = g_stall_loads.load();
     const int out = o_dtype == HIFA4_F16 ? 0 : (o_dtype == HIFA4_BF16 ? 1 : 2);
-    return from_cuda(launch_attention(&tq, &tk, &tv, p, D, (int)norm, causal, out, dump,
+    return from_cuda(launch_attention(&tq, &tk, &tv, p, D, (int)norm, causal, out, dump, dec,
                                       reinterpret_cast<cudaStream_t>(stream)));
 }
 
@@ -178,6 +186,11 @@ size_t hifa4_packed_bytes(int B, int Hq, int Hkv, int Nq, int Nkv, int D, size_t
         out[5] = s.vts;
     }
     return s.qc + s.qs + s.kc + s.ks + s.vtc + s.vts;
+}
+
+int hifa4_attention_splits(int B, int Hq, int Hkv, int Nq, int Nkv, int D, unsigned flags) {
+    if (!shape_ok(B, Hq, Hkv, Nq, Nkv, D)) return 0;
+    return decode_mode(Hq, Hkv, Nq, Nkv, D, flags) ? kDecodeSplits : 1;
 }
 
 size_t hifa4_workspace_bytes(int B, int Hq, int Hkv, int Nq, int Nkv, int D) {

@@ -8,32 +8,43 @@
 // One CTA computes NQT 128-row query tiles (2 for D <= 128, 1 for D = 256) of
 // one (batch, kv head) group. A tile's rows are the group's query rows stacked
 // head after head (GQA), so a tile may mix heads when Nq is small. Warp roles:
-//   warp 0      TMA / bulk-copy producer: Q_hat tiles once, then K_hat and
-//               V_hat^T tiles (128 keys) with their scale atoms, 3-stage rings
+//   warp 0      TMA / bulk-copy producer: Q_hat once, then K_hat and V_hat^T
+//               tiles (128 keys) with their scale atoms through shared rings
 //   warp 1      TMEM owner; moves the Q scales to TMEM and issues every S MMA
 //   warps 2, 3  PV MMA issuers, one per query tile
 //   warps 4..   one softmax warpgroup per query tile, thread t owns row t:
 //               block maxima of S, running max, P = 2^(S*c - RN(m*c)),
 //               P quantized per 16 keys to E2M1 + E4M3 in registers, O rescaled
-//               in TMEM when some row's max moved, P_hat codes and scales
-//               written to shared memory for the PV MMA.
+//               in TMEM when some row's max moved, P_hat codes written to
+//               shared memory and their scales to TMEM for the PV MMA.
 // The S MMAs run one at a time through one 128-column S buffer in TMEM, in the
-// order (kv tile 0, query tile 0), (0, 1), (1, 0), ...: once a warpgroup has
+// order (kv step 0, query tile 0), (0, 1), (1, 0), ...: once a warpgroup has
 // loaded its scores it arrives (without waiting) at its named barrier
 // "scores loaded", and the S issuer, blocked in that barrier, issues the next S
 // MMA of the order; no warp polls an mbarrier on this path. After the second
-// named barrier of the tile (P_hat stored, O rescaled) the tile's PV issuer
+// named barrier of the step (P_hat stored, O rescaled) the tile's PV issuer
 // issues its PV MMA. An MMA depends only on tcgen05 operations already observed
 // complete through an mbarrier, or issued earlier by the same thread.
-// With P-Reordering the V tile carries 16 extra rows: a row of E2M1 ones
-// (scale 1.0) and 15 zero rows, so the PV MMA also produces sum(P_hat) in
+// With P-Reordering the V tile carries extra rows: a row of E2M1 ones (scale
+// 1.0) and zero rows, so the PV MMA (N = D + 8) also produces sum(P_hat) in
 // output column D: the normalizer from exactly the codes x scales the MMA used.
-// TMEM (512 columns): S [0,128), O tiles [128, 128 + NQT*NO), NO = D (+16),
-// then the scale-factor regions of Q, K, P and V (P and V per query tile).
+//
+// Split-kv decode mode (DEC, G*Nq <= 64 query rows per group, D <= 128): the
+// kv tiles are cut into 4 contiguous ranges (flash-decoding), all run by one
+// CTA. A query tile holds the group's rows twice: lanes 0..63 run range 2x,
+// lanes 64..127 range 2x+1 of query tile x. Two zero-padded copies of Q_hat
+// (rows in the top half only / in the bottom half only) and two MMAs that
+// accumulate into one S give each half its own kv tile; two P_hat buffers with
+// the other half zeroed do the same for PV. Each range keeps its own running
+// max; at the end the four partial (O, m, l) of a row are merged in shared
+// memory with log-sum-exp weights.
+//
+// TMEM (512 columns): S [0,128), O tiles [128, 128 + NQT*NO), then the
+// scale-factor regions of Q, K, P and V.
 // Every mbarrier wait is bounded; when one gives up the CTA records
 // HIFA4_ERR_TIMEOUT in the workspace, drains its copies and MMAs, frees TMEM
-// and exits. The named barriers also OR a failure flag over their threads, so a
-// warpgroup and its issuer leave the loop together.
+// and exits; the warps then keep meeting at the named barriers (doing no
+// work), so every barrier phase still completes.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -42,12 +53,15 @@
 
 namespace hifa4 {
 
-constexpr int kStages = 4;
 constexpr int kSmWarp0 = 4;          // first softmax warp (0: loads, 1: TMEM owner + S MMAs, 2-3: PV MMAs)
+constexpr int kMaxStages = 8;
+constexpr int kDecSplits = 4;        // kv ranges of the split-kv decode mode
 
-template <int D, bool PREORDER>
+template <int D, bool PREORDER, bool DEC>
 struct Cfg {
+    static_assert(!DEC || D <= 128, "decode mode needs two query tiles per CTA");
     static constexpr int NQT = D == 256 ? 1 : 2;          // 128-row query tiles per CTA
+    static constexpr int STAGES = DEC ? 8 : 4;            // kv tiles in flight (decode: 4 per step)
     static constexpr int THREADS = 128 + 128 * NQT;
     static constexpr int KS = D / 64;                     // 64-wide K steps of QK^T
     static constexpr int QK_ROW = D / 2;                  // bytes per Q/K row
@@ -63,47 +77,52 @@ struct Cfg {
     static constexpr int NRB = (D + 127) / 128;           // 128-row blocks of V^T scales
     static constexpr int SFV_BYTES = NRB * 2 * 512;
     static constexpr int P_BYTES = 128 * 64;
-    static constexpr int SFP_BYTES = 2 * 512;
-    static constexpr int NO = PREORDER ? D + 16 : D;      // accumulator columns per query tile
+    static constexpr int NO = PREORDER ? D + 8 : D;       // accumulator columns per query tile
     static constexpr int NCH = D / 32;                    // 32-column chunks of O
+    // scale columns per PV K step: one 4-column block per 128 rows of the B operand
+    static constexpr int SFV_PER_KS = 4 * (NRB + ((PREORDER && D >= 128) ? 1 : 0));
+    static constexpr int N_SFQ = DEC ? 1 : NQT;           // Q scale regions
+    static constexpr int N_SFK = DEC ? 2 : 1;             // K scale regions (decode: one per half)
+    static constexpr int N_SFV = DEC ? 2 * NQT : NQT;     // V scale regions
     // TMEM columns
     static constexpr uint32_t COL_S = 0;
     static constexpr uint32_t COL_O = 128;                                // + qt * NO
-    static constexpr uint32_t COL_SFQ = COL_O + NQT * NO;                 // + qt * 4 * KS
-    static constexpr uint32_t COL_SFK = COL_SFQ + NQT * 4 * KS;
-    static constexpr uint32_t COL_SFP = COL_SFK + 4 * KS;                 // + qt * 8
-    static constexpr uint32_t COL_SFV = COL_SFP + NQT * 8;                 // + qt * 2 * SFV_PER_KS
-    // scale columns per PV K step: one 4-column block per 128 rows of the B operand
-    static constexpr int SFV_PER_KS = 4 * (NRB + ((PREORDER && D >= 128) ? 1 : 0));
-    static constexpr uint32_t COL_END = COL_SFV + NQT * 2 * SFV_PER_KS;
+    static constexpr uint32_t COL_SFQ = COL_O + NQT * NO;
+    static constexpr uint32_t COL_SFK = COL_SFQ + N_SFQ * 4 * KS;
+    static constexpr uint32_t COL_SFP = COL_SFK + N_SFK * 4 * KS;          // + qt * 8
+    static constexpr uint32_t COL_SFV = COL_SFP + NQT * 8;                 // + region * 2 * SFV_PER_KS
+    static constexpr uint32_t COL_END = COL_SFV + N_SFV * 2 * SFV_PER_KS;
     static_assert(COL_END <= 512, "TMEM budget");
     // shared memory offsets (operand tiles 1024-aligned)
-    static constexpr int OFF_Q = 0;                                       // + qt * Q_BYTES
+    static constexpr int OFF_Q = 0;                                       // + buffer * Q_BYTES
     static constexpr int OFF_K = OFF_Q + NQT * Q_BYTES;
-    static constexpr int OFF_V = OFF_K + kStages * K_BYTES;
-    static constexpr int OFF_P = OFF_V + kStages * V_STRIDE;              // + (qt * 2 + buf) * P_BYTES
+    static constexpr int OFF_V = OFF_K + STAGES * K_BYTES;
+    static constexpr int OFF_P = OFF_V + STAGES * V_STRIDE;              // + (qt * 2 + buf) * P_BYTES
     static constexpr int OFF_SFQ = OFF_P + NQT * 2 * P_BYTES;             // + qt * SFQK_BYTES
     static constexpr int OFF_SFK = OFF_SFQ + NQT * SFQK_BYTES;
-    static constexpr int OFF_SFV = OFF_SFK + kStages * SFQK_BYTES;
-    static constexpr int OFF_SFP = OFF_SFV + kStages * SFV_BYTES;         // + (qt * 2 + buf) * SFP_BYTES
-    static constexpr int OFF_ONES = OFF_SFP + NQT * 2 * SFP_BYTES;
+    static constexpr int OFF_SFV = OFF_SFK + STAGES * SFQK_BYTES;
+    static constexpr int OFF_ONES = OFF_SFV + STAGES * SFV_BYTES;
     static constexpr int OFF_LUT = OFF_ONES + 512;                        // float [128]
     static constexpr int OFF_BAR = OFF_LUT + 128 * 4;
-    static constexpr int OFF_MISC = OFF_BAR + 256;
+    static constexpr int OFF_MISC = OFF_BAR + 512;
     static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;              // + alignment slack
+    static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
+    // decode merge scratch, after the loop: partial O rows (fp32, rows padded by
+    // 4 floats) in the K/V ring, the (mc, l) pairs in the P buffers
+    static constexpr int MERGE_ROW = D + 4;
+    static_assert(!DEC || kDecSplits * 64 * MERGE_ROW * 4 <= OFF_P - OFF_K, "merge scratch");
 };
 
 struct Bars {
     uint64_t q_full;
-    uint64_t k_full[kStages];
-    uint64_t v_full[kStages];
-    uint64_t v_empty[kStages][2];   // K and V slot no longer read by query tile x's MMAs
-    uint64_t s_full[2];             // S of query tile x is in TMEM
-    uint64_t o_done[2];             // PV MMA of query tile x finished
-    uint64_t sfk_full;              // K scales of the next kv tile moved to TMEM
-    uint64_t drain[3];              // teardown: MMAs issued by the starter / by each tile's leader
+    uint64_t k_full[kMaxStages];
+    uint64_t v_full[kMaxStages];
+    uint64_t v_empty[kMaxStages][2];   // K and V slot no longer read by query tile x's MMAs
+    uint64_t s_full[2];                // S of query tile x is in TMEM
+    uint64_t o_done[2];                // PV MMA of query tile x finished
+    uint64_t drain[3];                 // teardown: MMAs issued by the S issuer / each PV issuer
 };
-static_assert(sizeof(Bars) <= 256, "barrier area");
+static_assert(sizeof(Bars) <= 512, "barrier area");
 
 #ifndef HIFA4_TRACE_POINT
 #define HIFA4_TRACE_POINT(role, j, e)
@@ -111,30 +130,6 @@ static_assert(sizeof(Bars) <= 256, "barrier area");
 
 __device__ __forceinline__ uint32_t p_swizzle64(uint32_t row, uint32_t chunk) {
     return row * 64u + ((chunk ^ ((row >> 1) & 3u)) << 4);
-}
-
-template <int OUT>
-__device__ __forceinline__ void store_out32(void* dst, const float (&v)[32]) {
-    if constexpr (OUT == 2) {
-        float4* d = reinterpret_cast<float4*>(dst);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) d[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
-    } else {
-        uint32_t w[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            if constexpr (OUT == 1) {
-                __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
-                w[i] = *reinterpret_cast<uint32_t*>(&h);
-            } else {
-                __half2 h = __floats2half2_rn(v[2 * i], v[2 * i + 1]);
-                w[i] = *reinterpret_cast<uint32_t*>(&h);
-            }
-        }
-        uint4* d = reinterpret_cast<uint4*>(dst);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) d[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
-    }
 }
 
 // Maximum of 16 values held as 8 pairs (three-input max, depth 3).
@@ -155,12 +150,38 @@ __device__ __forceinline__ void scale_chunk(uint32_t (&o)[32], float2 a2) {
     }
 }
 
-template <int D, bool PREORDER, bool CAUSAL, int OUT, bool DUMP>
-__global__ void __launch_bounds__(Cfg<D, PREORDER>::THREADS, 1)
+// Stores n (a multiple of 8) fp32 values as fp32 / bf16 / fp16 (OUT 2 / 1 / 0).
+template <int OUT, int N>
+__device__ __forceinline__ void store_out(void* dst, const float* v) {
+    if constexpr (OUT == 2) {
+        float4* d = reinterpret_cast<float4*>(dst);
+#pragma unroll
+        for (int i = 0; i < N / 4; ++i) d[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+    } else {
+        uint32_t w[N / 2];
+#pragma unroll
+        for (int i = 0; i < N / 2; ++i) {
+            if constexpr (OUT == 1) {
+                __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+                w[i] = *reinterpret_cast<uint32_t*>(&h);
+            } else {
+                __half2 h = __floats2half2_rn(v[2 * i], v[2 * i + 1]);
+                w[i] = *reinterpret_cast<uint32_t*>(&h);
+            }
+        }
+        uint4* d = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+        for (int i = 0; i < N / 8; ++i) d[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+    }
+}
+
+template <int D, bool PREORDER, bool CAUSAL, int OUT, bool DUMP, bool DEC>
+__global__ void __launch_bounds__(Cfg<D, PREORDER, DEC>::THREADS, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
-    using C = Cfg<D, PREORDER>;
+    using C = Cfg<D, PREORDER, DEC>;
     constexpr int NQT = C::NQT;
+    constexpr int ST = C::STAGES;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     Bars* bars = reinterpret_cast<Bars*>(smem + C::OFF_BAR);
@@ -173,11 +194,12 @@ __global__ void __launch_bounds__(Cfg<D, PREORDER>::THREADS, 1)
     const int lane = threadIdx.x & 31;
 
     // ---------------------------------------------------------------- work
-    // One work unit = up to NQT consecutive 128-row query tiles of one group.
+    // One work unit = up to NQT consecutive 128-row query tiles of one group
+    // (decode: the whole group, whose rows fit in half a tile).
     const int w = blockIdx.x;
-    const int units_per_grp = (p.Tq + NQT - 1) / NQT;
+    const int units_per_grp = DEC ? 1 : (p.Tq + NQT - 1) / NQT;
     int grp, t0;
-    if (p.heavy_first) {
+    if (!DEC && p.heavy_first) {
         // causal with Nq % (128 * NQT) == 0: units with the most keys first
         const int per_head = p.Nq / (128 * NQT);
         const int per = p.B * p.Hkv * p.G;
@@ -189,25 +211,39 @@ __global__ void __launch_bounds__(Cfg<D, PREORDER>::THREADS, 1)
         grp = w / units_per_grp;
         t0 = (w % units_per_grp) * NQT;
     }
-    const int n_qt = min(NQT, p.Tq - t0);
+    const int n_qt = DEC ? NQT : min(NQT, p.Tq - t0);
     const int rows_in_grp = p.G * p.Nq;
+    const int T = p.n_kv_tiles;
+    // decode: kv range r covers tiles [T*r/4, T*(r+1)/4)
+    auto range_begin = [&](int r) -> int { return (int)(((long long)T * r) / kDecSplits); };
+    auto range_len = [&](int r) -> int { return range_begin(r + 1) - range_begin(r); };
     // kv tiles each query tile visits (causal: up to the last visible key of its last row)
     auto kv_tiles_of = [&](int qt) -> int {
         if (qt >= n_qt) return 0;
-        if (!CAUSAL) return p.n_kv_tiles;
+        if (DEC) return max(range_len(2 * qt), range_len(2 * qt + 1));   // steps of the tile
+        if (!CAUSAL) return T;
         const int p0 = (t0 + qt) * 128;
         const int p_max = min(p0 + 127, rows_in_grp - 1);
         const int i_max = (p_max / p.Nq == p0 / p.Nq) ? (p_max % p.Nq) : (p.Nq - 1);
-        return min(p.n_kv_tiles, (i_max + p.Nkv - p.Nq) / 128 + 1);
+        return min(T, (i_max + p.Nkv - p.Nq) / 128 + 1);
     };
     int n_tiles[2];
     n_tiles[0] = kv_tiles_of(0);
     n_tiles[1] = NQT > 1 ? kv_tiles_of(1) : 0;
     const int n_tiles_max = max(n_tiles[0], n_tiles[1]);
+    // Loads: one kv tile (K and V) each, in consumption order. Plain mode:
+    // load j = kv tile j for the tiles visiting it; decode: load 4t + 2x + h =
+    // step t of range 2x + h (a null load past the end of a shorter range).
+    const int n_loads = DEC ? 4 * n_tiles_max : n_tiles_max;
+    auto load_tile = [&](int i) -> int { return DEC ? range_begin(i & 3) + (i >> 2) : i; };
+    auto load_users = [&](int i) -> int {   // bit x: query tile x reads this load
+        if (DEC) return (i >> 2) < range_len(i & 3) ? 1 << ((i & 3) >> 1) : 0;
+        return (i < n_tiles[0] ? 1 : 0) | (NQT > 1 && i < n_tiles[1] ? 2 : 0);
+    };
 
     // The S MMAs run one at a time through the one S buffer, in the order
-    // (kv tile 0, query tile 0), (0, 1), (1, 0), (1, 1), ... skipping the kv
-    // tiles a query tile does not visit. The item after (j, x) in that order:
+    // (step 0, query tile 0), (0, 1), (1, 0), (1, 1), ... skipping the steps a
+    // query tile does not take. The item after (j, x) in that order:
     auto next_item = [&](int j, int x, int& nj, int& nx) -> bool {
 #pragma unroll 1
         for (int guard = 0; guard < 2 * NQT + 2; ++guard) {
@@ -221,7 +257,7 @@ __global__ void __launch_bounds__(Cfg<D, PREORDER>::THREADS, 1)
     // --------------------------------------------------------------- setup
     if (threadIdx.x == 0) {
         mbar_init(&bars->q_full, 1);
-        for (int s = 0; s < kStages; ++s) {
+        for (int s = 0; s < ST; ++s) {
             mbar_init(&bars->k_full[s], 1);
             mbar_init(&bars->v_full[s], 1);
             for (int x = 0; x < 2; ++x) mbar_init(&bars->v_empty[s][x], 1);
@@ -231,7 +267,6 @@ __global__ void __launch_bounds__(Cfg<D, PREORDER>::THREADS, 1)
             mbar_init(&bars->o_done[x], 1);
         }
         for (int k = 0; k < 3; ++k) mbar_init(&bars->drain[k], 1);
-        mbar_init(&bars->sfk_full, 1);
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -239,13 +274,21 @@ __global__ void __launch_bounds__(Cfg<D, PREORDER>::THREADS, 1)
         const uint32_t i = threadIdx.x - 128;
         lut[i] = (i == 0) ? 0.0f : __frcp_rn(e4m3_to_f32(i));
         // normalizer block of V^T (rows D..D+15 of every stage): one row of E2M1
-        // ones (code 2 in both nibbles), 15 zero rows; and the scale atom of the
+        // ones (code 2 in both nibbles), zero rows; and the scale atom of the
         // ones row (row 0 of an atom = 1.0) used when D >= 128.
-        for (int s = 0; s < kStages; ++s) {
+        for (int s = 0; s < ST; ++s) {
             uint32_t* row = reinterpret_cast<uint32_t*>(smem + C::OFF_V + s * C::V_STRIDE + D * 64);
             for (int k = i; k < 16 * 16; k += 128) row[k] = (k < 16) ? 0x22222222u : 0u;
         }
         reinterpret_cast<uint32_t*>(smem + C::OFF_ONES)[i] = (i == 0) ? 0x38383838u : 0u;
+    }
+    if constexpr (DEC) {
+        // the P_hat buffers: a thread only ever writes its own row, in the
+        // buffer of its half, so the other half of every buffer stays zero
+        if (threadIdx.x >= 128) {
+            uint4* pz = reinterpret_cast<uint4*>(smem + C::OFF_P);
+            for (int k = threadIdx.x - 128; k < NQT * 2 * C::P_BYTES / 16; k += 128 * NQT) pz[k] = make_uint4(0, 0, 0, 0);
+        }
     }
     if (warp == 1) {
         tmem_alloc(tmem_slot, 512);
@@ -263,88 +306,121 @@ __global__ void __launch_bounds__(Cfg<D, PREORDER>::THREADS, 1)
     const uint32_t tmem = *tmem_slot;
     const WaitCtl ctl{abort_flag, p.status, p.wait_limit_ns};
 
-    // Scale atoms moved shared->TMEM, and the MMAs. Issued by one thread at a
-    // time; an MMA is issued only after every tcgen05 operation it depends on
-    // has completed (observed through an mbarrier), except where one thread
-    // issues both: its tcgen05 operations run in issue order.
+    // Scale atoms moved shared->TMEM, and the MMAs. An MMA is issued only after
+    // every tcgen05 operation it depends on has completed (observed through an
+    // mbarrier), or was issued earlier by the same thread (one thread's
+    // tcgen05 operations run in issue order).
     // Shared-memory descriptors: a base descriptor plus (byte offset >> 4) in
     // the 14-bit address field (all shared addresses are below 256 KB).
     const uint32_t idesc_s = idesc_fp4_block16(128);
     auto sf_desc = [&](uint32_t off) { return smem_desc(sbase + off, 0u, 128u, 0u); };
     const uint64_t qk_desc0 = smem_desc(sbase, 16u, C::QK_SBO, C::QK_SWZ);
     const uint64_t pv_desc0 = smem_desc(sbase, 16u, 512u, 4u);
-    // first and last query tile (in S order) that visit kv tile j
-    auto first_x_of = [&](int j) -> int { return j < n_tiles[0] ? 0 : 1; };
+    // last query tile (in S order) that visits plain-mode kv tile j
     auto last_x_of = [&](int j) -> int { return (NQT > 1 && j < n_tiles[1]) ? 1 : 0; };
-    auto copy_sfk = [&](int j) {
-        const int st = j % kStages;
+    auto copy_sfk = [&](int li, int region) {
+        const int st = li % ST;
 #pragma unroll
         for (int s = 0; s < C::KS; ++s)
-            tmem_cp_scale_atom(tmem + C::COL_SFK + 4 * s, sf_desc(C::OFF_SFK + st * C::SFQK_BYTES + 512 * s));
+            tmem_cp_scale_atom(tmem + C::COL_SFK + region * 4 * C::KS + 4 * s,
+                               sf_desc(C::OFF_SFK + st * C::SFQK_BYTES + 512 * s));
     };
-    auto copy_sfv = [&](int j, int x) {
-        const int st = j % kStages;
+    auto copy_sfv = [&](int li, int region) {
+        const int st = li % ST;
         const uint32_t sfv = C::OFF_SFV + st * C::SFV_BYTES;
-        const uint32_t col_sfv = C::COL_SFV + x * 2 * C::SFV_PER_KS;
+        const uint32_t col = C::COL_SFV + region * 2 * C::SFV_PER_KS;
 #pragma unroll
         for (int s = 0; s < 2; ++s)
 #pragma unroll
             for (int rb = 0; rb < C::NRB; ++rb)
-                tmem_cp_scale_atom(tmem + col_sfv + s * C::SFV_PER_KS + 4 * rb, sf_desc(sfv + (rb * 2 + s) * 512));
+                tmem_cp_scale_atom(tmem + col + s * C::SFV_PER_KS + 4 * rb, sf_desc(sfv + (rb * 2 + s) * 512));
     };
-    // S = Q_hat(x) K_hat(j)^T. The issuer of the last S MMA on tile j then
-    // moves the next tile's K scales in (they replace tile j's only after that
-    // MMA: same thread, issue order) and signals sfk_full; the first S MMA on a
-    // tile waits for that signal (the scales of tile 0 come with the first MMA).
-    // Returns false if a wait gave up.
-    auto issue_s = [&](int j, int x) -> bool {
-        const int st = j % kStages;
-        if (j > 0 && x == first_x_of(j) && !mbar_wait_poll(&bars->sfk_full, (j - 1) & 1, ctl, 32)) {
-            tc_commit(&bars->s_full[x]);
-            return false;
-        }
-        tc_fence_after();
-        const uint64_t kd = qk_desc0 + ((C::OFF_K + st * C::K_BYTES) >> 4);
-        const uint64_t qd = qk_desc0 + ((C::OFF_Q + x * C::Q_BYTES) >> 4);
+    // the K scales an item needs next (plain: the next kv tile, after the last
+    // item on this one; decode: the two loads of the next item), moved in by the
+    // S issuer right after the current MMAs. Returns false if a load never came.
+    auto prefetch_sfk = [&](int j, int x) -> bool {
+        int nj, nx;
+        if (!next_item(j, x, nj, nx)) return true;
+        if constexpr (DEC) {
 #pragma unroll
-        for (int s = 0; s < C::KS; ++s)
-            mma_fp4_block16(tmem + C::COL_S, qd + 2 * s, kd + 2 * s, idesc_s, tmem + C::COL_SFQ + x * 4 * C::KS + 4 * s,
-                            tmem + C::COL_SFK + 4 * s, s > 0 ? 1u : 0u);
-        tc_commit(&bars->s_full[x]);
-        if (x == last_x_of(j) && j + 1 < n_tiles_max) {
-            if (!mbar_wait_poll(&bars->k_full[(j + 1) % kStages], ((j + 1) / kStages) & 1, ctl, 32)) return false;
-            copy_sfk(j + 1);
-            tc_commit(&bars->sfk_full);
+            for (int h = 0; h < 2; ++h) {
+                const int li = 4 * nj + 2 * nx + h;
+                if (!(load_users(li) & (1 << nx))) continue;
+                if (!mbar_wait_poll(&bars->k_full[li % ST], (li / ST) & 1, ctl, 32)) return false;
+                copy_sfk(li, h);
+            }
+        } else {
+            if (nj == j) return true;
+            if (!mbar_wait_poll(&bars->k_full[nj % ST], (nj / ST) & 1, ctl, 32)) return false;
+            copy_sfk(nj, 0);
         }
         return true;
     };
-    // O(x) += P_hat(x, j) V_hat(j) (P scales written to TMEM by the softmax
-    // threads, V scales of tile j already in x's columns); then the V scales
-    // of tile j + 1 are moved in for the next PV MMA of this tile.
-    auto issue_pv = [&](int j, int x) -> bool {
-        const int st = j % kStages;
-        const uint64_t vd = pv_desc0 + ((C::OFF_V + st * C::V_STRIDE) >> 4);
-        const uint64_t pd = pv_desc0 + ((C::OFF_P + (x * 2 + (j & 1)) * C::P_BYTES) >> 4);
-        const uint32_t col_sfv = C::COL_SFV + x * 2 * C::SFV_PER_KS;
-        const uint32_t o = tmem + C::COL_O + x * C::NO;
+    // S = Q_hat K_hat^T of item (j, x): one MMA per half (decode: Q_hat copy h
+    // against range 2x+h's kv tile, accumulating into the same S).
+    auto issue_s = [&](int j, int x) -> bool {
+        bool first = true;
 #pragma unroll
-        for (int s = 0; s < 2; ++s) {
-            const uint32_t acc = (j > 0 || s > 0) ? 1u : 0u;
-            const uint32_t sfa = tmem + C::COL_SFP + x * 8 + 4 * s;
-            const uint32_t sfb = tmem + col_sfv + s * C::SFV_PER_KS;
-            if constexpr (D == 256 && PREORDER) {
-                mma_fp4_block16(o, pd + 2 * s, vd + 2 * s, idesc_fp4_block16(128), sfa, sfb, acc);
-                mma_fp4_block16(o + 128, pd + 2 * s, vd + ((128 * 64) >> 4) + 2 * s, idesc_fp4_block16(144), sfa,
-                                sfb + 4, acc);
-            } else {
-                mma_fp4_block16(o, pd + 2 * s, vd + 2 * s, idesc_fp4_block16(C::NO), sfa, sfb, acc);
+        for (int h = 0; h < (DEC ? 2 : 1); ++h) {
+            const int li = DEC ? 4 * j + 2 * x + h : j;
+            if (DEC && !(load_users(li) & (1 << x))) continue;
+            const int st = li % ST;
+            const uint64_t kd = qk_desc0 + ((C::OFF_K + st * C::K_BYTES) >> 4);
+            const uint64_t qd = qk_desc0 + ((C::OFF_Q + (DEC ? h : x) * C::Q_BYTES) >> 4);
+            const uint32_t sfq = tmem + C::COL_SFQ + (DEC ? 0 : x) * 4 * C::KS;
+            const uint32_t sfk = tmem + C::COL_SFK + (DEC ? h : 0) * 4 * C::KS;
+#pragma unroll
+            for (int s = 0; s < C::KS; ++s)
+                mma_fp4_block16(tmem + C::COL_S, qd + 2 * s, kd + 2 * s, idesc_s, sfq + 4 * s, sfk + 4 * s,
+                                (first && s == 0) ? 0u : 1u);
+            first = false;
+        }
+        tc_commit(&bars->s_full[x]);
+        if (!DEC && !(x == last_x_of(j))) return true;
+        return prefetch_sfk(j, x);
+    };
+    // O(x) += P_hat V_hat of step j (decode: one MMA per half), then the V
+    // scales of the next step are moved in for the next PV MMA of this tile.
+    auto issue_pv = [&](int j, int x) -> bool {
+        const uint32_t o = tmem + C::COL_O + x * C::NO;
+        bool first = j == 0;
+#pragma unroll
+        for (int h = 0; h < (DEC ? 2 : 1); ++h) {
+            const int li = DEC ? 4 * j + 2 * x + h : j;
+            if (DEC && !(load_users(li) & (1 << x))) continue;
+            const int st = li % ST;
+            const uint64_t vd = pv_desc0 + ((C::OFF_V + st * C::V_STRIDE) >> 4);
+            const uint64_t pd = pv_desc0 + ((C::OFF_P + (x * 2 + (DEC ? h : (j & 1))) * C::P_BYTES) >> 4);
+            const uint32_t col_sfv = C::COL_SFV + (DEC ? 2 * x + h : x) * 2 * C::SFV_PER_KS;
+#pragma unroll
+            for (int s = 0; s < 2; ++s) {
+                const uint32_t acc = (first && s == 0) ? 0u : 1u;
+                const uint32_t sfa = tmem + C::COL_SFP + x * 8 + 4 * s;
+                const uint32_t sfb = tmem + col_sfv + s * C::SFV_PER_KS;
+                if constexpr (D == 256 && PREORDER) {
+                    mma_fp4_block16(o, pd + 2 * s, vd + 2 * s, idesc_fp4_block16(128), sfa, sfb, acc);
+                    mma_fp4_block16(o + 128, pd + 2 * s, vd + ((128 * 64) >> 4) + 2 * s, idesc_fp4_block16(C::NO - 128),
+                                    sfa, sfb + 4, acc);
+                } else {
+                    mma_fp4_block16(o, pd + 2 * s, vd + 2 * s, idesc_fp4_block16(C::NO), sfa, sfb, acc);
+                }
             }
+            first = false;
         }
         tc_commit(&bars->o_done[x]);
-        tc_commit(&bars->v_empty[st][x]);
+#pragma unroll
+        for (int h = 0; h < (DEC ? 2 : 1); ++h) {
+            const int li = DEC ? 4 * j + 2 * x + h : j;
+            if (load_users(li) & (1 << x)) tc_commit(&bars->v_empty[li % ST][x]);
+        }
         if (j + 1 < n_tiles[x]) {
-            if (!mbar_wait_poll(&bars->v_full[(j + 1) % kStages], ((j + 1) / kStages) & 1, ctl, 32)) return false;
-            copy_sfv(j + 1, x);
+#pragma unroll
+            for (int h = 0; h < (DEC ? 2 : 1); ++h) {
+                const int li = DEC ? 4 * (j + 1) + 2 * x + h : j + 1;
+                if (!(load_users(li) & (1 << x))) continue;
+                if (!mbar_wait_poll(&bars->v_full[li % ST], (li / ST) & 1, ctl, 32)) return false;
+                copy_sfv(li, DEC ? 2 * x + h : x);
+            }
         }
         return true;
     };
@@ -355,50 +431,59 @@ __global__ void __launch_bounds__(Cfg<D, PREORDER>::THREADS, 1)
         // stream (programmatic dependent launch); the packed operands are read
         // only after it has completed. Every other read of those operands
         // goes through this warp's copies. A slot is refilled once every query
-        // tile that read the previous kv tile in it has released it.
+        // tile that read the previous load in it has released it (a finished
+        // PV MMA of that load also means its S MMA finished).
         grid_dependency_wait();
         if (lane == 0 && !p.stall_loads) {
             int issued = 0;
             bool ok = true;
-            mbar_arrive_expect_tx(&bars->q_full, n_qt * (C::Q_BYTES + C::SFQK_BYTES));
-            for (int qt = 0; qt < n_qt; ++qt) {
+            const int nq_load = DEC ? 1 : n_qt;
+            mbar_arrive_expect_tx(&bars->q_full, nq_load * (C::Q_BYTES + C::SFQK_BYTES));
+            for (int qt = 0; qt < nq_load; ++qt) {
                 tma_load_2d(smem + C::OFF_Q + qt * C::Q_BYTES, &tmQ, 0, grp * rows_in_grp + (t0 + qt) * 128,
                             &bars->q_full);
                 bulk_load(smem + C::OFF_SFQ + qt * C::SFQK_BYTES,
                           p.qs + ((size_t)grp * p.Tq + t0 + qt) * C::SFQK_BYTES, C::SFQK_BYTES, &bars->q_full);
             }
-            for (int j = 0; j < n_tiles_max && ok; ++j) {
-                const int st = j % kStages;
-                const int jp = j - kStages;                          // previous kv tile in this slot
-                const uint32_t ph = (jp / kStages) & 1;
-                // a finished PV MMA of tile jp also means its S MMAs finished
-                for (int x = 0; x < NQT && jp >= 0 && ok; ++x)
-                    if (jp < n_tiles[x] && !mbar_wait_poll(&bars->v_empty[st][x], ph, ctl, 256)) ok = false;
+            for (int i = 0; i < n_loads && ok; ++i) {
+                const int st = i % ST;
+                const int ip = i - ST;                               // previous load in this slot
+                if (ip >= 0) {
+                    const int users = load_users(ip);
+                    const uint32_t ph = (ip / ST) & 1;
+                    for (int x = 0; x < NQT && ok; ++x)
+                        if ((users >> x) & 1) ok = mbar_wait_poll(&bars->v_empty[st][x], ph, ctl, 256);
+                }
                 if (!ok) break;
-                mbar_arrive_expect_tx(&bars->k_full[st], C::K_BYTES + C::SFQK_BYTES);
-                tma_load_2d(smem + C::OFF_K + st * C::K_BYTES, &tmK, 0, grp * p.Nkv + j * 128, &bars->k_full[st]);
-                bulk_load(smem + C::OFF_SFK + st * C::SFQK_BYTES,
-                          p.ks + ((size_t)grp * p.n_kv_tiles + j) * C::SFQK_BYTES, C::SFQK_BYTES, &bars->k_full[st]);
-                issued = 2 * j + 1;
-                mbar_arrive_expect_tx(&bars->v_full[st], C::V_TMA_BYTES + C::SFV_BYTES);
-                tma_load_2d(smem + C::OFF_V + st * C::V_STRIDE, &tmV, j * 64, grp * D, &bars->v_full[st]);
-                bulk_load(smem + C::OFF_SFV + st * C::SFV_BYTES,
-                          p.vts + ((size_t)grp * p.n_kv_tiles + j) * C::SFV_BYTES, C::SFV_BYTES, &bars->v_full[st]);
-                issued = 2 * j + 2;
+                if (load_users(i) == 0) {
+                    // a null load (past the end of a shorter range): nothing reads it
+                    mbar_arrive(&bars->k_full[st]);
+                    mbar_arrive(&bars->v_full[st]);
+                } else {
+                    const int j = load_tile(i);
+                    mbar_arrive_expect_tx(&bars->k_full[st], C::K_BYTES + C::SFQK_BYTES);
+                    tma_load_2d(smem + C::OFF_K + st * C::K_BYTES, &tmK, 0, grp * p.Nkv + j * 128, &bars->k_full[st]);
+                    bulk_load(smem + C::OFF_SFK + st * C::SFQK_BYTES,
+                              p.ks + ((size_t)grp * T + j) * C::SFQK_BYTES, C::SFQK_BYTES, &bars->k_full[st]);
+                    mbar_arrive_expect_tx(&bars->v_full[st], C::V_TMA_BYTES + C::SFV_BYTES);
+                    tma_load_2d(smem + C::OFF_V + st * C::V_STRIDE, &tmV, j * 64, grp * D, &bars->v_full[st]);
+                    bulk_load(smem + C::OFF_SFV + st * C::SFV_BYTES,
+                              p.vts + ((size_t)grp * T + j) * C::SFV_BYTES, C::SFV_BYTES, &bars->v_full[st]);
+                }
+                issued = i + 1;
             }
             if (!ok) {
                 // drain the copies still in flight before the CTA exits
-                const int nk = (issued + 1) / 2, nv = issued / 2;
-                for (int j = max(0, nk - kStages); j < nk; ++j)
-                    mbar_wait_drain(&bars->k_full[j % kStages], (j / kStages) & 1, p.wait_limit_ns);
-                for (int j = max(0, nv - kStages); j < nv; ++j)
-                    mbar_wait_drain(&bars->v_full[j % kStages], (j / kStages) & 1, p.wait_limit_ns);
+                for (int i = max(0, issued - ST); i < issued; ++i) {
+                    mbar_wait_drain(&bars->k_full[i % ST], (i / ST) & 1, p.wait_limit_ns);
+                    mbar_wait_drain(&bars->v_full[i % ST], (i / ST) & 1, p.wait_limit_ns);
+                }
                 mbar_wait_drain(&bars->q_full, 0, p.wait_limit_ns);
             }
         }
     } else if (warp == 1) {
         // ------------------------------------------------------- S issuer
-        // Moves the Q scales (and the first tiles' K and V scales) to TMEM,
+        // Moves the Q scales (and the first step's K and V scales) to TMEM,
         // issues the first S MMA, then walks the S order: once the consumer of
         // an S tile has loaded it (named barrier "scores loaded" of that
         // warpgroup, which arrives without waiting) the next S MMA is issued.
@@ -406,28 +491,68 @@ __global__ void __launch_bounds__(Cfg<D, PREORDER>::THREADS, 1)
         bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(&bars->q_full, 0, ctl));
         int j = 0, x = 0;
         bool more = next_item(0, -1, j, x);
-        if (ok && more) ok = __all_sync(0xFFFFFFFFu, mbar_wait(&bars->k_full[0], 0, ctl));
-        if (ok && more) ok = __all_sync(0xFFFFFFFFu, mbar_wait(&bars->v_full[0], 0, ctl));
+        // the loads the first step reads (plain: load 0; decode: loads 0..3)
+        for (int i = 0; i < (DEC ? 4 : 1) && ok && more; ++i) {
+            if (load_users(i) == 0) continue;
+            ok = __all_sync(0xFFFFFFFFu, mbar_wait(&bars->k_full[i % ST], 0, ctl));
+            if (ok) ok = __all_sync(0xFFFFFFFFu, mbar_wait(&bars->v_full[i % ST], 0, ctl));
+        }
+        if constexpr (DEC) {
+            if (ok) {
+                // Q_hat copy 0 = the group's rows in the top half (rows past
+                // them zeroed); copy 1 = the same rows in the bottom half. Rows r
+                // and r + 64 share their swizzle phase, so rows move as bytes.
+                const int nrow = rows_in_grp;                            // <= 64
+                uint4* q0 = reinterpret_cast<uint4*>(smem + C::OFF_Q);
+                uint4* q1 = reinterpret_cast<uint4*>(smem + C::OFF_Q + C::Q_BYTES);
+                constexpr int PER_ROW = C::QK_ROW / 16;
+                for (int k = lane; k < 128 * PER_ROW; k += 32) {
+                    const int r = k / PER_ROW;
+                    q1[k] = (r >= 64 && r - 64 < nrow) ? q0[k - 64 * PER_ROW] : make_uint4(0, 0, 0, 0);
+                }
+                __syncwarp();
+                for (int k = lane; k < 128 * PER_ROW; k += 32)
+                    if (k / PER_ROW >= nrow) q0[k] = make_uint4(0, 0, 0, 0);
+                // Q scales: rows r + 64 and r + 96 of each atom take rows r and
+                // r + 32 (bytes 8..15 of a 16-byte atom row = bytes 0..7)
+                for (int a = 0; a < C::KS; ++a) {
+                    uint2* row = reinterpret_cast<uint2*>(smem + C::OFF_SFQ + a * 512 + 16 * lane);
+                    row[1] = row[0];
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+            }
+        }
         bool issued_any = false;
         if (ok) {
             tc_fence_after();
             if (lane == 0) {
-                for (int qt = 0; qt < n_qt; ++qt) {
+                for (int qt = 0; qt < C::N_SFQ; ++qt) {
 #pragma unroll
                     for (int s = 0; s < C::KS; ++s)
                         tmem_cp_scale_atom(tmem + C::COL_SFQ + qt * 4 * C::KS + 4 * s,
                                            sf_desc(C::OFF_SFQ + qt * C::SFQK_BYTES + 512 * s));
+                }
+                for (int rg = 0; rg < C::N_SFV; ++rg) {
                     // scale atom of the normalizer rows (rows D.. of the V operand)
                     if constexpr (PREORDER && D >= 128) {
 #pragma unroll
                         for (int s = 0; s < 2; ++s)
-                            tmem_cp_scale_atom(tmem + C::COL_SFV + qt * 2 * C::SFV_PER_KS + s * C::SFV_PER_KS + 4 * C::NRB,
+                            tmem_cp_scale_atom(tmem + C::COL_SFV + rg * 2 * C::SFV_PER_KS + s * C::SFV_PER_KS + 4 * C::NRB,
                                                sf_desc(C::OFF_ONES));
                     }
                 }
                 if (more) {
-                    copy_sfk(0);
-                    for (int qt = 0; qt < n_qt; ++qt) copy_sfv(0, qt);
+                    if constexpr (DEC) {
+                        for (int i = 0; i < 4; ++i) {
+                            if (load_users(i) == 0) continue;
+                            if (i < 2) copy_sfk(i, i);
+                            copy_sfv(i, i);
+                        }
+                    } else {
+                        copy_sfk(0, 0);
+                        for (int qt = 0; qt < n_qt; ++qt) copy_sfv(0, qt);
+                    }
                     (void)issue_s(j, x);
                     issued_any = true;
                 }
@@ -442,6 +567,7 @@ __global__ void __launch_bounds__(Cfg<D, PREORDER>::THREADS, 1)
             int nj = 0, nx = 0;
             more = next_item(j, x, nj, nx);
             if (more && lane == 0 && !*abort_flag) {
+                tc_fence_after();
                 (void)issue_s(nj, nx);
                 issued_any = true;
             }
@@ -462,7 +588,7 @@ __global__ void __launch_bounds__(Cfg<D, PREORDER>::THREADS, 1)
         // rescaled (named barrier "P stored"), it issues the PV MMA.
         const int qt = warp - 2;
         bool issued_any = false;
-        // the warpgroup arrives on every kv tile, also after a failure
+        // the warpgroup arrives on every step, also after a failure
         for (int jj = 0; jj < n_tiles[qt]; ++jj) {
             named_barrier_sync(2 + 2 * qt, 160);
             if (lane == 0 && !*abort_flag) {
@@ -487,12 +613,16 @@ __global__ void __launch_bounds__(Cfg<D, PREORDER>::THREADS, 1)
         const int row = wq * 32 + lane;
         const uint32_t tl = tmem + ((uint32_t)(wq * 32) << 16);
         const uint32_t tO = tl + C::COL_O + qt * C::NO;
-        const int prow = (t0 + qt) * 128 + row;
+        const int half = DEC ? row >> 6 : 0;               // decode: which kv range of the tile
+        const int range = 2 * qt + half;
+        const int prow = DEC ? (row & 63) : (t0 + qt) * 128 + row;   // row within the group
         const bool valid = qt < n_qt && prow < rows_in_grp;
         const int qi = prow % p.Nq;
         const int last = valid ? (CAUSAL ? qi + p.Nkv - p.Nq : p.Nkv - 1) : -1;
         const size_t out_row = (size_t)grp * rows_in_grp + prow;
         const int nt = n_tiles[qt];
+        const int own_steps = DEC ? range_len(range) : nt;
+        const int kt0 = DEC ? range_begin(range) : 0;
         const float c = p.c;
         const float2 c2 = make_float2(c, c);
         const float one_sixth = rn_one_sixth();
@@ -518,18 +648,21 @@ __global__ void __launch_bounds__(Cfg<D, PREORDER>::THREADS, 1)
             }
             // every row has its scores: the S buffer is free for the next S MMA.
             // Arriving without waiting is safe while the waits succeed (this
-            // warpgroup cannot reach the next tile's arrival before the issuer
+            // warpgroup cannot reach the next step's arrival before the issuer
             // has passed this barrier: that S MMA is issued after it); after a
             // failure the waits no longer hold it back, so it syncs instead.
             if (ok) named_barrier_arrive(id_s, 160); else named_barrier_sync(id_s, 160);
             HIFA4_TRACE_POINT(qt, j, 2);
             if (ok) {
-                const int n0 = j * 128;
-                if (n0 + 127 > last) {
+                // this row's kv tile of the step; keys past `last` are masked
+                // (decode: a row whose range has ended masks the whole step)
+                const int n0 = (kt0 + j) * 128;
+                const int lim = j < own_steps ? last : -1;
+                if (n0 + 127 > lim) {
 #pragma unroll
                     for (int e = 0; e < 64; ++e) {
-                        if (n0 + 2 * e > last) S[e].x = -INFINITY;
-                        if (n0 + 2 * e + 1 > last) S[e].y = -INFINITY;
+                        if (n0 + 2 * e > lim) S[e].x = -INFINITY;
+                        if (n0 + 2 * e + 1 > lim) S[e].y = -INFINITY;
                     }
                 }
                 // block maxima of S (they also give the block maxima of P: 2^x is monotone)
@@ -601,7 +734,7 @@ __global__ void __launch_bounds__(Cfg<D, PREORDER>::THREADS, 1)
                 HIFA4_TRACE_POINT(qt, j, 5);
                 if constexpr (!PREORDER) l_hp = __fmaf_rn(alpha, l_hp, lsum2.x + lsum2.y);
                 {
-                    const uint32_t pb = sbase + C::OFF_P + (qt * 2 + (j & 1)) * C::P_BYTES;
+                    const uint32_t pb = sbase + C::OFF_P + (qt * 2 + (DEC ? half : (j & 1))) * C::P_BYTES;
 #pragma unroll
                     for (int q = 0; q < 4; ++q)
                         sts_v4(pb + p_swizzle64(row, q), code[4 * q], code[4 * q + 1], code[4 * q + 2], code[4 * q + 3]);
@@ -613,7 +746,7 @@ __global__ void __launch_bounds__(Cfg<D, PREORDER>::THREADS, 1)
                     tmem_wait_st();
                     if constexpr (DUMP) {
                         // debug copy of this row's P_hat codes and scales
-                        if (valid) {
+                        if (valid && j < own_steps) {
                             uint4* dc = reinterpret_cast<uint4*>(p.p_codes + out_row * (size_t)(p.Nkv / 2) + n0 / 2);
 #pragma unroll
                             for (int q = 0; q < 4; ++q)
@@ -634,9 +767,9 @@ __global__ void __launch_bounds__(Cfg<D, PREORDER>::THREADS, 1)
         }
         // ---------------------------------------------------------- epilogue
         if (ok && nt > 0) ok = __all_sync(0xFFFFFFFFu, mbar_wait(&bars->o_done[qt], (nt - 1) & 1, ctl));
+        float l = 0.0f;
         if (ok && nt > 0) {
             tc_fence_after();
-            float l;
             if constexpr (PREORDER) {
                 uint32_t lv;
                 tmem_ld1(tO + D, lv);
@@ -645,22 +778,91 @@ __global__ void __launch_bounds__(Cfg<D, PREORDER>::THREADS, 1)
             } else {
                 l = l_hp;
             }
-            const float inv = l > 0.0f ? __frcp_rn(l) : 0.0f;
+        }
+        if constexpr (!DEC) {
+            if (ok && nt > 0) {
+                const float inv = l > 0.0f ? __frcp_rn(l) : 0.0f;
 #pragma unroll 1
-            for (int cc = 0; cc < D; cc += 32) {
-                uint32_t o[32];
-                tmem_ld32(tO + cc, o);
-                tmem_wait_ld_dep(o);
-                float v[32];
+                for (int cc = 0; cc < D; cc += 32) {
+                    uint32_t o[32];
+                    tmem_ld32(tO + cc, o);
+                    tmem_wait_ld_dep(o);
+                    float v[32];
 #pragma unroll
-                for (int e = 0; e < 32; ++e) v[e] = __uint_as_float(o[e]) * inv;
-                if (valid) {
-                    uint8_t* dst = reinterpret_cast<uint8_t*>(p.o) + (out_row * D + cc) * (OUT == 2 ? 4 : 2);
-                    store_out32<OUT>(dst, v);
+                    for (int e = 0; e < 32; ++e) v[e] = __uint_as_float(o[e]) * inv;
+                    if (valid) {
+                        uint8_t* dst = reinterpret_cast<uint8_t*>(p.o) + (out_row * D + cc) * (OUT == 2 ? 4 : 2);
+                        store_out<OUT, 32>(dst, v);
+                    }
+                }
+                if (valid && p.lse != nullptr)
+                    p.lse[out_row] = l > 0.0f ? mc_old * 0.69314718055994531f + __logf(l) : -INFINITY;
+            }
+        } else {
+            // merge the four kv ranges of each row. After the first barrier all
+            // MMAs of both tiles are done (every thread waited for its tile's
+            // last PV), so the K/V ring and the P buffers are free scratch.
+            float* part = reinterpret_cast<float*>(smem + C::OFF_K);          // [range][row][MERGE_ROW]
+            float2* ml = reinterpret_cast<float2*>(smem + C::OFF_P);          // [range][row] = (mc, l)
+            named_barrier_sync(5, 128 * NQT);
+            const bool mine = ok && valid && l > 0.0f;
+            if (valid) ml[range * 64 + prow] = mine ? make_float2(mc_old, l) : make_float2(0.0f, 0.0f);
+            named_barrier_sync(5, 128 * NQT);
+            float M = -INFINITY, L = 0.0f;
+            if (valid) {
+#pragma unroll
+                for (int r = 0; r < kDecSplits; ++r) {
+                    const float2 e = ml[r * 64 + prow];
+                    if (e.y > 0.0f) M = fmaxf(M, e.x);
+                }
+#pragma unroll
+                for (int r = 0; r < kDecSplits; ++r) {
+                    const float2 e = ml[r * 64 + prow];
+                    if (e.y > 0.0f) L = __fmaf_rn(ex2_approx(e.x - M), e.y, L);
                 }
             }
-            if (valid && p.lse != nullptr)
-                p.lse[out_row] = l > 0.0f ? mc_old * 0.69314718055994531f + __logf(l) : -INFINITY;
+            const float wgt = (mine && L > 0.0f) ? __fdividef(ex2_approx(mc_old - M), L) : 0.0f;
+            if (valid) {
+                float* dst = part + ((size_t)range * 64 + prow) * C::MERGE_ROW;
+#pragma unroll 1
+                for (int cc = 0; cc < D; cc += 32) {
+                    uint32_t o[32];
+                    if (mine) {
+                        tmem_ld32(tO + cc, o);
+                        tmem_wait_ld_dep(o);
+                    }
+#pragma unroll
+                    for (int e = 0; e < 32; e += 4)
+                        *reinterpret_cast<float4*>(dst + cc + e) =
+                            mine ? make_float4(__uint_as_float(o[e]) * wgt, __uint_as_float(o[e + 1]) * wgt,
+                                               __uint_as_float(o[e + 2]) * wgt, __uint_as_float(o[e + 3]) * wgt)
+                                 : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+                }
+            }
+            named_barrier_sync(5, 128 * NQT);
+            // thread (range r, row q) writes columns [r*D/4, (r+1)*D/4) of row q
+            constexpr int CW = D / kDecSplits;
+            if (valid && ok) {
+                float v[CW];
+#pragma unroll
+                for (int e = 0; e < CW; ++e) v[e] = 0.0f;
+#pragma unroll
+                for (int r = 0; r < kDecSplits; ++r) {
+                    const float* src = part + ((size_t)r * 64 + prow) * C::MERGE_ROW + range * CW;
+#pragma unroll
+                    for (int e = 0; e < CW; e += 4) {
+                        const float4 t4 = *reinterpret_cast<const float4*>(src + e);
+                        v[e] += t4.x;
+                        v[e + 1] += t4.y;
+                        v[e + 2] += t4.z;
+                        v[e + 3] += t4.w;
+                    }
+                }
+                uint8_t* dst = reinterpret_cast<uint8_t*>(p.o) + (out_row * D + range * CW) * (OUT == 2 ? 4 : 2);
+                store_out<OUT, CW>(dst, v);
+                if (range == 0 && p.lse != nullptr)
+                    p.lse[out_row] = L > 0.0f ? M * 0.69314718055994531f + __logf(L) : -INFINITY;
+            }
         }
     }
     // ---------------------------------------------------------------- teardown
@@ -670,11 +872,11 @@ __global__ void __launch_bounds__(Cfg<D, PREORDER>::THREADS, 1)
     if (warp == 1) tmem_dealloc(tmem, 512);
 }
 
-template <int D, bool PRE, bool CAUSAL, int OUT, bool DUMP>
+template <int D, bool PRE, bool CAUSAL, int OUT, bool DUMP, bool DEC>
 static cudaError_t launch_one(const CUtensorMap* q, const CUtensorMap* k, const CUtensorMap* v, const AttnParams& p,
                               cudaStream_t st) {
-    using C = Cfg<D, PRE>;
-    auto kern = attn_fwd_kernel<D, PRE, CAUSAL, OUT, DUMP>;
+    using C = Cfg<D, PRE, DEC>;
+    auto kern = attn_fwd_kernel<D, PRE, CAUSAL, OUT, DUMP, DEC>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t lc{};
@@ -690,40 +892,51 @@ static cudaError_t launch_one(const CUtensorMap* q, const CUtensorMap* k, const 
     return cudaLaunchKernelEx(&lc, kern, *q, *k, *v, p);
 }
 
+template <int D, bool PRE, bool CAUSAL, int OUT, bool DUMP>
+static cudaError_t launch_dec(const CUtensorMap* q, const CUtensorMap* k, const CUtensorMap* v, const AttnParams& p,
+                              bool dec, cudaStream_t st) {
+    if constexpr (D <= 128) {
+        if (dec) return launch_one<D, PRE, CAUSAL, OUT, DUMP, true>(q, k, v, p, st);
+    } else {
+        if (dec) return cudaErrorInvalidValue;
+    }
+    return launch_one<D, PRE, CAUSAL, OUT, DUMP, false>(q, k, v, p, st);
+}
+
 template <int D, bool PRE, bool CAUSAL, int OUT>
 static cudaError_t launch_dump(const CUtensorMap* q, const CUtensorMap* k, const CUtensorMap* v, const AttnParams& p,
-                               bool dump, cudaStream_t st) {
-    return dump ? launch_one<D, PRE, CAUSAL, OUT, true>(q, k, v, p, st)
-                : launch_one<D, PRE, CAUSAL, OUT, false>(q, k, v, p, st);
+                               bool dump, bool dec, cudaStream_t st) {
+    return dump ? launch_dec<D, PRE, CAUSAL, OUT, true>(q, k, v, p, dec, st)
+                : launch_dec<D, PRE, CAUSAL, OUT, false>(q, k, v, p, dec, st);
 }
 
 template <int D, bool PRE, bool CAUSAL>
 static cudaError_t launch_out(const CUtensorMap* q, const CUtensorMap* k, const CUtensorMap* v, const AttnParams& p,
-                              int out, bool dump, cudaStream_t st) {
+                              int out, bool dump, bool dec, cudaStream_t st) {
     switch (out) {
-        case 0: return launch_dump<D, PRE, CAUSAL, 0>(q, k, v, p, dump, st);
-        case 1: return launch_dump<D, PRE, CAUSAL, 1>(q, k, v, p, dump, st);
-        default: return launch_dump<D, PRE, CAUSAL, 2>(q, k, v, p, dump, st);
+        case 0: return launch_dump<D, PRE, CAUSAL, 0>(q, k, v, p, dump, dec, st);
+        case 1: return launch_dump<D, PRE, CAUSAL, 1>(q, k, v, p, dump, dec, st);
+        default: return launch_dump<D, PRE, CAUSAL, 2>(q, k, v, p, dump, dec, st);
     }
 }
 
 template <int D>
 static cudaError_t launch_d(const CUtensorMap* q, const CUtensorMap* k, const CUtensorMap* v, const AttnParams& p,
-                            int norm, bool causal, int out, bool dump, cudaStream_t st) {
+                            int norm, bool causal, int out, bool dump, bool dec, cudaStream_t st) {
     if (norm == 0)
-        return causal ? launch_out<D, true, true>(q, k, v, p, out, dump, st)
-                      : launch_out<D, true, false>(q, k, v, p, out, dump, st);
-    return causal ? launch_out<D, false, true>(q, k, v, p, out, dump, st)
-                  : launch_out<D, false, false>(q, k, v, p, out, dump, st);
+        return causal ? launch_out<D, true, true>(q, k, v, p, out, dump, dec, st)
+                      : launch_out<D, true, false>(q, k, v, p, out, dump, dec, st);
+    return causal ? launch_out<D, false, true>(q, k, v, p, out, dump, dec, st)
+                  : launch_out<D, false, false>(q, k, v, p, out, dump, dec, st);
 }
 
 cudaError_t launch_attention(const CUtensorMap* tmQ, const CUtensorMap* tmK, const CUtensorMap* tmV,
-                             const AttnParams& p, int D, int norm, bool causal, int out_dtype, bool dump,
+                             const AttnParams& p, int D, int norm, bool causal, int out_dtype, bool dump, bool dec,
                              cudaStream_t st) {
     switch (D) {
-        case 64: return launch_d<64>(tmQ, tmK, tmV, p, norm, causal, out_dtype, dump, st);
-        case 128: return launch_d<128>(tmQ, tmK, tmV, p, norm, causal, out_dtype, dump, st);
-        case 256: return launch_d<256>(tmQ, tmK, tmV, p, norm, causal, out_dtype, dump, st);
+        case 64: return launch_d<64>(tmQ, tmK, tmV, p, norm, causal, out_dtype, dump, dec, st);
+        case 128: return launch_d<128>(tmQ, tmK, tmV, p, norm, causal, out_dtype, dump, dec, st);
+        case 256: return launch_d<256>(tmQ, tmK, tmV, p, norm, causal, out_dtype, dump, dec, st);
         default: return cudaErrorInvalidValue;
     }
 }

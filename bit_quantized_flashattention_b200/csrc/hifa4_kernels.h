@@ -38,7 +38,7 @@ struct AttnParams {
     int B, Hq, Hkv, Nq, Nkv, G;
     int Tq;                  // 128-row tiles per (b, kv head) group
     int n_kv_tiles;          // Nkv / 128
-    int n_work;              // grid size = B * Hkv * Tq
+    int n_work;              // grid size (work units)
     int heavy_first;         // causal: longest tiles first
     float c;                 // RN(sm_scale * log2 e)
     unsigned long long wait_limit_ns;
@@ -46,9 +46,13 @@ struct AttnParams {
 };
 
 // D in {64,128,256}; norm 0 = P-Reordering, 1 = high-precision l;
-// out_dtype 0 = f16, 1 = bf16, 2 = f32.
+// out_dtype 0 = f16, 1 = bf16, 2 = f32; dec: split-kv decode mode (D <= 128,
+// G*Nq <= 64, at least 4 kv tiles; one CTA per group).
 cudaError_t launch_attention(const CUtensorMap* tmQ, const CUtensorMap* tmK, const CUtensorMap* tmV,
-                             const AttnParams& p, int D, int norm, bool causal, int out_dtype, bool dump,
+                             const AttnParams& p, int D, int norm, bool causal, int out_dtype, bool dump, bool dec,
                              cudaStream_t st);
+
+// Number of contiguous kv ranges the decode mode cuts the keys into.
+constexpr int kDecodeSplits = 4;
 
 }  // namespace hifa4

@@ -58,7 +58,17 @@ typedef enum { HIFA4_NORM_P_REORDER = 0, HIFA4_NORM_HIGH_PRECISION_L = 1 } hifa4
 
 typedef enum { HIFA4_F16 = 0, HIFA4_BF16 = 1, HIFA4_F32 = 2 } hifa4_dtype;
 
-enum { HIFA4_CAUSAL = 1u << 0 };
+/* Flags of the attention calls.
+ * HIFA4_CAUSAL    bottom-right aligned causal mask.
+ * HIFA4_SPLIT_KV  inference option (flash-decoding): the kernels may cut the
+ *                 kv tiles into hifa4_attention_splits() contiguous ranges, run
+ *                 the online softmax of each range from its own start (its own
+ *                 running max, so P_hat is taken relative to the range's max),
+ *                 and merge the ranges with their log-sum-exp weights:
+ *                 O = sum_r 2^(mc_r - M) O_acc_r / sum_r 2^(mc_r - M) l_r,
+ *                 M = max mc_r, LSE = M ln 2 + ln(sum_r 2^(mc_r - M) l_r).
+ *                 With one range this is the plain pass. */
+enum { HIFA4_CAUSAL = 1u << 0, HIFA4_SPLIT_KV = 1u << 1 };
 
 /* Quantized operands. Layouts (u8 everywhere; codes hold two E2M1 elements
  * per byte, element 2i in the low nibble; scales are E4M3 bytes):
@@ -91,6 +101,13 @@ typedef struct {
 /* Bytes of each packed buffer, in the order qc, qs, kc, ks, vtc, vts, written
  * to out[6] (may be NULL). Returns their sum, or 0 for an unsupported shape. */
 size_t hifa4_packed_bytes(int B, int Hq, int Hkv, int Nq, int Nkv, int D, size_t out[6]);
+
+/* Number of kv ranges the attention calls use for this shape and flags: 4 when
+ * HIFA4_SPLIT_KV is set, D <= 128, a group's query rows fit in half a tile
+ * (Hq/Hkv * Nq <= 64: decode-style chunks) and Nkv >= 512; otherwise 1 (the
+ * plain pass). Range r covers the kv tiles [T*r/n, T*(r+1)/n), T = Nkv/128.
+ * Returns 0 for an unsupported shape. */
+int hifa4_attention_splits(int B, int Hq, int Hkv, int Nq, int Nkv, int D, unsigned flags);
 
 /* Bytes of the device workspace hifa4_attention_fwd needs: one status word
  * (padded to 256 bytes). The caller zeroes it once after allocating; a kernel
@@ -137,7 +154,8 @@ hifa4_status hifa4_quantize_kv(const void* k, const void* v, hifa4_dtype dtype,
  * normalizer l per `norm` (see hifa4_norm_mode). Output O = O_acc / l in
  * `o_dtype` [B,Hq,Nq,D]; lse (fp32 [B,Hq,Nq], may be NULL) =
  * RN(m*c)*ln 2 + ln l, the natural-log log-sum-exp of sm_scale*S.
- * sm_scale: finite and > 0 (1/sqrt(D) is the usual value). flags: HIFA4_CAUSAL.
+ * sm_scale: finite and > 0 (1/sqrt(D) is the usual value). flags: HIFA4_CAUSAL,
+ * HIFA4_SPLIT_KV (see above).
  * workspace: hifa4_workspace_bytes() bytes, zeroed once by the caller; a
  * bounded wait that expires inside the kernel records HIFA4_ERR_TIMEOUT there
  * (read it with hifa4_get_status). Concurrent calls must use different

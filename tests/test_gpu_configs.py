@@ -34,6 +34,7 @@ def H():
 
 
 ALL_ROWS = (1, 2)          # configs compared on every group and row
+SPLIT_KV = (5,)            # decode-style configs run (and are timed) in the split-kv mode
 
 
 def _sample_groups(cfg, rng):
@@ -68,9 +69,11 @@ def test_config_parity(H, index):
     pk = H.quantize_qkv(q, k, v, s, s_inv)
     dump = True                # the P_hat dump fits on a B200 for every config (8.6 GB at config 4)
     results = {}
+    split = cfg.index in SPLIT_KV
+    n_splits = H.attention_splits(cfg.B, cfg.Hq, cfg.Hkv, cfg.Nq, cfg.Nkv, cfg.D, causal=cfg.causal, split_kv=split)
     for norm in cfg.modes:
-        o, lse, pc, ps = H.attention_fwd_debug(pk, causal=cfg.causal, norm=norm)
-        o_bf16, _ = H.attention_fwd(pk, causal=cfg.causal, norm=norm, out_dtype=torch.bfloat16)
+        o, lse, pc, ps = H.attention_fwd_debug(pk, causal=cfg.causal, norm=norm, split_kv=split)
+        o_bf16, _ = H.attention_fwd(pk, causal=cfg.causal, norm=norm, out_dtype=torch.bfloat16, split_kv=split)
         torch.cuda.synchronize()
         results[norm] = (o, lse, pc, ps, o_bf16)
 
@@ -98,7 +101,7 @@ def test_config_parity(H, index):
             o, lse, pc, ps, o_bf16 = results[norm]
             ref = oracle.attention_rows((1, G, 1, cfg.Nq, cfg.Nkv, cfg.D), rows_local, packed=ref_p,
                                         causal=cfg.causal, norm_mode=0 if norm == "p_reorder" else 1,
-                                        want_p=dump)
+                                        want_p=dump, n_splits=n_splits)
             og = o[b, hs][:, idx].reshape(-1, cfg.D).float().cpu().numpy()
             max_abs, rel = U.row_errors(og, ref["O"])
             assert max_abs <= O_MAX_ABS, (norm, b, g, max_abs)

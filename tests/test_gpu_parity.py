@@ -247,3 +247,31 @@ def test_quantize_kv_matches_oracle(H, shape, dtype, smooth):
     assert np.array_equal(ks_g, ks)
     assert np.array_equal(pk.vtc.cpu().numpy().reshape(vtc.shape), vtc)
     assert np.array_equal(vts_g, vts)
+
+
+@pytest.mark.parametrize("shape,causal", [
+    ((1, 8, 2, 16, 512, 128), False),          # 4 heads x 16 queries = 64 rows per group, 4 ranges of 1 tile
+    ((2, 4, 1, 16, 640, 64), True),            # 5 tiles over 4 ranges (ragged), causal, D = 64
+    ((1, 2, 2, 32, 1024, 128), False),         # 32 rows per group (half of each range's lanes idle)
+    ((1, 4, 1, 16, 384, 128), False),          # 3 tiles: too few for 4 ranges -> one pass
+])
+@pytest.mark.parametrize("norm", ["p_reorder", "high_precision_l"])
+def test_attention_split_kv_matches_oracle(H, shape, causal, norm):
+    """Split-kv decode mode (HIFA4_SPLIT_KV): the library reports its range
+    count, and the oracle with that many ranges is the reference (P_hat relative
+    to each range's own running max, ranges merged by log-sum-exp weights)."""
+    B, Hq, Hkv, Nq, Nkv, D = shape
+    n_splits = H.attention_splits(B, Hq, Hkv, Nq, Nkv, D, causal=causal, split_kv=True)
+    assert n_splits == (1 if Nkv < 512 else 4)
+    rng = np.random.default_rng(18)
+    q = W.round_to_dtype(_rand(rng, (B, Hq, Nq, D)), "bf16")
+    k = W.round_to_dtype(_rand(rng, (B, Hkv, Nkv, D)) * rng.lognormal(0, 1, (1, Hkv, 1, D)).astype(np.float32), "bf16")
+    v = W.round_to_dtype(_rand(rng, (B, Hkv, Nkv, D)), "bf16")
+    s, si = oracle.calibrate(q, k)
+    pk = _gpu_quant(H, q, k, v, "bf16", s, si)
+    o, lse, pc, ps = H.attention_fwd_debug(pk, causal=causal, norm=norm, split_kv=True)
+    torch.cuda.synchronize()
+    ref_p = oracle.quantize_qkv(q, k, v, s, si)
+    ref = oracle.attention_rows(shape, oracle.all_rows(B, Hq, Nq), packed=ref_p, causal=causal,
+                                norm_mode=0 if norm == "p_reorder" else 1, want_p=True, n_splits=n_splits)
+    _check_attention(o, lse, pc, ps, ref, D)
