@@ -110,7 +110,7 @@ hifa4_status hifa4::check_attention_args(const hifa4_packed* in, int B, int Hq, 
         if (q == nullptr || !aligned16(q)) return HIFA4_ERR_INVALID_ARG;
     if (!aligned16(o) || (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u))) return HIFA4_ERR_INVALID_ARG;
     const long long rows_q = (long long)B * Hq * Nq, rows_k = (long long)B * Hkv * Nkv, rows_v = (long long)B * Hkv * D;
-    if (rows_q > INT32_MAX || rows_k > INT32_MAX || rows_v > INT32_MAX) return HIFA4_ERR_UNSUPPORTED;
+    if (rows_q > INT32_MAX || rows_k > INT32_MAX || rows_v * (Nkv / 128) > INT32_MAX) return HIFA4_ERR_UNSUPPORTED;
     const Sizes sz = sizes_of(B, Hq, Hkv, Nq, Nkv, D);
     const int nqt = D == 256 ? 1 : 2;              // query tiles per CTA (see attention.cu)
     if ((long long)B * Hkv * ((sz.Tq + nqt - 1) / nqt) > INT32_MAX) return HIFA4_ERR_UNSUPPORTED;
@@ -139,7 +139,7 @@ hifa4_status attention_impl(const hifa4_packed* in, int B, int Hq, int Hkv, int 
     CUtensorMap tq, tk, tv;
     if (!make_map(&tq, in->qc, (uint64_t)D / 2, (uint64_t)rows_q, D / 2, 128, swz_qk) ||
         !make_map(&tk, in->kc, (uint64_t)D / 2, (uint64_t)rows_k, D / 2, 128, swz_qk) ||
-        !make_map(&tv, in->vtc, (uint64_t)Nkv / 2, (uint64_t)rows_v, 64, (uint32_t)D, CU_TENSOR_MAP_SWIZZLE_64B))
+        !make_map(&tv, in->vtc, 64, (uint64_t)rows_v * (Nkv / 128), 64, (uint32_t)D, CU_TENSOR_MAP_SWIZZLE_64B))
         return from_cuda(cudaErrorInvalidValue);
 
     AttnParams p{};

@@ -54,14 +54,21 @@
 namespace hifa4 {
 
 constexpr int kSmWarp0 = 4;          // first softmax warp (0: loads, 1: TMEM owner + S MMAs, 2-3: PV MMAs)
-constexpr int kMaxStages = 8;
+constexpr int kMaxStages = 12;
 constexpr int kDecSplits = 4;        // kv ranges of the split-kv decode mode
 
 template <int D, bool PREORDER, bool DEC>
 struct Cfg {
     static_assert(!DEC || D <= 128, "decode mode needs two query tiles per CTA");
     static constexpr int NQT = D == 256 ? 1 : 2;          // 128-row query tiles per CTA
-    static constexpr int STAGES = DEC ? 8 : 4;            // kv tiles in flight (decode: 4 per step)
+    // ring slots of K and of V tiles (decode: 4 loads per step; K is read a
+    // step before V, so its ring runs further ahead)
+    static constexpr int STK = DEC ? 8 : 4;
+    static constexpr int STV = DEC ? 8 : 4;
+    // every slot of a ring must always hold loads of the same query tile (the
+    // empty-barrier parities count that tile's uses of the slot): in decode
+    // mode the loads of a step alternate between tiles, so depths are multiples of 4
+    static_assert(!DEC || (STK % 4 == 0 && STV % 4 == 0), "ring depth");
     static constexpr int THREADS = 128 + 128 * NQT;
     static constexpr int KS = D / 64;                     // 64-wide K steps of QK^T
     static constexpr int QK_ROW = D / 2;                  // bytes per Q/K row
@@ -96,15 +103,15 @@ struct Cfg {
     // shared memory offsets (operand tiles 1024-aligned)
     static constexpr int OFF_Q = 0;                                       // + buffer * Q_BYTES
     static constexpr int OFF_K = OFF_Q + NQT * Q_BYTES;
-    static constexpr int OFF_V = OFF_K + STAGES * K_BYTES;
-    static constexpr int OFF_P = OFF_V + STAGES * V_STRIDE;              // + (qt * 2 + buf) * P_BYTES
+    static constexpr int OFF_V = OFF_K + STK * K_BYTES;
+    static constexpr int OFF_P = OFF_V + STV * V_STRIDE;                 // + (qt * 2 + buf) * P_BYTES
     static constexpr int OFF_SFQ = OFF_P + NQT * 2 * P_BYTES;             // + qt * SFQK_BYTES
     static constexpr int OFF_SFK = OFF_SFQ + NQT * SFQK_BYTES;
-    static constexpr int OFF_SFV = OFF_SFK + STAGES * SFQK_BYTES;
-    static constexpr int OFF_ONES = OFF_SFV + STAGES * SFV_BYTES;
+    static constexpr int OFF_SFV = OFF_SFK + STK * SFQK_BYTES;
+    static constexpr int OFF_ONES = OFF_SFV + STV * SFV_BYTES;
     static constexpr int OFF_LUT = OFF_ONES + 512;                        // float [128]
     static constexpr int OFF_BAR = OFF_LUT + 128 * 4;
-    static constexpr int OFF_MISC = OFF_BAR + 512;
+    static constexpr int OFF_MISC = OFF_BAR + 1024;
     static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;              // + alignment slack
     static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
     // decode merge scratch, after the loop: partial O rows (fp32, rows padded by
@@ -117,12 +124,13 @@ struct Bars {
     uint64_t q_full;
     uint64_t k_full[kMaxStages];
     uint64_t v_full[kMaxStages];
-    uint64_t v_empty[kMaxStages][2];   // K and V slot no longer read by query tile x's MMAs
+    uint64_t k_empty[kMaxStages][2];   // K slot no longer read by query tile x's S MMA
+    uint64_t v_empty[kMaxStages][2];   // V slot no longer read by query tile x's PV MMA
     uint64_t s_full[2];                // S of query tile x is in TMEM
     uint64_t o_done[2];                // PV MMA of query tile x finished
     uint64_t drain[3];                 // teardown: MMAs issued by the S issuer / each PV issuer
 };
-static_assert(sizeof(Bars) <= 512, "barrier area");
+static_assert(sizeof(Bars) <= 1024, "barrier area");
 
 #ifndef HIFA4_TRACE_POINT
 #define HIFA4_TRACE_POINT(role, j, e)
@@ -181,7 +189,7 @@ __global__ void __launch_bounds__(Cfg<D, PREORDER, DEC>::THREADS, 1)
                     const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
     using C = Cfg<D, PREORDER, DEC>;
     constexpr int NQT = C::NQT;
-    constexpr int ST = C::STAGES;
+    constexpr int STK = C::STK, STV = C::STV;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     Bars* bars = reinterpret_cast<Bars*>(smem + C::OFF_BAR);
@@ -256,11 +264,15 @@ __global__ void __launch_bounds__(Cfg<D, PREORDER, DEC>::THREADS, 1)
 
     // --------------------------------------------------------------- setup
     if (threadIdx.x == 0) {
+        HIFA4_TRACE_POINT(4, 63, 0);
         mbar_init(&bars->q_full, 1);
-        for (int s = 0; s < ST; ++s) {
+        for (int s = 0; s < kMaxStages; ++s) {
             mbar_init(&bars->k_full[s], 1);
             mbar_init(&bars->v_full[s], 1);
-            for (int x = 0; x < 2; ++x) mbar_init(&bars->v_empty[s][x], 1);
+            for (int x = 0; x < 2; ++x) {
+                mbar_init(&bars->k_empty[s][x], 1);
+                mbar_init(&bars->v_empty[s][x], 1);
+            }
         }
         for (int x = 0; x < 2; ++x) {
             mbar_init(&bars->s_full[x], 1);
@@ -276,7 +288,7 @@ __global__ void __launch_bounds__(Cfg<D, PREORDER, DEC>::THREADS, 1)
         // normalizer block of V^T (rows D..D+15 of every stage): one row of E2M1
         // ones (code 2 in both nibbles), zero rows; and the scale atom of the
         // ones row (row 0 of an atom = 1.0) used when D >= 128.
-        for (int s = 0; s < ST; ++s) {
+        for (int s = 0; s < STV; ++s) {
             uint32_t* row = reinterpret_cast<uint32_t*>(smem + C::OFF_V + s * C::V_STRIDE + D * 64);
             for (int k = i; k < 16 * 16; k += 128) row[k] = (k < 16) ? 0x22222222u : 0u;
         }
@@ -319,14 +331,14 @@ __global__ void __launch_bounds__(Cfg<D, PREORDER, DEC>::THREADS, 1)
     // last query tile (in S order) that visits plain-mode kv tile j
     auto last_x_of = [&](int j) -> int { return (NQT > 1 && j < n_tiles[1]) ? 1 : 0; };
     auto copy_sfk = [&](int li, int region) {
-        const int st = li % ST;
+        const int st = li % STK;
 #pragma unroll
         for (int s = 0; s < C::KS; ++s)
             tmem_cp_scale_atom(tmem + C::COL_SFK + region * 4 * C::KS + 4 * s,
                                sf_desc(C::OFF_SFK + st * C::SFQK_BYTES + 512 * s));
     };
     auto copy_sfv = [&](int li, int region) {
-        const int st = li % ST;
+        const int st = li % STV;
         const uint32_t sfv = C::OFF_SFV + st * C::SFV_BYTES;
         const uint32_t col = C::COL_SFV + region * 2 * C::SFV_PER_KS;
 #pragma unroll
@@ -346,12 +358,12 @@ __global__ void __launch_bounds__(Cfg<D, PREORDER, DEC>::THREADS, 1)
             for (int h = 0; h < 2; ++h) {
                 const int li = 4 * nj + 2 * nx + h;
                 if (!(load_users(li) & (1 << nx))) continue;
-                if (!mbar_wait_poll(&bars->k_full[li % ST], (li / ST) & 1, ctl, 32)) return false;
+                if (!mbar_wait_poll(&bars->k_full[li % STK], (li / STK) & 1, ctl, 32)) return false;
                 copy_sfk(li, h);
             }
         } else {
             if (nj == j) return true;
-            if (!mbar_wait_poll(&bars->k_full[nj % ST], (nj / ST) & 1, ctl, 32)) return false;
+            if (!mbar_wait_poll(&bars->k_full[nj % STK], (nj / STK) & 1, ctl, 32)) return false;
             copy_sfk(nj, 0);
         }
         return true;
@@ -364,7 +376,7 @@ __global__ void __launch_bounds__(Cfg<D, PREORDER, DEC>::THREADS, 1)
         for (int h = 0; h < (DEC ? 2 : 1); ++h) {
             const int li = DEC ? 4 * j + 2 * x + h : j;
             if (DEC && !(load_users(li) & (1 << x))) continue;
-            const int st = li % ST;
+            const int st = li % STK;
             const uint64_t kd = qk_desc0 + ((C::OFF_K + st * C::K_BYTES) >> 4);
             const uint64_t qd = qk_desc0 + ((C::OFF_Q + (DEC ? h : x) * C::Q_BYTES) >> 4);
             const uint32_t sfq = tmem + C::COL_SFQ + (DEC ? 0 : x) * 4 * C::KS;
@@ -376,6 +388,11 @@ __global__ void __launch_bounds__(Cfg<D, PREORDER, DEC>::THREADS, 1)
             first = false;
         }
         tc_commit(&bars->s_full[x]);
+#pragma unroll
+        for (int h = 0; h < (DEC ? 2 : 1); ++h) {
+            const int li = DEC ? 4 * j + 2 * x + h : j;
+            if (load_users(li) & (1 << x)) tc_commit(&bars->k_empty[li % STK][x]);
+        }
         if (!DEC && !(x == last_x_of(j))) return true;
         return prefetch_sfk(j, x);
     };
@@ -388,7 +405,7 @@ __global__ void __launch_bounds__(Cfg<D, PREORDER, DEC>::THREADS, 1)
         for (int h = 0; h < (DEC ? 2 : 1); ++h) {
             const int li = DEC ? 4 * j + 2 * x + h : j;
             if (DEC && !(load_users(li) & (1 << x))) continue;
-            const int st = li % ST;
+            const int st = li % STV;
             const uint64_t vd = pv_desc0 + ((C::OFF_V + st * C::V_STRIDE) >> 4);
             const uint64_t pd = pv_desc0 + ((C::OFF_P + (x * 2 + (DEC ? h : (j & 1))) * C::P_BYTES) >> 4);
             const uint32_t col_sfv = C::COL_SFV + (DEC ? 2 * x + h : x) * 2 * C::SFV_PER_KS;
@@ -411,14 +428,14 @@ __global__ void __launch_bounds__(Cfg<D, PREORDER, DEC>::THREADS, 1)
 #pragma unroll
         for (int h = 0; h < (DEC ? 2 : 1); ++h) {
             const int li = DEC ? 4 * j + 2 * x + h : j;
-            if (load_users(li) & (1 << x)) tc_commit(&bars->v_empty[li % ST][x]);
+            if (load_users(li) & (1 << x)) tc_commit(&bars->v_empty[li % STV][x]);
         }
         if (j + 1 < n_tiles[x]) {
 #pragma unroll
             for (int h = 0; h < (DEC ? 2 : 1); ++h) {
                 const int li = DEC ? 4 * (j + 1) + 2 * x + h : j + 1;
                 if (!(load_users(li) & (1 << x))) continue;
-                if (!mbar_wait_poll(&bars->v_full[li % ST], (li / ST) & 1, ctl, 32)) return false;
+                if (!mbar_wait_poll(&bars->v_full[li % STV], (li / STV) & 1, ctl, 32)) return false;
                 copy_sfv(li, DEC ? 2 * x + h : x);
             }
         }
@@ -431,12 +448,9 @@ __global__ void __launch_bounds__(Cfg<D, PREORDER, DEC>::THREADS, 1)
         // stream (programmatic dependent launch); the packed operands are read
         // only after it has completed. Every other read of those operands
         // goes through this warp's copies. A slot is refilled once every query
-        // tile that read the previous load in it has released it (a finished
-        // PV MMA of that load also means its S MMA finished).
+        // tile that read the previous load in it has released it.
         grid_dependency_wait();
         if (lane == 0 && !p.stall_loads) {
-            int issued = 0;
-            bool ok = true;
             const int nq_load = DEC ? 1 : n_qt;
             mbar_arrive_expect_tx(&bars->q_full, nq_load * (C::Q_BYTES + C::SFQK_BYTES));
             for (int qt = 0; qt < nq_load; ++qt) {
@@ -445,39 +459,71 @@ __global__ void __launch_bounds__(Cfg<D, PREORDER, DEC>::THREADS, 1)
                 bulk_load(smem + C::OFF_SFQ + qt * C::SFQK_BYTES,
                           p.qs + ((size_t)grp * p.Tq + t0 + qt) * C::SFQK_BYTES, C::SFQK_BYTES, &bars->q_full);
             }
-            for (int i = 0; i < n_loads && ok; ++i) {
-                const int st = i % ST;
-                const int ip = i - ST;                               // previous load in this slot
-                if (ip >= 0) {
-                    const int users = load_users(ip);
-                    const uint32_t ph = (ip / ST) & 1;
-                    for (int x = 0; x < NQT && ok; ++x)
-                        if ((users >> x) & 1) ok = mbar_wait_poll(&bars->v_empty[st][x], ph, ctl, 256);
+            // K and V go through their rings independently: a K slot is free
+            // once the S MMAs that read it finished, a V slot once the PV MMAs
+            // did, so K runs a step further ahead than V needs to.
+            auto slot_free = [&](uint64_t (*empty)[2], int i, int stages) -> bool {
+                const int ip = i - stages;                           // previous load in this slot
+                if (ip < 0) return true;
+                const int users = load_users(ip);
+                const uint32_t ph = (ip / stages) & 1;
+                for (int x = 0; x < NQT; ++x)
+                    if (((users >> x) & 1) && !mbar_test(&empty[ip % stages][x], ph)) return false;
+                return true;
+            };
+            int ik = 0, iv = 0;
+            bool ok = true;
+            uint64_t t_last = global_timer_ns();
+            while ((ik < n_loads || iv < n_loads) && ok) {
+                bool progressed = false;
+                if (ik < n_loads && slot_free(bars->k_empty, ik, STK)) {
+                    const int st = ik % STK;
+                    if (load_users(ik) == 0) {
+                        mbar_arrive(&bars->k_full[st]);              // null load: nothing reads it
+                    } else {
+                        const int j = load_tile(ik);
+                        mbar_arrive_expect_tx(&bars->k_full[st], C::K_BYTES + C::SFQK_BYTES);
+                        tma_load_2d(smem + C::OFF_K + st * C::K_BYTES, &tmK, 0, grp * p.Nkv + j * 128, &bars->k_full[st]);
+                        bulk_load(smem + C::OFF_SFK + st * C::SFQK_BYTES,
+                                  p.ks + ((size_t)grp * T + j) * C::SFQK_BYTES, C::SFQK_BYTES, &bars->k_full[st]);
+                    }
+                    HIFA4_TRACE_POINT(4, ik, 1);
+                    ++ik;
+                    progressed = true;
                 }
-                if (!ok) break;
-                if (load_users(i) == 0) {
-                    // a null load (past the end of a shorter range): nothing reads it
-                    mbar_arrive(&bars->k_full[st]);
-                    mbar_arrive(&bars->v_full[st]);
+                if (iv < n_loads && slot_free(bars->v_empty, iv, STV)) {
+                    const int st = iv % STV;
+                    if (load_users(iv) == 0) {
+                        mbar_arrive(&bars->v_full[st]);
+                    } else {
+                        const int j = load_tile(iv);
+                        mbar_arrive_expect_tx(&bars->v_full[st], C::V_TMA_BYTES + C::SFV_BYTES);
+                        tma_load_2d(smem + C::OFF_V + st * C::V_STRIDE, &tmV, 0, (grp * T + j) * D, &bars->v_full[st]);
+                        bulk_load(smem + C::OFF_SFV + st * C::SFV_BYTES,
+                                  p.vts + ((size_t)grp * T + j) * C::SFV_BYTES, C::SFV_BYTES, &bars->v_full[st]);
+                    }
+                    ++iv;
+                    progressed = true;
+                }
+                if (progressed) {
+                    t_last = global_timer_ns();
                 } else {
-                    const int j = load_tile(i);
-                    mbar_arrive_expect_tx(&bars->k_full[st], C::K_BYTES + C::SFQK_BYTES);
-                    tma_load_2d(smem + C::OFF_K + st * C::K_BYTES, &tmK, 0, grp * p.Nkv + j * 128, &bars->k_full[st]);
-                    bulk_load(smem + C::OFF_SFK + st * C::SFQK_BYTES,
-                              p.ks + ((size_t)grp * T + j) * C::SFQK_BYTES, C::SFQK_BYTES, &bars->k_full[st]);
-                    mbar_arrive_expect_tx(&bars->v_full[st], C::V_TMA_BYTES + C::SFV_BYTES);
-                    tma_load_2d(smem + C::OFF_V + st * C::V_STRIDE, &tmV, j * 64, grp * D, &bars->v_full[st]);
-                    bulk_load(smem + C::OFF_SFV + st * C::SFV_BYTES,
-                              p.vts + ((size_t)grp * T + j) * C::SFV_BYTES, C::SFV_BYTES, &bars->v_full[st]);
+                    __nanosleep(128);
+                    if (*abort_flag) {
+                        ok = false;
+                    } else if (global_timer_ns() - t_last > p.wait_limit_ns) {
+                        *abort_flag = 1;
+                        atomicExch(p.status, kStatusTimeout);
+                        ok = false;
+                    }
                 }
-                issued = i + 1;
             }
             if (!ok) {
                 // drain the copies still in flight before the CTA exits
-                for (int i = max(0, issued - ST); i < issued; ++i) {
-                    mbar_wait_drain(&bars->k_full[i % ST], (i / ST) & 1, p.wait_limit_ns);
-                    mbar_wait_drain(&bars->v_full[i % ST], (i / ST) & 1, p.wait_limit_ns);
-                }
+                for (int i = max(0, ik - STK); i < ik; ++i)
+                    mbar_wait_drain(&bars->k_full[i % STK], (i / STK) & 1, p.wait_limit_ns);
+                for (int i = max(0, iv - STV); i < iv; ++i)
+                    mbar_wait_drain(&bars->v_full[i % STV], (i / STV) & 1, p.wait_limit_ns);
                 mbar_wait_drain(&bars->q_full, 0, p.wait_limit_ns);
             }
         }
@@ -494,8 +540,8 @@ __global__ void __launch_bounds__(Cfg<D, PREORDER, DEC>::THREADS, 1)
         // the loads the first step reads (plain: load 0; decode: loads 0..3)
         for (int i = 0; i < (DEC ? 4 : 1) && ok && more; ++i) {
             if (load_users(i) == 0) continue;
-            ok = __all_sync(0xFFFFFFFFu, mbar_wait(&bars->k_full[i % ST], 0, ctl));
-            if (ok) ok = __all_sync(0xFFFFFFFFu, mbar_wait(&bars->v_full[i % ST], 0, ctl));
+            ok = __all_sync(0xFFFFFFFFu, mbar_wait(&bars->k_full[i % STK], 0, ctl));
+            if (ok) ok = __all_sync(0xFFFFFFFFu, mbar_wait(&bars->v_full[i % STV], 0, ctl));
         }
         if constexpr (DEC) {
             if (ok) {
@@ -766,6 +812,7 @@ __global__ void __launch_bounds__(Cfg<D, PREORDER, DEC>::THREADS, 1)
             HIFA4_TRACE_POINT(qt, j, 6);
         }
         // ---------------------------------------------------------- epilogue
+        HIFA4_TRACE_POINT(qt, 62, 0);
         if (ok && nt > 0) ok = __all_sync(0xFFFFFFFFu, mbar_wait(&bars->o_done[qt], (nt - 1) & 1, ctl));
         float l = 0.0f;
         if (ok && nt > 0) {
@@ -870,6 +917,7 @@ __global__ void __launch_bounds__(Cfg<D, PREORDER, DEC>::THREADS, 1)
     __syncthreads();
     tc_fence_after();
     if (warp == 1) tmem_dealloc(tmem, 512);
+    if (threadIdx.x == 0) HIFA4_TRACE_POINT(4, 63, 2);
 }
 
 template <int D, bool PRE, bool CAUSAL, int OUT, bool DUMP, bool DEC>

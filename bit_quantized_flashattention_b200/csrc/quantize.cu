@@ -158,7 +158,8 @@ __device__ __forceinline__ void quantize_rows_cta(const RowJob& jb, unsigned cta
 
 // ---------------------------------------------------------------------- V
 
-// V quantized along tokens, written transposed. A warp covers 32 channels x 64
+// V quantized along tokens, written transposed and tiled (each 128-token tile
+// of V^T is one contiguous D x 64-byte block). A warp covers 32 channels x 64
 // tokens of one group; lane (cc, tb) owns 4 channels (cc = 0..7) x one 16-token
 // block (tb = 0..3): it reads 16 rows of 8 bytes (each load instruction reads 4
 // rows of 64 contiguous bytes), quantizes one block per channel and writes 8
@@ -192,7 +193,9 @@ __device__ __forceinline__ void quantize_v_warp(const VJob& jb, unsigned gw_all,
         uint32_t lo, hi;
         const uint32_t sf = quant_block16_lut(x, lut, lo, hi);
         const unsigned d = d0 + k;
-        *reinterpret_cast<uint2*>(jb.vtc + ((size_t)grp * D + d) * (nkv / 2) + tok0 / 2) = make_uint2(lo, hi);
+        // tiled V^T codes: the 64 bytes of channel d for kv tile tok0/128
+        *reinterpret_cast<uint2*>(jb.vtc + (((size_t)grp * (nkv / 128) + tok0 / 128) * D + d) * 64 + (tok0 % 128) / 2) =
+            make_uint2(lo, hi);
         uint32_t word = sf << (8u * tb);
         word |= __shfl_xor_sync(0xFFFFFFFFu, word, 1);
         word |= __shfl_xor_sync(0xFFFFFFFFu, word, 2);

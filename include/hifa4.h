@@ -74,7 +74,9 @@ enum { HIFA4_CAUSAL = 1u << 0, HIFA4_SPLIT_KV = 1u << 1 };
  * per byte, element 2i in the low nibble; scales are E4M3 bytes):
  *   qc  [B, Hq, Nq, D/2]         Q codes, row-major
  *   kc  [B, Hkv, Nkv, D/2]       K codes, row-major
- *   vtc [B, Hkv, D, Nkv/2]       V codes, transposed (tokens contiguous)
+ *   vtc [B, Hkv, Nkv/128, D, 64] V codes, transposed and tiled: each 128-token
+ *                                tile of V^T is one contiguous block, channel d's
+ *                                64 bytes (tokens 128j..128j+127) at row d
  *   qs, ks, vts                  scales in the MMA-ready layout below
  * MMA-ready scale layout: 512-byte atoms, each holding the scales of 128 rows x
  * 64 contraction elements (4 scales per row); row r, scale k (0..3) of an atom
@@ -88,7 +90,9 @@ enum { HIFA4_CAUSAL = 1u << 0, HIFA4_SPLIT_KV = 1u << 1 };
  *       When D = 64 the padding row 64 holds 0x38 (1.0): the scale of the
  *       normalizer column used by P-Reordering. Other padding rows are 0.
  * The canonical scale tensors Qs [B,Hq,Nq,D/16], Ks [B,Hkv,Nkv,D/16] and
- * Vts [B,Hkv,D,Nkv/16] map one-to-one onto these bytes. */
+ * Vts [B,Hkv,D,Nkv/16], and the canonical V codes Vtc [B,Hkv,D,Nkv/2]
+ * (byte c of a channel row: Vtc[b,g,d,c] = vtc[b,g,c/64,d,c%64]), map one-to-one
+ * onto these bytes. */
 typedef struct {
     void* qc;
     void* qs;

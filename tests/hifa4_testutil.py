@@ -46,6 +46,12 @@ def v_scale_index(B, Hkv, N, D):
     return ((((b * Hkv + g) * NT + j) * NRB + rb) * 2 + s) * 512 + _atom(r) + k
 
 
+def canonical_vtc(vtc_tiled, B, Hkv, Nkv, D) -> np.ndarray:
+    """Tiled V codes [B,Hkv,Nkv/128,D,64] (device or host) -> canonical Vtc [B,Hkv,D,Nkv/2]."""
+    a = vtc_tiled.cpu().numpy() if hasattr(vtc_tiled, "cpu") else np.asarray(vtc_tiled)
+    return np.ascontiguousarray(a.reshape(B, Hkv, Nkv // 128, D, 64).transpose(0, 1, 3, 2, 4).reshape(B, Hkv, D, Nkv // 2))
+
+
 def canonical_scales(packed, B, Hq, Hkv, Nq, Nkv, D):
     """Device packed buffers -> canonical numpy (qs [B,Hq,Nq,D/16], ks, vts)."""
     qs_raw = packed.qs.cpu().numpy()

@@ -80,7 +80,7 @@ def test_config_parity(H, index):
     qs_all, ks_all, vts_all = U.canonical_scales(pk, cfg.B, cfg.Hq, cfg.Hkv, cfg.Nq, cfg.Nkv, cfg.D)
     qc_all = pk.qc.view(cfg.B, cfg.Hq, cfg.Nq, cfg.D // 2)
     kc_all = pk.kc.view(cfg.B, cfg.Hkv, cfg.Nkv, cfg.D // 2)
-    vtc_all = pk.vtc.view(cfg.B, cfg.Hkv, cfg.D, cfg.Nkv // 2)
+    vtc_all = pk.vtc.view(cfg.B, cfg.Hkv, cfg.Nkv // 128, cfg.D, 64)
     G = cfg.G
     n_codes = n_mism = 0
     for (b, g) in _sample_groups(cfg, rng):
@@ -93,7 +93,7 @@ def test_config_parity(H, index):
         assert np.array_equal(qs_all[b, hs], ref_p["qs"][0])
         assert np.array_equal(kc_all[b, g].cpu().numpy(), ref_p["kc"][0, 0])
         assert np.array_equal(ks_all[b, g], ref_p["ks"][0, 0])
-        assert np.array_equal(vtc_all[b, g].cpu().numpy(), ref_p["vtc"][0, 0])
+        assert np.array_equal(U.canonical_vtc(vtc_all[b, g], 1, 1, cfg.Nkv, cfg.D)[0, 0], ref_p["vtc"][0, 0])
         assert np.array_equal(vts_all[b, g], ref_p["vts"][0, 0])
         idx = _sample_rows(cfg, rng)
         rows_local = np.concatenate([hh * cfg.Nq + idx for hh in range(G)])
