@@ -10,11 +10,21 @@ value    attention FLOPs (4*B*Hq*Nq*Nkv*D/2 for causal) per second over the
          whole step, inputs resident in HBM, L2 flushed between steps
 e2e      the same metric through the public API with host buffers: pinned
          host->device copy of Q, K, V, the step, device->host copy of O, LSE
-roofline the attention kernel alone against the FP4 dense tensor peak
-cpu_baseline  the CPU oracle on a bounded sample of the same workload
+roofline the attention kernel alone against its bound: the FP4 dense tensor
+         peak (prefill), or the HBM copy bandwidth (split-kv decode chunks)
+context  torch bf16 SDPA on the same inputs and GPU; error of the 4-bit
+         output against unquantized fp32 attention (torch fp32 SDPA) on
+         sampled groups; a measured NVFP4 GEMM peak (torch scaled_mm)
+cpu_baseline  the CPU oracle on a bounded sample of the same workload, on all
+         host cores and on one core
 
 ``--impl reference`` times the CPU oracle (the slow, plainly written CPU
 implementation of the same computation) on the host cores instead.
+``--all-configs`` times every workload (both normalizer modes where the
+workload names two) and prints one JSON line each; ``--table PATH`` also
+writes them as a markdown table. ``--ingest-ncu CSV --workload NAME`` records
+the DRAM bytes per attention launch from an ncu CSV capture (with the
+kernel-source hash it belongs to) in profiles/attn_traffic.json.
 Multi-GPU (torchrun): every rank runs its own replica of the workload (the
 path has no exchange step); value sums the ranks' work over the max time.
 """
@@ -81,26 +91,53 @@ def attention_source_hash() -> str:
     return h.hexdigest()
 
 
+TRAFFIC_JSON = os.path.join(ROOT, "profiles", "attn_traffic.json")
+
+
 def profiled_traffic(cfg):
-    """DRAM bytes per attention launch from the committed ncu summary of this workload, or None
-    when there is none or the kernel sources changed since it was captured."""
-    path = os.path.join(ROOT, "profiles", f"attn_fwd_kernel_{cfg.name}.md")
+    """DRAM bytes per attention launch of this workload as recorded from an ncu
+    capture by --ingest-ncu, or None when there is none or the kernel sources
+    changed since it was captured."""
     try:
-        with open(path) as f:
-            text = f.read()
-    except OSError:
+        with open(TRAFFIC_JSON) as f:
+            rec = json.load(f).get(cfg.name)
+    except (OSError, ValueError):
         return None
-    vals = {}
-    for ln in text.splitlines():
-        for key in ("source sha256:", "traffic bytes per launch:"):
-            if ln.strip().startswith(key):
-                vals[key] = ln.split(":", 1)[1].strip().strip("`")
-    if vals.get("source sha256:") != attention_source_hash():
+    if not rec or rec.get("source_sha256") != attention_source_hash():
         return None
+    return rec.get("dram_bytes_per_launch")
+
+
+def ingest_ncu(csv_path, workload, command):
+    """Sum dram__bytes_read/write of the attention kernel's captured launches in an
+    ncu CSV (``ncu --csv --metrics dram__bytes_read.sum,dram__bytes_write.sum ...``)
+    and record the per-launch mean, with the kernel-source hash, in the JSON."""
+    import csv
+    per_launch = {}
+    with open(csv_path) as f:
+        lines = [ln for ln in f if ln.startswith('"')]
+    for row in csv.DictReader(lines):
+        if "attn_fwd_kernel" not in row.get("Kernel Name", ""):
+            continue
+        name, unit, val = row["Metric Name"], row.get("Metric Unit", ""), row["Metric Value"].replace(",", "")
+        scale = {"byte": 1, "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9}.get(unit, 1)
+        if name in ("dram__bytes_read.sum", "dram__bytes_write.sum"):
+            per_launch.setdefault(row["ID"], 0.0)
+            per_launch[row["ID"]] += float(val) * scale
+    if not per_launch:
+        raise SystemExit(f"no attn_fwd_kernel DRAM counters in {csv_path}")
+    rec = {}
     try:
-        return int(vals["traffic bytes per launch:"])
-    except (KeyError, ValueError):
-        return None
+        with open(TRAFFIC_JSON) as f:
+            rec = json.load(f)
+    except (OSError, ValueError):
+        pass
+    rec[workload] = {"dram_bytes_per_launch": int(round(statistics.mean(per_launch.values()))),
+                     "launches": len(per_launch), "source_sha256": attention_source_hash(), "command": command}
+    os.makedirs(os.path.dirname(TRAFFIC_JSON), exist_ok=True)
+    with open(TRAFFIC_JSON, "w") as f:
+        json.dump(rec, f, indent=1, sort_keys=True)
+    print(json.dumps({workload: rec[workload]}))
 
 
 def max_over_ranks(x: float, device) -> float:
@@ -128,12 +165,13 @@ class Clocks:
     def __init__(self, index: int):
         self.index = index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_gpu{index}.csv")
+        self.path = None
 
     def __enter__(self):
         try:
-            os.makedirs(os.path.dirname(self.path), exist_ok=True)
-            self.f = open(self.path, "w")
+            import tempfile
+            fd, self.path = tempfile.mkstemp(prefix=f"hifa4_clocks{self.index}_", suffix=".csv")
+            self.f = os.fdopen(fd, "w")
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.index),
                  "--query-gpu=index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -157,7 +195,9 @@ class Clocks:
 
     def summary(self):
         try:
-            rows = [r.split(",") for r in open(self.path).read().strip().splitlines()]
+            with open(self.path) as f:
+                rows = [r.split(",") for r in f.read().strip().splitlines()]
+            os.unlink(self.path)
             rows = [[c.strip() for c in r] for r in rows if len(r) >= 9]
         except Exception:
             return None
@@ -206,10 +246,11 @@ def make_inputs(cfg, device, rank=0):
 
 # -------------------------------------------------------------- CPU oracle
 
-def oracle_sample(cfg, seconds_target=12.0, n_threads=0, rows_per_head=None):
+def oracle_sample(cfg, seconds_target=12.0, n_threads=0, rows_per_head=None, n_splits=1):
     """Time the CPU oracle on a bounded sample of the workload: one kv group's
-    quantization plus the attention of a strided subset of its query rows.
-    Returns (flops_of_sample / seconds, description, threads)."""
+    quantization plus the attention of a strided subset of its query rows
+    (n_threads = 0: all host cores). Returns (flops_of_sample / seconds,
+    description, seconds)."""
     import oracle
     gains = W.k_gains(cfg)
     b, g = 0, 0
@@ -231,7 +272,7 @@ def oracle_sample(cfg, seconds_target=12.0, n_threads=0, rows_per_head=None):
     rows = np.concatenate([hh * cfg.Nq + idx for hh in range(G)])
     t0 = time.perf_counter()
     pk = oracle.quantize_qkv(q, k, v, s, si)
-    oracle.attention_rows(shape, rows, packed=pk, causal=cfg.causal, n_threads=n_threads)
+    oracle.attention_rows(shape, rows, packed=pk, causal=cfg.causal, n_threads=n_threads, n_splits=n_splits)
     dt = time.perf_counter() - t0
     if cfg.causal:
         keys = np.minimum(idx + cfg.Nkv - cfg.Nq + 1, cfg.Nkv)
@@ -241,7 +282,7 @@ def oracle_sample(cfg, seconds_target=12.0, n_threads=0, rows_per_head=None):
     # grow the sample to the target CPU time
     if dt < seconds_target / 4 and n_rows < cfg.Nq:
         scale = min(cfg.Nq / n_rows, max(2.0, seconds_target / max(dt, 1e-3)))
-        return oracle_sample(cfg, seconds_target, n_threads, int(min(cfg.Nq, n_rows * scale)))
+        return oracle_sample(cfg, seconds_target, n_threads, int(min(cfg.Nq, n_rows * scale)), n_splits)
     desc = (f"quantize one (b, kv head) group (Q {G}x{cfg.Nq}x{cfg.D}, K/V {cfg.Nkv}x{cfg.D}) + attention of "
             f"{rows.size} query rows ({n_rows} per head, evenly spaced) of that group")
     return flops / dt, desc, dt
@@ -249,22 +290,100 @@ def oracle_sample(cfg, seconds_target=12.0, n_threads=0, rows_per_head=None):
 
 # ----------------------------------------------------------------- our arm
 
-def run_ours(args):
+def attn_bytes(cfg, H):
+    """Algorithmic HBM bytes of one attention launch: the packed operands read
+    once, O (bf16) and LSE written."""
+    packed = sum(H.packed_bytes(cfg.B, cfg.Hq, cfg.Hkv, cfg.Nq, cfg.Nkv, cfg.D))
+    return packed + cfg.B * cfg.Hq * cfg.Nq * (cfg.D * 2 + 4)
+
+
+def fp4_gemm_peak(device):
+    """Dense block-scaled FP4 (NVFP4: E2M1, E4M3 per 16) GEMM throughput of this
+    GPU, 8192^3 through torch's scaled_mm (cuBLASLt), best of 10; None when this
+    torch cannot run it."""
+    import torch
+    import torch.nn.functional as F
+    try:
+        from torch.nn.functional import ScalingType, SwizzleType
+        M = N = K = 8192
+        a = torch.randint(0, 256, (M, K // 2), dtype=torch.uint8, device=device).view(torch.float4_e2m1fn_x2)
+        b = torch.randint(0, 256, (N, K // 2), dtype=torch.uint8, device=device).view(torch.float4_e2m1fn_x2)
+        sa = torch.full((M * (K // 16),), 1.0, device=device).to(torch.float8_e4m3fn)
+        sb = torch.full((N * (K // 16),), 1.0, device=device).to(torch.float8_e4m3fn)
+
+        def f():
+            return F.scaled_mm(a, b.t(), sa, ScalingType.BlockWise1x16, sb, ScalingType.BlockWise1x16,
+                               swizzle_a=SwizzleType.SWIZZLE_32_4_4, swizzle_b=SwizzleType.SWIZZLE_32_4_4,
+                               output_dtype=torch.bfloat16)
+        for _ in range(3):
+            f()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(10):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            f()
+            e1.record()
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        return 2.0 * M * N * K / (min(ts) * 1e-3) / 1e12
+    except Exception:
+        return None
+
+
+def sdpa_context(q, k, v, cfg, flush):
+    """torch bf16 scaled_dot_product_attention on the same inputs (same FLOP formula)."""
+    import torch
+    import torch.nn.functional as F
+    ts = []
+    for i in range(8):
+        flush(i)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        F.scaled_dot_product_attention(q, k, v, is_causal=cfg.causal, enable_gqa=True)
+        e1.record()
+        torch.cuda.synchronize()
+        if i >= 3:
+            ts.append(e0.elapsed_time(e1))
+    return round(cfg.flops() / (statistics.mean(ts) * 1e-3) / 1e12, 2)
+
+
+def error_vs_fp32(H, packed, q, k, v, cfg, norm, split_kv, max_groups=2):
+    """Error of the 4-bit output (fp32) against unquantized fp32 softmax attention
+    of the same bf16 inputs (torch fp32 SDPA), on up to max_groups (b, kv head)
+    groups: max abs error and max / median per-row relative L2. Context only."""
+    import torch
+    import torch.nn.functional as F
+    o4, _ = H.attention_fwd(packed, causal=cfg.causal, norm=norm, out_dtype=torch.float32, split_kv=split_kv)
+    G = cfg.G
+    errs, rels = [], []
+    groups = [(0, 0), (cfg.B - 1, cfg.Hkv - 1)][:max_groups]
+    for b, g in sorted(set(groups)):
+        hs = slice(g * G, (g + 1) * G)
+        qq = q[b:b + 1, hs].float()
+        kk = k[b:b + 1, g:g + 1].float().expand(1, G, cfg.Nkv, cfg.D)
+        vv = v[b:b + 1, g:g + 1].float().expand(1, G, cfg.Nkv, cfg.D)
+        ref = F.scaled_dot_product_attention(qq, kk, vv, is_causal=cfg.causal)
+        d = (o4[b:b + 1, hs] - ref).double()
+        errs.append(float(d.abs().max()))
+        rels.append((d.norm(dim=-1) / ref.double().norm(dim=-1).clamp_min(1e-30)).flatten())
+    rel = torch.cat(rels)
+    return {"max_abs": round(max(errs), 6), "row_rel_l2_max": round(float(rel.max()), 6),
+            "row_rel_l2_median": round(float(rel.median()), 6), "groups": len(rels),
+            "reference": "torch fp32 SDPA on the bf16 inputs (unquantized)"}
+
+
+def measure(cfg, norm, args, dev, rank, ws, H, want_e2e=True):
+    """Time one workload: the step (quantize + attention, one CUDA graph) with a
+    cold L2, the two kernels separately, and (want_e2e) the end-to-end loop."""
     import torch
     import torch.distributed as dist
-
-    import bit_quantized_flashattention_b200 as H
-    ws, rank, local = dist_env()
-    if ws > 1:
-        dist.init_process_group("nccl", init_method="env://", timeout=__import__("datetime").timedelta(seconds=120))
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    cfg = W.get(args.config)
-    norm = args.norm
     q, k, v, cal = make_inputs(cfg, dev, rank)
     s = s_inv = None
     if cal is not None:
         s, s_inv = H.calibrate_smooth(cal[0], cal[1], cfg.alpha)
+    split_kv = True               # decode-style chunks take the split-kv mode (one pass otherwise)
+    n_splits = H.attention_splits(cfg.B, cfg.Hq, cfg.Hkv, cfg.Nq, cfg.Nkv, cfg.D, causal=cfg.causal, split_kv=True)
     packed = H.alloc_packed(cfg.B, cfg.Hq, cfg.Hkv, cfg.Nq, cfg.Nkv, cfg.D, dev)
     o = torch.empty(cfg.B, cfg.Hq, cfg.Nq, cfg.D, dtype=torch.bfloat16, device=dev)
     lse = torch.empty(cfg.B, cfg.Hq, cfg.Nq, dtype=torch.float32, device=dev)
@@ -274,9 +393,8 @@ def run_ours(args):
 
     def step():
         H.quantize_qkv(q, k, v, s, s_inv, out=packed)
-        H.attention_fwd(packed, causal=cfg.causal, norm=norm, out=o, lse=lse, workspace=wsp, split_kv=True)
+        H.attention_fwd(packed, causal=cfg.causal, norm=norm, out=o, lse=lse, workspace=wsp, split_kv=split_kv)
 
-    launches_per_step = 2          # quantize_qkv_kernel (Q, K and V), attn_fwd_kernel
     for _ in range(max(args.warmup, 3)):
         step()
     torch.cuda.synchronize()
@@ -295,7 +413,7 @@ def run_ours(args):
     with torch.cuda.graph(g_quant):
         H.quantize_qkv(q, k, v, s, s_inv, out=packed)
     with torch.cuda.graph(g_attn):
-        H.attention_fwd(packed, causal=cfg.causal, norm=norm, out=o, lse=lse, workspace=wsp, split_kv=True)
+        H.attention_fwd(packed, causal=cfg.causal, norm=norm, out=o, lse=lse, workspace=wsp, split_kv=split_kv)
     for g in (g_step, g_quant, g_attn):
         g.replay()
     torch.cuda.synchronize()
@@ -305,7 +423,7 @@ def run_ours(args):
     if ws > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    with Clocks(local) as clk:
+    with Clocks(torch.cuda.current_device()) as clk:
         for i in range(n):
             flush(i)
             ev[i][0].record(stream)
@@ -332,13 +450,12 @@ def run_ours(args):
     st = max_over_ranks(H.get_status(wsp), dev)
     if st != 0:
         raise RuntimeError(f"kernel status {int(st)} in the timed region (max over ranks)")
-
-    flops = cfg.flops()
-    value = ws * flops * n / (total_ms * 1e-3) / 1e12
-    attn_mean = statistics.mean(attn_ms)
-    attn_tflops = flops / (attn_mean * 1e-3) / 1e12
-    pk = peaks()
-    fp4_peak = 4.0 * pk["bf16"]                       # burst: the kernel is timed alone, per launch
+    res = dict(q=q, k=k, v=v, s=s, s_inv=s_inv, packed=packed, o=o, lse=lse, wsp=wsp, flush=flush,
+               total_ms=total_ms, attn_ms=statistics.mean(attn_ms), quant_ms=statistics.mean(quant_ms),
+               clocks=clk.summary(), n_splits=n_splits, split_kv=split_kv)
+    del g_step, g_quant, g_attn
+    if not want_e2e:
+        return res
 
     # End to end through the public API: every step copies its inputs from
     # pinned host memory and reads its results (O and the LSE) back to pinned
@@ -373,7 +490,7 @@ def run_ours(args):
                 s_cp.wait_event(ev_out[b])         # step i-2's results have left this output buffer
             H.quantize_qkv(dq[b], dk[b], dv[b], s, s_inv, out=dpk[b], stream=s_cp)
             H.attention_fwd(dpk[b], causal=cfg.causal, norm=norm, out=do[b], lse=dl[b], workspace=dws[b],
-                            stream=s_cp, split_kv=True)
+                            stream=s_cp, split_kv=split_kv)
             ev_cp[b].record(s_cp)
         with torch.cuda.stream(s_out):
             s_out.wait_event(ev_cp[b])
@@ -396,10 +513,58 @@ def run_ours(args):
     st = max_over_ranks(max(H.get_status(w_) for w_ in dws), dev)
     if st != 0:
         raise RuntimeError(f"kernel status {int(st)} in the end-to-end loop (max over ranks)")
-    e2e_total = max_over_ranks(t_beg.elapsed_time(t_end), dev)
-    h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv))
-    d2h = ho[0].numel() * ho[0].element_size() + hl[0].numel() * hl[0].element_size()
+    res["e2e_ms"] = max_over_ranks(t_beg.elapsed_time(t_end), dev)
+    res["h2d"] = sum(x.numel() * x.element_size() for x in (hq, hk, hv))
+    res["d2h"] = ho[0].numel() * ho[0].element_size() + hl[0].numel() * hl[0].element_size()
+    return res
 
+
+def roofline(cfg, H, attn_ms, fp4_peak, hbm_peak):
+    """The attention kernel against the bound of its workload: tensor (FLOPs over
+    the FP4 peak) or HBM (algorithmic bytes over the copy bandwidth), whichever
+    takes longer at peak."""
+    flops = cfg.flops()
+    nbytes = attn_bytes(cfg, H)
+    t_tensor = flops / (fp4_peak * 1e12)
+    t_hbm = nbytes / (hbm_peak * 1e9)
+    if t_hbm > t_tensor:
+        achieved = nbytes / (attn_ms * 1e-3) / 1e9
+        return {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
+                "frac": round(achieved / hbm_peak, 4), "algorithmic_bytes": nbytes}
+    achieved = flops / (attn_ms * 1e-3) / 1e12
+    return {"bound": "tensor", "achieved": round(achieved, 2), "peak": round(fp4_peak, 1), "unit": "TFLOP/s",
+            "frac": round(achieved / fp4_peak, 4), "algorithmic_flops": flops}
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    import bit_quantized_flashattention_b200 as H
+    ws, rank, local = dist_env()
+    if ws > 1:
+        dist.init_process_group("nccl", init_method="env://", timeout=__import__("datetime").timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pk = peaks()
+    fp4_peak = 4.0 * pk["bf16"]                       # burst: the kernel is timed alone, per launch
+    if args.all_configs:
+        run_all_configs(args, dev, rank, ws, H, pk, fp4_peak)
+        if ws > 1:
+            dist.destroy_process_group()
+        return
+    cfg = W.get(args.config)
+    norm = args.norm
+    r = measure(cfg, norm, args, dev, rank, ws, H)
+    n = args.steps
+    flops = cfg.flops()
+    value = ws * flops * n / (r["total_ms"] * 1e-3) / 1e12
+    attn_tflops = flops / (r["attn_ms"] * 1e-3) / 1e12
+    launches_per_step = 2          # quantize_qkv_kernel (Q, K and V), attn_fwd_kernel
+    roof = roofline(cfg, H, r["attn_ms"], fp4_peak, pk["hbm"])
+    roof.update({"traffic": profiled_traffic(cfg), "kernel": "attn_fwd_kernel",
+                 "peak_source": (f"4 x {pk['src']} bf16 burst" if roof["bound"] == "tensor"
+                                 else f"{pk['src']} HBM copy bandwidth")})
     line = {
         "metric": METRIC,
         "value": round(value, 3),
@@ -407,7 +572,7 @@ def run_ours(args):
         "n_gpus": ws,
         "steps": n,
         "warmup": args.warmup,
-        "ms_per_step": round(total_ms / n, 5),
+        "ms_per_step": round(r["total_ms"] / n, 5),
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
@@ -415,32 +580,39 @@ def run_ours(args):
         "data": "synthetic (seeded normal Q/K/V, lognormal K channel gains + outlier channels)",
         "config": {"workload": cfg.name, "B": cfg.B, "Hq": cfg.Hq, "Hkv": cfg.Hkv, "Nq": cfg.Nq, "Nkv": cfg.Nkv,
                    "D": cfg.D, "causal": cfg.causal, "norm": norm, "smooth_qk": cfg.smooth != "off",
+                   "kv_splits": r["n_splits"],
                    "inputs": cfg.dtype, "output": "bf16", "parallelism": f"replicas{ws}" if ws > 1 else "single",
                    "l2": "cold and clean between steps (256 MiB write, then 256 MiB read)",
                    "step": "quantize_qkv + attention_fwd (calibration offline)",
                    "launch": "the step replayed from a CUDA graph (programmatic dependent launch between its two kernels)"},
         "fp4_tensor_pct": round(100.0 * value / ws / fp4_peak, 2),
-        "breakdown_ms": {"quantize": round(statistics.mean(quant_ms), 5), "attention": round(attn_mean, 5)},
+        "breakdown_ms": {"quantize": round(r["quant_ms"], 5), "attention": round(r["attn_ms"], 5)},
         "attention_only_tflops": round(attn_tflops, 2),
-        "roofline": {"bound": "tensor", "achieved": round(attn_tflops, 2), "peak": round(fp4_peak, 1),
-                     "unit": "TFLOP/s", "frac": round(attn_tflops / fp4_peak, 4), "traffic": profiled_traffic(cfg),
-                     "kernel": "attn_fwd_kernel", "peak_source": f"4 x {pk['src']} bf16 burst"},
-        "e2e": {"value": round(ws * flops * n / (e2e_total * 1e-3) / 1e12, 3), "unit": "TFLOPS",
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_total / n, 4),
+        "roofline": roof,
+        "e2e": {"value": round(ws * flops * n / (r["e2e_ms"] * 1e-3) / 1e12, 3), "unit": "TFLOPS",
+                "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"],
+                "ms_per_step": round(r["e2e_ms"] / n, 4),
                 "pipeline": "H2D, compute and D2H of consecutive steps overlap (3 streams, 2 buffers)"},
         "gpu_launches": launches_per_step * n,
-        "clocks": clk.summary(),
+        "clocks": r["clocks"],
     }
     # the HBM-bound quantize pass: algorithmic bytes (read 2 B/elem, write 0.5625 B/elem)
     elems = cfg.B * cfg.Hq * cfg.Nq * cfg.D + 2 * cfg.B * cfg.Hkv * cfg.Nkv * cfg.D
-    qbytes = elems * (2 + 0.5625)
-    line["quantize_gbs"] = round(qbytes / (statistics.mean(quant_ms) * 1e-3) / 1e9, 1)
-    if args.sdpa and rank == 0:
-        line["sdpa_bf16_tflops"] = sdpa_context(q, k, v, cfg, flush)
+    line["quantize_gbs"] = round(elems * (2 + 0.5625) / (r["quant_ms"] * 1e-3) / 1e9, 1)
+    if rank == 0 and not args.no_extras:
+        line["sdpa_bf16_tflops"] = sdpa_context(r["q"], r["k"], r["v"], cfg, r["flush"])
+        line["error_vs_fp32"] = error_vs_fp32(H, r["packed"], r["q"], r["k"], r["v"], cfg, norm, r["split_kv"])
+        g = fp4_gemm_peak(dev)
+        if g is not None:
+            line["fp4_gemm_tflops_measured"] = round(g, 1)
+            line["attention_frac_of_measured_fp4_gemm"] = round(attn_tflops / g, 4)
     if rank == 0 and not args.no_cpu:
-        v_cpu, desc, secs = oracle_sample(cfg)
+        v_cpu, desc, secs = oracle_sample(cfg, n_splits=r["n_splits"])
         line["cpu_baseline"] = {"value": round(v_cpu / 1e12, 8), "unit": "TFLOPS", "cores": os.cpu_count(),
                                 "kind": "oracle", "sample": desc, "seconds": round(secs, 2)}
+        v1, desc1, secs1 = oracle_sample(cfg, seconds_target=4.0, n_threads=1, n_splits=r["n_splits"])
+        line["cpu_baseline_1core"] = {"value": round(v1 / 1e12, 9), "unit": "TFLOPS", "cores": 1, "kind": "oracle",
+                                      "sample": desc1, "seconds": round(secs1, 2)}
     if ws > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -448,20 +620,43 @@ def run_ours(args):
         print(json.dumps(line), flush=True)
 
 
-def sdpa_context(q, k, v, cfg, flush):
+def run_all_configs(args, dev, rank, ws, H, pk, fp4_peak):
+    """Every workload, in the launch configuration of the main line; one JSON
+    line per (workload, normalizer mode)."""
     import torch
-    import torch.nn.functional as F
-    ts = []
-    for i in range(8):
-        flush(i)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        F.scaled_dot_product_attention(q, k, v, is_causal=cfg.causal, enable_gqa=True)
-        e1.record()
-        torch.cuda.synchronize()
-        if i >= 3:
-            ts.append(e0.elapsed_time(e1))
-    return round(cfg.flops() / (statistics.mean(ts) * 1e-3) / 1e12, 2)
+    rows = []
+    for cfg in W.CONFIGS:
+        for norm in cfg.modes:
+            r = measure(cfg, norm, args, dev, rank, ws, H, want_e2e=False)
+            roof = roofline(cfg, H, r["attn_ms"], fp4_peak, pk["hbm"])
+            rec = {"workload": cfg.name, "norm": norm, "kv_splits": r["n_splits"],
+                   "step_ms": round(r["total_ms"] / args.steps, 5),
+                   "step_tflops": round(cfg.flops() / (r["total_ms"] / args.steps * 1e-3) / 1e12, 2),
+                   "attention_ms": round(r["attn_ms"], 5),
+                   "attention_tflops": round(cfg.flops() / (r["attn_ms"] * 1e-3) / 1e12, 2),
+                   "quantize_ms": round(r["quant_ms"], 5), "roofline": roof, "clocks": r["clocks"]}
+            if rank == 0 and not args.no_extras:
+                rec["sdpa_bf16_tflops"] = sdpa_context(r["q"], r["k"], r["v"], cfg, r["flush"])
+                rec["error_vs_fp32"] = error_vs_fp32(H, r["packed"], r["q"], r["k"], r["v"], cfg, norm, r["split_kv"])
+            if rank == 0:
+                print(json.dumps(rec), flush=True)
+            rows.append(rec)
+            del r
+            torch.cuda.empty_cache()
+    if rank == 0 and args.table:
+        with open(args.table, "w") as f:
+            f.write("| workload | norm | kv ranges | step ms | step TFLOP/s | attention ms | attention TFLOP/s | "
+                    "bound | roofline frac | quantize ms | bf16 SDPA TFLOP/s | max abs err vs fp32 | "
+                    "row rel L2 (median / max) | SM MHz |\n")
+            f.write("|" + "---|" * 14 + "\n")
+            for x in rows:
+                e = x.get("error_vs_fp32", {})
+                f.write(f"| {x['workload']} | {x['norm']} | {x['kv_splits']} | {x['step_ms']:.4f} | "
+                        f"{x['step_tflops']:.1f} | {x['attention_ms']:.4f} | {x['attention_tflops']:.1f} | "
+                        f"{x['roofline']['bound']} | {x['roofline']['frac']:.3f} | {x['quantize_ms']:.4f} | "
+                        f"{x.get('sdpa_bf16_tflops', '')} | {e.get('max_abs', '')} | "
+                        f"{e.get('row_rel_l2_median', '')} / {e.get('row_rel_l2_max', '')} | "
+                        f"{(x['clocks'] or {}).get('sm_mhz', '')} |\n")
 
 
 # ----------------------------------------------------------- reference arm
@@ -504,10 +699,17 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", type=int, default=2, help="workload index 1..5 (2 = the headline)")
     ap.add_argument("--norm", choices=["p_reorder", "high_precision_l"], default="p_reorder")
-    ap.add_argument("--sdpa", action="store_true", help="also time torch bf16 SDPA as context")
-    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle sample")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle samples")
+    ap.add_argument("--no-extras", action="store_true", help="skip SDPA, fp32-error and FP4-GEMM context")
+    ap.add_argument("--all-configs", action="store_true", help="time every workload (one JSON line each)")
+    ap.add_argument("--table", help="with --all-configs: also write a markdown table here")
+    ap.add_argument("--ingest-ncu", help="record DRAM bytes per attention launch from this ncu CSV")
+    ap.add_argument("--workload", help="with --ingest-ncu: the workload name the capture ran")
+    ap.add_argument("--ncu-command", default="", help="with --ingest-ncu: the command that made the capture")
     args = ap.parse_args()
-    if args.impl == "reference":
+    if args.ingest_ncu:
+        ingest_ncu(args.ingest_ncu, args.workload or W.get(args.config).name, args.ncu_command)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_ours(args)
