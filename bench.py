@@ -554,6 +554,8 @@ def run_ours(args):
             dist.destroy_process_group()
         return
     cfg = W.get(args.config)
+    if args.batch:
+        cfg = cfg.replace(B=args.batch)      # smaller case of the same workload (profiling captures)
     norm = args.norm
     r = measure(cfg, norm, args, dev, rank, ws, H)
     n = args.steps
@@ -699,6 +701,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", type=int, default=2, help="workload index 1..5 (2 = the headline)")
     ap.add_argument("--norm", choices=["p_reorder", "high_precision_l"], default="p_reorder")
+    ap.add_argument("--batch", type=int, default=0, help="override the workload's batch (smaller profiling cases)")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle samples")
     ap.add_argument("--no-extras", action="store_true", help="skip SDPA, fp32-error and FP4-GEMM context")
     ap.add_argument("--all-configs", action="store_true", help="time every workload (one JSON line each)")
