@@ -226,6 +226,80 @@ void ora_quantize_v(const float* v, int B, int Hkv, int N, int D, uint8_t* vtc, 
     }
 }
 
+/* ----------------------------------------- steps before quantization */
+
+/* Rotary position embedding, rotate-half pairing: channel d < D/2 pairs with
+ * channel d + D/2 (the abstract applies Smooth-QK "after RoPE"; RoPE itself
+ * is the standard rotation of the RoFormer paper in this pairing). In place on
+ * x [rows, D], with c = cos_t[pos[row], d] and s = sin_t[pos[row], d]
+ * (tables [*, D/2]):
+ *   x[d]       <- RN(RN(x[d]*c) - RN(x[d+D/2]*s))
+ *   x[d+D/2]   <- RN(RN(x[d+D/2]*c) + RN(x[d]*s))
+ * each product and sum rounded to fp32 (no fused multiply-add). */
+void ora_rope_neox(float* x, long long rows, int D, const float* cos_t, const float* sin_t, const int* pos) {
+    int H2 = D / 2;
+    for (long long r = 0; r < rows; ++r) {
+        float* xr = x + (size_t)r * D;
+        const float* cr = cos_t + (size_t)pos[r] * H2;
+        const float* sr = sin_t + (size_t)pos[r] * H2;
+        for (int d = 0; d < H2; ++d) {
+            float a = xr[d], b = xr[d + H2];
+            float ac = a * cr[d], bs = b * sr[d], bc = b * cr[d], as = a * sr[d];
+            xr[d] = ac - bs;
+            xr[d + H2] = bc + as;
+        }
+    }
+}
+
+/* Smooth-QK multiply in place: x[b,h,i,d] <- RN(x * scale[h/group, d])
+ * (the same product ora_quantize_rows takes when given a scale). */
+void ora_smooth_rows(float* x, int B, int H, int N, int D, int group, const float* scale) {
+    for (long long row = 0; row < (long long)B * H * N; ++row) {
+        int h = (int)((row / N) % H);
+        float* xr = x + (size_t)row * D;
+        for (int d = 0; d < D; ++d) xr[d] = mul_f32(xr[d], scale[(size_t)(h / group) * D + d]);
+    }
+}
+
+/* Q-Mean auxiliary, first half: the per-(batch, head, channel) mean of the
+ * pre-quantization Q over its N tokens, mean[bh, d] = RN_fp32(sum_i x / N),
+ * with the sum accumulated in fp64 and divided in fp64 (x [BH, N, D]). */
+void ora_q_mean(const float* x, long long BH, int N, int D, float* mean) {
+    for (long long bh = 0; bh < BH; ++bh) {
+        for (int d = 0; d < D; ++d) {
+            double sum = 0.0;
+            for (int i = 0; i < N; ++i) sum += (double)x[((size_t)bh * N + i) * D + d];
+            mean[(size_t)bh * D + d] = (float)(sum / (double)N);
+        }
+    }
+}
+
+/* x[bh, i, d] <- RN(x - mean[bh, d]): the residual that is quantized. */
+void ora_sub_mean(float* x, long long BH, int N, int D, const float* mean) {
+    for (long long bh = 0; bh < BH; ++bh)
+        for (int i = 0; i < N; ++i)
+            for (int d = 0; d < D; ++d) x[((size_t)bh * N + i) * D + d] -= mean[(size_t)bh * D + d];
+}
+
+/* Q-Mean auxiliary, second half: the rank-one score term the residual leaves
+ * out, bias[b,h,j] = sum_d mean[b,h,d] * K'[b,g,j,d] (g = h / (Hq/Hkv)), with
+ * K' the keys as they enter quantization (after RoPE and smoothing, before
+ * 4-bit rounding: the term is kept at full precision), accumulated in fp64.
+ * kf [B,Hkv,Nkv,D]; bias [B,Hq,Nkv]. */
+void ora_q_mean_bias(const float* mean, const float* kf, int B, int Hq, int Hkv, int Nkv, int D, double* bias) {
+    int G = Hq / Hkv;
+    for (long long bh = 0; bh < (long long)B * Hq; ++bh) {
+        long long b = bh / Hq;
+        int g = (int)(bh % Hq) / G;
+        for (int j = 0; j < Nkv; ++j) {
+            const float* kr = kf + (((size_t)b * Hkv + g) * (size_t)Nkv + j) * D;
+            double acc = 0.0;
+            for (int d = 0; d < D; ++d) acc += (double)mean[(size_t)bh * D + d] * (double)kr[d];
+            bias[(size_t)bh * Nkv + j] = acc;
+        }
+    }
+}
+
 /* Decode helpers over the canonical packed layouts. */
 static double dec_row(const uint8_t* codes, const uint8_t* sf, int idx) {
     uint8_t byte = codes[idx >> 1];
@@ -260,6 +334,9 @@ void ora_qk_row(const uint8_t* qc, const uint8_t* qs, const uint8_t* kc, const u
 
 /* norm_mode: 0 = P-Reordering (l from P_hat), 1 = high-precision l (from P).
  * n_splits >= 1: kv split count (see the header; 1 = one pass).
+ * s_bias: NULL, or a per-(b, h, key) score term [B,Hq,Nkv] added to the fp64
+ * dot product before its one rounding, S = RN_fp32(Q_hat K_hat^T + s_bias)
+ * (the Q-Mean auxiliary: ora_q_mean_bias; 4-bit path only).
  * quant: 1 = 4-bit path on the packed operands; 0 = the same online softmax
  * on the fp32 operands qf/kf/vf ([B,H,N,D], already smoothed) with P unquantized.
  * rows: flat query-row ids (b*Hq + h)*Nq + i. Outputs are per requested row.
@@ -272,7 +349,7 @@ int ora_attention_rows(const uint8_t* qc, const uint8_t* qs, const uint8_t* kc, 
                        const float* qf, const float* kf, const float* vf,
                        int B, int Hq, int Hkv, int Nq, int Nkv, int D,
                        float sm_scale, int causal, int norm_mode, int quant, int n_splits,
-                       const long long* rows, long long n_rows,
+                       const double* s_bias, const long long* rows, long long n_rows,
                        double* O, double* lse, double* l_hat_out, double* l_hp_out,
                        double* eps_tile, uint8_t* p_codes, uint8_t* p_sf, int n_threads) {
     if (D > 256 || D % 16 || Nkv % TILE_KV || Hq % Hkv || n_splits < 1) return -1;
@@ -328,6 +405,7 @@ int ora_attention_rows(const uint8_t* qc, const uint8_t* qs, const uint8_t* kc, 
                     const uint8_t* kcr = kc + (kvbase + n) * (D / 2);
                     const uint8_t* ksr = ks + (kvbase + n) * (D / 16);
                     for (int d = 0; d < D; ++d) acc += qd[d] * dec_row(kcr, ksr, d);
+                    if (s_bias) acc += s_bias[(size_t)bh * Nkv + n];     /* bh = b*Hq + h */
                 } else {
                     const float* kr = kf + (kvbase + n) * D;
                     for (int d = 0; d < D; ++d) acc += qd[d] * (double)kr[d];

@@ -491,3 +491,194 @@ def test_split_kv_p_hat_is_relative_to_the_split_max():
     assert nib(one["p_codes"][0]) == 0                    # 2^((2 - 60) c) flushes to zero in one pass
     # tiles 0 and 1 (the first split) are the same either way
     assert np.array_equal(one["p_codes"][0][:128], two["p_codes"][0][:128])
+
+
+# ------------------------------------------------ RoPE (steps before the path)
+
+def _rope_tables(n_pos, D, base=10000.0):
+    """cos/sin of pos * base^(-2d/D) in fp64, rounded to fp32 (the caller's tables)."""
+    inv = base ** (-np.arange(0, D // 2, dtype=np.float64) * 2.0 / D)
+    ang = np.arange(n_pos, dtype=np.float64)[:, None] * inv[None, :]
+    return np.cos(ang).astype(np.float32), np.sin(ang).astype(np.float32)
+
+
+def test_rope_identity_and_quarter_turn_are_exact():
+    """cos = 1, sin = 0 leaves x unchanged; cos = 0, sin = 1 is the quarter
+    turn of rotate-half pairing: (x[d], x[d+D/2]) -> (-x[d+D/2], x[d]). A swapped
+    sign or the interleaved (2i, 2i+1) pairing fails the second check."""
+    D = 16
+    rng = np.random.default_rng(40)
+    x = rng.standard_normal((1, 1, 3, D)).astype(np.float32)
+    cos_t = np.stack([np.ones(D // 2), np.zeros(D // 2)]).astype(np.float32)
+    sin_t = np.stack([np.zeros(D // 2), np.ones(D // 2)]).astype(np.float32)
+    same = oracle.rope_neox(x, cos_t, sin_t, [0, 0, 0])
+    assert np.array_equal(same, x)
+    turned = oracle.rope_neox(x, cos_t, sin_t, [1, 0, 1])
+    want = np.concatenate([-x[..., D // 2:], x[..., :D // 2]], axis=-1)
+    assert np.array_equal(turned[:, :, 0], want[:, :, 0]) and np.array_equal(turned[:, :, 2], want[:, :, 2])
+    assert np.array_equal(turned[:, :, 1], x[:, :, 1])
+
+
+def test_rope_preserves_pair_norms_and_depends_on_relative_position():
+    """A rotation keeps |(x[d], x[d+D/2])|, and the score between a query at
+    position m and a key at n depends only on m - n."""
+    D = 64
+    cos_t, sin_t = _rope_tables(64, D)
+    rng = np.random.default_rng(41)
+    q = rng.standard_normal((1, 1, 1, D)).astype(np.float32)
+    k = rng.standard_normal((1, 1, 1, D)).astype(np.float32)
+    y = oracle.rope_neox(q, cos_t, sin_t, [37]).astype(np.float64)
+    n_in = np.hypot(q[..., :D // 2], q[..., D // 2:])
+    n_out = np.hypot(y[..., :D // 2], y[..., D // 2:])
+    assert np.abs(n_out / n_in - 1).max() <= 1e-6
+    s = [float(np.sum(oracle.rope_neox(q, cos_t, sin_t, [m]).astype(np.float64)
+                      * oracle.rope_neox(k, cos_t, sin_t, [n]).astype(np.float64)))
+         for m, n in ((10, 3), (20, 13), (57, 50))]
+    assert max(s) - min(s) <= 1e-5 * np.abs(q).sum() * np.abs(k).sum()
+
+
+def test_prequant_smoothing_step_equals_quantize_rows_scale():
+    """The separate Smooth-QK step followed by plain quantization gives the same
+    codes as quantize_rows with the scale (one product, one rounding)."""
+    rng = np.random.default_rng(42)
+    x = rng.standard_normal((1, 4, 32, 64)).astype(np.float32)
+    s = rng.lognormal(0, 1, (2, 64)).astype(np.float32)
+    a = oracle.quantize_rows(x, s, 2)
+    b = oracle.quantize_rows(oracle.prequant_rows(x, scale=s, group=2))
+    assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
+
+
+# ------------------------------------------------------------------ Q-Mean
+
+def test_q_mean_hand_values_and_exact_shift():
+    N, D = 8, 16
+    x = np.zeros((1, 2, N, D), np.float32)
+    x[0, 0, :, 0] = np.arange(N) * 0.125            # mean 0.4375
+    x[0, 1, :, 3] = [1, -1] * (N // 2)               # mean 0
+    x[0, 1, :, 5] = 3.0
+    m = oracle.q_mean(x)
+    assert m[0, 0, 0] == np.float32(0.4375) and m[0, 1, 3] == 0 and m[0, 1, 5] == 3
+    assert np.count_nonzero(m) == 2
+    # adding a dyadic vector to every token moves the mean by exactly that vector
+    rng = np.random.default_rng(43)
+    y = W.round_to_dtype(rng.standard_normal((1, 2, 64, D)).astype(np.float32), "bf16")
+    shift = (rng.integers(-8, 8, D) * 0.25).astype(np.float32)
+    base = oracle.q_mean(y).astype(np.float64)
+    moved = oracle.q_mean(y + shift).astype(np.float64)
+    # y + shift is exact in fp32 (bf16 values plus quarter integers of small size)
+    assert np.abs(moved - base - shift).max() <= 2 * np.spacing(np.float32(4))
+
+
+def test_q_mean_residual_sums_to_zero():
+    """sum_i (x_i - mean) = N (mean_exact - mean) is within rounding of zero."""
+    rng = np.random.default_rng(44)
+    x = W.round_to_dtype((rng.standard_normal((2, 2, 128, 64)) + 3).astype(np.float32), "bf16")
+    r = oracle.sub_mean(x, oracle.q_mean(x)).astype(np.float64)
+    assert np.abs(r.sum(axis=2)).max() <= 128 * 4 * np.spacing(np.float32(4))
+
+
+def test_q_mean_bias_closed_form_and_bruteforce():
+    """K' = 1 everywhere: the bias of every key is the sum of the mean's
+    channels. Then random keys against a plain fp64 product with GQA heads."""
+    B, Hq, Hkv, Nkv, D = 1, 4, 2, 128, 64
+    rng = np.random.default_rng(45)
+    mean = rng.standard_normal((B, Hq, D)).astype(np.float32)
+    bias = oracle.q_mean_bias(mean, np.ones((B, Hkv, Nkv, D), np.float32), Hq)
+    assert np.abs(bias - mean.astype(np.float64).sum(-1)[..., None]).max() <= 1e-12
+    k = rng.standard_normal((B, Hkv, Nkv, D)).astype(np.float32)
+    bias = oracle.q_mean_bias(mean, k, Hq)
+    for h in range(Hq):
+        want = k[0, h // 2].astype(np.float64) @ mean[0, h].astype(np.float64)
+        assert np.abs(bias[0, h] - want).max() <= 1e-12 * np.abs(want).max()
+
+
+def test_q_mean_constant_rows_give_exact_scores():
+    """Every query row equal to u: the residual quantizes to zero codes, so the
+    scores are u . K exactly (the bias term alone), and the log-sum-exp
+    (high-precision l) equals the brute-force fp64 log-sum-exp of
+    sm_scale * u . K^T. Dropping the bias, flipping its sign or taking it from
+    the quantized keys fails."""
+    B, Hq, Hkv, Nq, Nkv, D = 1, 2, 1, 16, 256, 64
+    rng = np.random.default_rng(46)
+    u = W.round_to_dtype(rng.standard_normal((1, Hq, 1, D)).astype(np.float32) * 2, "bf16")
+    q = np.repeat(u, Nq, axis=2)
+    k = W.round_to_dtype(rng.standard_normal((B, Hkv, Nkv, D)).astype(np.float32), "bf16")
+    v = rng.standard_normal((B, Hkv, Nkv, D)).astype(np.float32)
+    m = oracle.q_mean(q)
+    assert np.array_equal(m[:, :, None, :], u)
+    pk = oracle.quantize_qkv(oracle.sub_mean(q, m), k, v)
+    assert not pk["qc"].any() and not pk["qs"].any()
+    bias = oracle.q_mean_bias(m, k, Hq)
+    out = oracle.attention_rows((B, Hq, Hkv, Nq, Nkv, D), oracle.all_rows(B, Hq, Nq), packed=pk, s_bias=bias,
+                                norm_mode=oracle.HIGH_PRECISION_L)
+    sm = oracle.default_sm_scale(D)
+    for h in range(Hq):
+        s = sm * (k[0, 0].astype(np.float64) @ u[0, h, 0].astype(np.float64))
+        want = s.max() + np.log(np.exp(s - s.max()).sum())
+        assert np.abs(out["lse"][h * Nq:(h + 1) * Nq] - want).max() <= 1e-5
+
+
+def _dequant_rows(codes, sf):
+    e2 = np.array([0, .5, 1, 1.5, 2, 3, 4, 6, -0., -.5, -1, -1.5, -2, -3, -4, -6])
+    el = np.stack([e2[codes & 15], e2[codes >> 4]], -1).reshape(*codes.shape[:-1], codes.shape[-1] * 2)
+    sc = np.array([_e4m3_closed_form(int(c)) for c in range(256)])[sf]
+    return el * np.repeat(sc, 16, axis=-1)
+
+
+def test_q_mean_reduces_score_error_with_a_common_offset():
+    """Q with a shared per-channel offset (the case Q smoothing targets): the
+    4-bit scores with the Q-Mean term are much closer to the fp64 scores of
+    the unquantized operands than the plain 4-bit scores."""
+    B, Hq, Hkv, Nq, Nkv, D = 1, 1, 1, 128, 256, 128
+    rng = np.random.default_rng(47)
+    off = rng.standard_normal(D).astype(np.float32) * 4
+    q = W.round_to_dtype((rng.standard_normal((B, Hq, Nq, D)) + off).astype(np.float32), "bf16")
+    k = W.round_to_dtype(rng.standard_normal((B, Hkv, Nkv, D)).astype(np.float32), "bf16")
+    exact = np.einsum("id,jd->ij", q[0, 0].astype(np.float64), k[0, 0].astype(np.float64))
+    plain = oracle.quantize_qkv(q, k, np.zeros_like(k))
+    S_plain = _dequant_rows(plain["qc"], plain["qs"])[0, 0] @ _dequant_rows(plain["kc"], plain["ks"])[0, 0].T
+    m = oracle.q_mean(q)
+    pm = oracle.quantize_qkv(oracle.sub_mean(q, m), k, np.zeros_like(k))
+    khat = _dequant_rows(pm["kc"], pm["ks"])[0, 0]
+    S_qm = _dequant_rows(pm["qc"], pm["qs"])[0, 0] @ khat.T + oracle.q_mean_bias(m, k, Hq)[0, 0][None, :]
+    e_plain = np.sqrt(np.mean((S_plain - exact) ** 2))
+    e_qm = np.sqrt(np.mean((S_qm - exact) ** 2))
+    assert e_qm < 0.5 * e_plain
+
+
+# ------------------------------------------------------ epsilon-bar tiles
+
+def test_eps_bar_hand_values():
+    """Tile mean over the rows with mass (NaN rows skipped); NaN when no row has any."""
+    B, Hq, Nq, T = 1, 1, 130, 2
+    e = np.full((Nq, T), np.nan)
+    e[0, 0], e[5, 0], e[127, 0] = -0.1, -0.2, 0.3      # q tile 0, kv tile 0: mean 0
+    e[128, 1], e[129, 1] = -0.5, -0.25                 # q tile 1, kv tile 1
+    out = oracle.eps_bar(e, B, Hq, Nq)
+    assert out.shape == (1, 1, 2, 2)
+    assert abs(out[0, 0, 0, 0]) <= 1e-15 and np.isnan(out[0, 0, 0, 1])
+    assert np.isnan(out[0, 0, 1, 0]) and out[0, 0, 1, 1] == -0.375
+
+
+def test_eps_rows_follow_definition_on_a_tiny_case():
+    """Per (row, tile): sum P_hat / sum P - 1, from the P_hat codes the oracle
+    dumps and the fp64 P of a brute-force online softmax."""
+    B, Hq, Hkv, Nq, Nkv, D = 1, 1, 1, 4, 256, 64
+    rng = np.random.default_rng(48)
+    q = W.round_to_dtype(rng.standard_normal((B, Hq, Nq, D)).astype(np.float32), "bf16")
+    k = W.round_to_dtype(rng.standard_normal((B, Hkv, Nkv, D)).astype(np.float32), "bf16")
+    pk = oracle.quantize_qkv(q, k, np.zeros_like(k))
+    out = oracle.attention_rows((B, Hq, Hkv, Nq, Nkv, D), oracle.all_rows(B, Hq, Nq), packed=pk,
+                                want_eps=True, want_p=True)
+    phat = _dequant_rows(out["p_codes"][:, None, None, :], out["p_sf"][:, None, None, :])[:, 0, 0]
+    S = _dequant_rows(pk["qc"], pk["qs"])[0, 0] @ _dequant_rows(pk["kc"], pk["ks"])[0, 0].T
+    c = np.float32(oracle.default_sm_scale(D) * np.log2(np.e))
+    for i in range(Nq):
+        m = -np.inf
+        for t in range(2):
+            s = S[i, 128 * t:128 * (t + 1)].astype(np.float32)
+            m = max(m, float(s.max()))
+            mc = np.float32(np.float32(m) * c)
+            p = np.exp2((s * np.float64(c) - np.float64(mc)))
+            want = phat[i, 128 * t:128 * (t + 1)].sum() / p.sum() - 1
+            assert abs(out["eps"][i, t] - want) <= 1e-6
