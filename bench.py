@@ -373,6 +373,142 @@ def error_vs_fp32(H, packed, q, k, v, cfg, norm, split_kv, max_groups=2):
             "reference": "torch fp32 SDPA on the bf16 inputs (unquantized)"}
 
 
+def eps_stats(H, packed, cfg, norm, split_kv):
+    """The epsilon-bar statistic of the HiFA4 abstract on this workload: per
+    (128-query-row, 128-key) tile, the mean over its rows with mass of
+    sum P_hat / sum P - 1, from the kernel's tile sums (one extra launch of the
+    statistics variant, outside every timed region)."""
+    import torch
+    r = H.attention_fwd_ex(packed, causal=cfg.causal, norm=norm, out_dtype=torch.bfloat16, split_kv=split_kv,
+                           want_tile_sums=True)
+    eb = H.tile_stats(r["tile_sums"])
+    x = eb[~torch.isnan(eb)].double()
+    out = {"tiles": int(x.numel()), "negative_frac": round(float((x < 0).double().mean()), 6),
+           "median": round(float(x.median()), 6), "mean": round(float(x.mean()), 6),
+           "p05": round(float(torch.quantile(x.float(), 0.05)), 6),
+           "p95": round(float(torch.quantile(x.float(), 0.95)), 6)}
+    del r, eb
+    return out
+
+
+def time_fn(fn, n, flush, stream):
+    """Mean device time (ms) of fn over n calls, L2 cold before each."""
+    import torch
+    fn()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+    for i in range(n):
+        flush(i)
+        ev[i][0].record(stream)
+        fn()
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    return statistics.mean(a.elapsed_time(b) for a, b in ev)
+
+
+def run_extensions(args, dev, H):
+    """Timings of the steps around the hot path (one JSON line each): the
+    Q-Mean auxiliary on the Smooth-QK-off workload, the fused RoPE quantize
+    pass, KV-cache appends on the decode workload, and the epsilon statistics."""
+    import torch
+    import torch.nn.functional as F
+    flush = L2Flush(dev)
+    stream = torch.cuda.current_stream()
+    n = args.steps
+    rows = []
+
+    def emit(rec):
+        print(json.dumps(rec), flush=True)
+        rows.append(rec)
+
+    # Q-Mean on the N = 16384 workload (Smooth-QK off)
+    cfg = W.get(4)
+    q, k, v, _ = make_inputs(cfg, dev)
+    packed = H.alloc_packed(cfg.B, cfg.Hq, cfg.Hkv, cfg.Nq, cfg.Nkv, cfg.D, dev)
+    o = torch.empty(cfg.B, cfg.Hq, cfg.Nq, cfg.D, dtype=torch.bfloat16, device=dev)
+    lse = torch.empty(cfg.B, cfg.Hq, cfg.Nq, dtype=torch.float32, device=dev)
+    wsp = H.alloc_workspace(cfg.B, cfg.Hq, cfg.Hkv, cfg.Nq, cfg.Nkv, cfg.D, dev)
+    qm = torch.empty(cfg.B, cfg.Hq, cfg.D, dtype=torch.float32, device=dev)
+    bias = torch.empty(cfg.B, cfg.Hq, cfg.Nkv, dtype=torch.float32, device=dev)
+    t_plain_q = time_fn(lambda: H.quantize_qkv(q, k, v, out=packed), n, flush, stream)
+    t_plain_a = time_fn(lambda: H.attention_fwd(packed, causal=True, out=o, lse=lse, workspace=wsp), n, flush, stream)
+    t_mean = time_fn(lambda: H.q_mean(q, out=qm), n, flush, stream)
+    t_qm_q = time_fn(lambda: H.quantize_qkv(q, k, v, out=packed, q_mean=qm, s_bias=bias), n, flush, stream)
+    t_qm_a = time_fn(lambda: H.attention_fwd_ex(packed, causal=True, out=o, lse=lse, workspace=wsp, s_bias=bias),
+                     n, flush, stream)
+    errs = {}
+    for name, use in (("plain", False), ("q_mean", True)):
+        H.quantize_qkv(q, k, v, out=packed, q_mean=qm if use else None, s_bias=bias if use else None)
+        o4 = H.attention_fwd_ex(packed, causal=True, out_dtype=torch.float32, s_bias=bias if use else None)["o"]
+        b, g = 0, 0
+        hs = slice(0, cfg.G)
+        qq = q[b:b + 1, hs].float()
+        kk = k[b:b + 1, g:g + 1].float().expand(1, cfg.G, cfg.Nkv, cfg.D)
+        vv = v[b:b + 1, g:g + 1].float().expand(1, cfg.G, cfg.Nkv, cfg.D)
+        ref = F.scaled_dot_product_attention(qq, kk, vv, is_causal=True)
+        d = (o4[b:b + 1, hs] - ref).double()
+        rel = (d.norm(dim=-1) / ref.double().norm(dim=-1).clamp_min(1e-30)).flatten()
+        errs[name] = {"max_abs": round(float(d.abs().max()), 6), "row_rel_l2_median": round(float(rel.median()), 6)}
+    fl = cfg.flops()
+    emit({"extension": "q_mean", "workload": cfg.name, "q_mean_ms": round(t_mean, 5),
+          "quantize_ms": {"plain": round(t_plain_q, 5), "q_mean": round(t_qm_q, 5)},
+          "attention_ms": {"plain": round(t_plain_a, 5), "q_mean_bias": round(t_qm_a, 5)},
+          "attention_tflops": {"plain": round(fl / t_plain_a / 1e9, 1), "q_mean_bias": round(fl / t_qm_a / 1e9, 1)},
+          "error_vs_fp32_group0": errs,
+          "note": "attention with the bias runs the extras variant of the kernel"})
+    del q, k, v, packed, o, lse, qm, bias
+    torch.cuda.empty_cache()
+
+    # fused RoPE -> Smooth-QK -> quantize on the headline workload
+    cfg = W.get(2)
+    q, k, v, cal = make_inputs(cfg, dev)
+    s, s_inv = H.calibrate_smooth(cal[0], cal[1], cfg.alpha)
+    cos_t, sin_t = W.rope_tables(cfg.Nkv, cfg.D)
+    pos = torch.arange(cfg.Nkv, dtype=torch.int32, device=dev)
+    rope = H.Rope(torch.from_numpy(cos_t).to(dev), torch.from_numpy(sin_t).to(dev), pos[cfg.Nkv - cfg.Nq:].contiguous(),
+                  pos)
+    packed = H.alloc_packed(cfg.B, cfg.Hq, cfg.Hkv, cfg.Nq, cfg.Nkv, cfg.D, dev)
+    t0 = time_fn(lambda: H.quantize_qkv(q, k, v, s, s_inv, out=packed), n, flush, stream)
+    t1 = time_fn(lambda: H.quantize_qkv(q, k, v, s, s_inv, out=packed, rope=rope), n, flush, stream)
+    elems = cfg.B * cfg.Hq * cfg.Nq * cfg.D + 2 * cfg.B * cfg.Hkv * cfg.Nkv * cfg.D
+    nbytes = elems * (2 + 0.5625)
+    emit({"extension": "rope_quantize", "workload": cfg.name, "quantize_ms": round(t0, 5),
+          "rope_quantize_ms": round(t1, 5), "quantize_gbs": round(nbytes / t0 / 1e6, 1),
+          "rope_quantize_gbs": round(nbytes / t1 / 1e6, 1),
+          "bytes": "algorithmic: 2 B read + 0.5625 B written per Q/K/V element (tables stay in L2)"})
+
+    # epsilon statistics on the headline workload
+    H.quantize_qkv(q, k, v, s, s_inv, out=packed)
+    o = torch.empty(cfg.B, cfg.Hq, cfg.Nq, cfg.D, dtype=torch.bfloat16, device=dev)
+    ts = torch.zeros(cfg.B, cfg.Hq, cfg.Nq, cfg.Nkv // 128, 2, dtype=torch.float32, device=dev)
+    eb = torch.empty(cfg.B, cfg.Hq, cfg.Nq // 128, cfg.Nkv // 128, dtype=torch.float32, device=dev)
+    ta = time_fn(lambda: H.attention_fwd(packed, causal=True, out=o), n, flush, stream)
+    te = time_fn(lambda: H.attention_fwd_ex(packed, causal=True, out=o, tile_sums=ts), n, flush, stream)
+    tt = time_fn(lambda: H.tile_stats(ts, out=eb), n, flush, stream)
+    emit({"extension": "eps_statistics", "workload": cfg.name, "attention_ms": round(ta, 5),
+          "attention_with_tile_sums_ms": round(te, 5), "tile_stats_ms": round(tt, 5),
+          "eps_bar": eps_stats(H, packed, cfg, "p_reorder", False)})
+    del q, k, v, packed, o, ts, eb
+    torch.cuda.empty_cache()
+
+    # KV-cache append on the decode workload (B = 64, 8 kv heads, 8192 slots)
+    cfg = W.get(5)
+    cache = H.alloc_packed(cfg.B, cfg.Hq, cfg.Hkv, cfg.Nq, cfg.Nkv, cfg.D, dev)
+    for n_new in (16, 1024):
+        kn = torch.randn(cfg.B, cfg.Hkv, n_new, cfg.D, device=dev).to(torch.bfloat16)
+        vn = torch.randn_like(kn)
+        start = cfg.Nkv - n_new
+        t = time_fn(lambda: H.append_kv(cache, kn, vn, start), n, flush, stream)
+        nb = 2 * kn.numel() * (2 + 0.5625)
+        emit({"extension": "append_kv", "workload": cfg.name, "new_tokens": n_new, "start": start,
+              "ms": round(t, 5), "gbs": round(nb / t / 1e6, 1),
+              "bytes": "algorithmic: new K and V, 2 B read + 0.5625 B written per element"})
+    if args.table:
+        with open(args.table, "w") as f:
+            for rec in rows:
+                f.write(json.dumps(rec) + "\n")
+
+
 def measure(cfg, norm, args, dev, rank, ws, H, want_e2e=True):
     """Time one workload: the step (quantize + attention, one CUDA graph) with a
     cold L2, the two kernels separately, and (want_e2e) the end-to-end loop."""
@@ -548,6 +684,12 @@ def run_ours(args):
     dev = torch.device("cuda", local)
     pk = peaks()
     fp4_peak = 4.0 * pk["bf16"]                       # burst: the kernel is timed alone, per launch
+    if args.extensions:
+        if rank == 0:
+            run_extensions(args, dev, H)
+        if ws > 1:
+            dist.destroy_process_group()
+        return
     if args.all_configs:
         run_all_configs(args, dev, rank, ws, H, pk, fp4_peak)
         if ws > 1:
@@ -604,6 +746,7 @@ def run_ours(args):
     if rank == 0 and not args.no_extras:
         line["sdpa_bf16_tflops"] = sdpa_context(r["q"], r["k"], r["v"], cfg, r["flush"])
         line["error_vs_fp32"] = error_vs_fp32(H, r["packed"], r["q"], r["k"], r["v"], cfg, norm, r["split_kv"])
+        line["eps_bar"] = eps_stats(H, r["packed"], cfg, norm, r["split_kv"])
         g = fp4_gemm_peak(dev)
         if g is not None:
             line["fp4_gemm_tflops_measured"] = round(g, 1)
@@ -640,6 +783,7 @@ def run_all_configs(args, dev, rank, ws, H, pk, fp4_peak):
             if rank == 0 and not args.no_extras:
                 rec["sdpa_bf16_tflops"] = sdpa_context(r["q"], r["k"], r["v"], cfg, r["flush"])
                 rec["error_vs_fp32"] = error_vs_fp32(H, r["packed"], r["q"], r["k"], r["v"], cfg, norm, r["split_kv"])
+                rec["eps_bar"] = eps_stats(H, r["packed"], cfg, norm, r["split_kv"])
             if rank == 0:
                 print(json.dumps(rec), flush=True)
             rows.append(rec)
@@ -649,8 +793,8 @@ def run_all_configs(args, dev, rank, ws, H, pk, fp4_peak):
         with open(args.table, "w") as f:
             f.write("| workload | norm | kv ranges | step ms | step TFLOP/s | attention ms | attention TFLOP/s | "
                     "bound | roofline frac | quantize ms | bf16 SDPA TFLOP/s | max abs err vs fp32 | "
-                    "row rel L2 (median / max) | SM MHz |\n")
-            f.write("|" + "---|" * 14 + "\n")
+                    "row rel L2 (median / max) | eps_bar median (tiles < 0) | SM MHz |\n")
+            f.write("|" + "---|" * 15 + "\n")
             for x in rows:
                 e = x.get("error_vs_fp32", {})
                 f.write(f"| {x['workload']} | {x['norm']} | {x['kv_splits']} | {x['step_ms']:.4f} | "
@@ -658,6 +802,7 @@ def run_all_configs(args, dev, rank, ws, H, pk, fp4_peak):
                         f"{x['roofline']['bound']} | {x['roofline']['frac']:.3f} | {x['quantize_ms']:.4f} | "
                         f"{x.get('sdpa_bf16_tflops', '')} | {e.get('max_abs', '')} | "
                         f"{e.get('row_rel_l2_median', '')} / {e.get('row_rel_l2_max', '')} | "
+                        f"{x.get('eps_bar', {}).get('median', '')} ({x.get('eps_bar', {}).get('negative_frac', '')}) | "
                         f"{(x['clocks'] or {}).get('sm_mhz', '')} |\n")
 
 
@@ -705,6 +850,8 @@ def main():
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle samples")
     ap.add_argument("--no-extras", action="store_true", help="skip SDPA, fp32-error and FP4-GEMM context")
     ap.add_argument("--all-configs", action="store_true", help="time every workload (one JSON line each)")
+    ap.add_argument("--extensions", action="store_true",
+                    help="time Q-Mean, fused RoPE quantize, KV appends and the epsilon statistics")
     ap.add_argument("--table", help="with --all-configs: also write a markdown table here")
     ap.add_argument("--ingest-ncu", help="record DRAM bytes per attention launch from this ncu CSV")
     ap.add_argument("--workload", help="with --ingest-ncu: the workload name the capture ran")

@@ -7,8 +7,9 @@ quantized probabilities that feed PV. The computation lives in libhifa4.so
 (C ABI, include/hifa4.h); this package is the PyTorch-facing binding.
 """
 from ._lib import HiFA4Error, load  # noqa: F401
-from .api import (PackedQKV, alloc_packed, alloc_workspace, attention_fwd, attention_splits,  # noqa: F401
-                  attention_fwd_debug, attention_fwd_noalloc, calibrate_smooth, debug_set_wait_limit, get_status,
-                  packed_bytes, quantize_kv, quantize_qkv, workspace_bytes)
+from .api import (PackedQKV, Rope, alloc_packed, alloc_workspace, append_kv, attention_fwd,  # noqa: F401
+                  attention_fwd_debug, attention_fwd_ex, attention_fwd_noalloc, attention_splits, calibrate_smooth,
+                  debug_set_wait_limit, get_status, packed_bytes, q_mean, quantize_kv, quantize_qkv, tile_stats,
+                  workspace_bytes)
 
 __version__ = "0.1.0"

@@ -8,7 +8,7 @@ import subprocess
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libhifa4.so")
-SOURCES = ["api.cu", "quantize.cu", "attention.cu", "noalloc.cu"]
+SOURCES = ["api.cu", "quantize.cu", "attention.cu", "stats.cu", "noalloc.cu"]
 HEADERS = ["hifa4_device.cuh", "hifa4_kernels.h", "api_internal.h", os.path.join("..", "..", "include", "hifa4.h")]
 
 

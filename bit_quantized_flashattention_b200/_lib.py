@@ -16,11 +16,23 @@ SPLIT_KV = 2
 EXPORTS = ["hifa4_packed_bytes", "hifa4_workspace_bytes", "hifa4_calibrate_smooth", "hifa4_quantize_qkv",
            "hifa4_quantize_kv", "hifa4_attention_fwd", "hifa4_attention_fwd_debug", "hifa4_get_status",
            "hifa4_debug_set_wait_limit", "hifa4_status_string", "hifa4_version", "hifa4_attention_fwd_noalloc",
-           "hifa4_last_cuda_error", "hifa4_attention_splits"]
+           "hifa4_last_cuda_error", "hifa4_attention_splits", "hifa4_quantize_qkv_ex", "hifa4_q_mean",
+           "hifa4_append_kv", "hifa4_attention_fwd_ex", "hifa4_tile_stats"]
 
 
 class Packed(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in ("qc", "qs", "kc", "ks", "vtc", "vts")]
+
+
+class Prequant(ctypes.Structure):
+    _fields_ = [("s", ctypes.c_void_p), ("s_inv", ctypes.c_void_p), ("rope_cos", ctypes.c_void_p),
+                ("rope_sin", ctypes.c_void_p), ("q_pos", ctypes.c_void_p), ("k_pos", ctypes.c_void_p),
+                ("n_pos", ctypes.c_int), ("q_mean", ctypes.c_void_p), ("s_bias", ctypes.c_void_p)]
+
+
+class AttentionExtras(ctypes.Structure):
+    _fields_ = [("s_bias", ctypes.c_void_p), ("p_codes", ctypes.c_void_p), ("p_scales", ctypes.c_void_p),
+                ("tile_sums", ctypes.c_void_p)]
 
 
 class HiFA4Error(RuntimeError):
@@ -61,6 +73,18 @@ def load():
     L.hifa4_attention_fwd_debug.restype = ci
     L.hifa4_attention_fwd_noalloc.argtypes = [pk] + [ci] * 6 + [cf, cu, ci, vp, ci, vp, vp]
     L.hifa4_attention_fwd_noalloc.restype = ci
+    pre = ctypes.POINTER(Prequant)
+    L.hifa4_quantize_qkv_ex.argtypes = [vp, vp, vp, ci] + [ci] * 6 + [pre, pk, vp]
+    L.hifa4_quantize_qkv_ex.restype = ci
+    L.hifa4_q_mean.argtypes = [vp, ci, ci, ci, ci, ci, ci, pre, vp, vp]
+    L.hifa4_q_mean.restype = ci
+    L.hifa4_append_kv.argtypes = [vp, vp, ci, ci, ci, ci, ci, pre, pk, ci, ci, vp]
+    L.hifa4_append_kv.restype = ci
+    L.hifa4_attention_fwd_ex.argtypes = [pk] + [ci] * 6 + [cf, cu, ci, vp, ci, vp, ctypes.POINTER(AttentionExtras),
+                                                           vp, vp]
+    L.hifa4_attention_fwd_ex.restype = ci
+    L.hifa4_tile_stats.argtypes = [vp, ci, ci, ci, ci, vp, vp]
+    L.hifa4_tile_stats.restype = ci
     L.hifa4_get_status.argtypes = [vp, vp]
     L.hifa4_get_status.restype = ci
     L.hifa4_debug_set_wait_limit.argtypes = [ctypes.c_longlong, ci]

@@ -53,6 +53,7 @@ class PackedQKV:
     Nq: int
     Nkv: int
     D: int
+    s_bias: torch.Tensor | None = None     # Q-Mean score bias written by quantize_qkv(q_mean=...)
 
     def struct(self) -> L.Packed:
         return L.Packed(*(ctypes.c_void_p(t.data_ptr()) for t in
@@ -103,8 +104,39 @@ def calibrate_smooth(q: torch.Tensor, k: torch.Tensor, alpha: float = 0.5, s=Non
     return s, s_inv
 
 
-def quantize_qkv(q, k, v, s=None, s_inv=None, out: PackedQKV | None = None, stream=None) -> PackedQKV:
-    """Smooth (when s/s_inv are given) and quantize Q, K, V to the packed 4-bit operands."""
+@dataclass
+class Rope:
+    """RoPE inputs: fp32 tables [n_pos, D/2] and int32 positions of the query
+    tokens [Nq] and key tokens [Nkv] (or the appended keys [n_new])."""
+    cos: torch.Tensor
+    sin: torch.Tensor
+    q_pos: torch.Tensor | None = None
+    k_pos: torch.Tensor | None = None
+
+
+def _prequant(s=None, s_inv=None, rope: Rope | None = None, q_mean=None, s_bias=None) -> L.Prequant:
+    pq = L.Prequant()
+    pq.s, pq.s_inv, pq.q_mean, pq.s_bias = _ptr(s), _ptr(s_inv), _ptr(q_mean), _ptr(s_bias)
+    if rope is not None:
+        for t, n in ((rope.cos, "rope.cos"), (rope.sin, "rope.sin")):
+            _check_input(t, n, 2)
+            if t.dtype != torch.float32:
+                raise ValueError(f"{n} must be float32")
+        for t, n in ((rope.q_pos, "rope.q_pos"), (rope.k_pos, "rope.k_pos")):
+            if t is not None and (t.dtype != torch.int32 or not t.is_contiguous()):
+                raise ValueError(f"{n} must be a contiguous int32 tensor")
+        pq.rope_cos, pq.rope_sin = _ptr(rope.cos), _ptr(rope.sin)
+        pq.q_pos, pq.k_pos = _ptr(rope.q_pos), _ptr(rope.k_pos)
+        pq.n_pos = int(rope.cos.shape[0])
+    return pq
+
+
+def quantize_qkv(q, k, v, s=None, s_inv=None, out: PackedQKV | None = None, stream=None, rope: Rope | None = None,
+                 q_mean=None, s_bias=None) -> PackedQKV:
+    """Quantize Q, K, V to the packed 4-bit operands, after (in order) RoPE
+    (rope), Smooth-QK (s / s_inv) and the Q-Mean subtraction (q_mean, from
+    q_mean(); the K pass then writes the score bias into s_bias [B,Hq,Nkv],
+    allocated here when None and q_mean is given: read it from ``out.s_bias``)."""
     for x, n in ((q, "q"), (k, "k"), (v, "v")):
         _check_input(x, n)
     B, Hq, Nq, D = q.shape
@@ -113,15 +145,39 @@ def quantize_qkv(q, k, v, s=None, s_inv=None, out: PackedQKV | None = None, stre
         raise ValueError("q, k, v shapes / dtypes do not match")
     if out is None:
         out = alloc_packed(B, Hq, Hkv, Nq, Nkv, D, q.device)
+    if q_mean is not None and s_bias is None:
+        s_bias = torch.empty(B, Hq, Nkv, dtype=torch.float32, device=q.device)
     st = out.struct()
-    L.check(L.load().hifa4_quantize_qkv(_ptr(q), _ptr(k), _ptr(v), _DT[q.dtype], B, Hq, Hkv, Nq, Nkv, D,
-                                        _ptr(s), _ptr(s_inv), ctypes.byref(st), _stream(stream)), "quantize_qkv")
+    if rope is None and q_mean is None:
+        L.check(L.load().hifa4_quantize_qkv(_ptr(q), _ptr(k), _ptr(v), _DT[q.dtype], B, Hq, Hkv, Nq, Nkv, D,
+                                            _ptr(s), _ptr(s_inv), ctypes.byref(st), _stream(stream)), "quantize_qkv")
+    else:
+        pq = _prequant(s, s_inv, rope, q_mean, s_bias)
+        L.check(L.load().hifa4_quantize_qkv_ex(_ptr(q), _ptr(k), _ptr(v), _DT[q.dtype], B, Hq, Hkv, Nq, Nkv, D,
+                                               ctypes.byref(pq), ctypes.byref(st), _stream(stream)),
+                "quantize_qkv_ex")
+    out.s_bias = s_bias
+    return out
+
+
+def q_mean(q, s=None, rope: Rope | None = None, out=None, Hkv: int | None = None, stream=None) -> torch.Tensor:
+    """Q-Mean auxiliary: per-(b, h, channel) mean [B,Hq,D] fp32 of Q after RoPE
+    and smoothing (s needs Hkv, the kv heads it is indexed by)."""
+    _check_input(q, "q")
+    B, Hq, Nq, D = q.shape
+    if Hkv is None:
+        Hkv = s.shape[0] if s is not None else Hq
+    if out is None:
+        out = torch.empty(B, Hq, D, dtype=torch.float32, device=q.device)
+    pq = _prequant(s, s, rope)
+    L.check(L.load().hifa4_q_mean(_ptr(q), _DT[q.dtype], B, Hq, Hkv, Nq, D, ctypes.byref(pq), _ptr(out),
+                                  _stream(stream)), "q_mean")
     return out
 
 
 def quantize_kv(k, v, s_inv=None, out: PackedQKV | None = None, Hq: int | None = None, Nq: int = 16,
                 stream=None) -> PackedQKV:
-    """Quantize K and V only (e.g. when a KV cache is appended)."""
+    """Quantize K and V only (a whole KV cache at once; see append_kv)."""
     _check_input(k, "k")
     _check_input(v, "v")
     B, Hkv, Nkv, D = k.shape
@@ -131,6 +187,23 @@ def quantize_kv(k, v, s_inv=None, out: PackedQKV | None = None, Hq: int | None =
     L.check(L.load().hifa4_quantize_kv(_ptr(k), _ptr(v), _DT[k.dtype], B, Hkv, Nkv, D, _ptr(s_inv),
                                        ctypes.byref(st), _stream(stream)), "quantize_kv")
     return out
+
+
+def append_kv(cache: PackedQKV, k_new, v_new, start: int, s_inv=None, rope: Rope | None = None,
+              stream=None) -> PackedQKV:
+    """Quantize new K/V tokens [B,Hkv,n_new,D] into cache token slots
+    [start, start + n_new) (both multiples of 16); RoPE uses rope.k_pos [n_new]."""
+    _check_input(k_new, "k_new")
+    _check_input(v_new, "v_new")
+    B, Hkv, n_new, D = k_new.shape
+    if v_new.shape != k_new.shape or (B, Hkv, D) != (cache.B, cache.Hkv, cache.D):
+        raise ValueError("new tokens do not match the cache")
+    pq = _prequant(s_inv, s_inv, rope)
+    pq.s = None
+    st = cache.struct()
+    L.check(L.load().hifa4_append_kv(_ptr(k_new), _ptr(v_new), _DT[k_new.dtype], B, Hkv, n_new, D, ctypes.byref(pq),
+                                     ctypes.byref(st), cache.Nkv, int(start), _stream(stream)), "append_kv")
+    return cache
 
 
 def attention_splits(B, Hq, Hkv, Nq, Nkv, D, causal=False, split_kv=False) -> int:
@@ -204,6 +277,51 @@ def attention_fwd_debug(packed: PackedQKV, sm_scale: float | None = None, causal
                                                _ptr(out), _DT[out.dtype], _ptr(lse), _ptr(pc), _ptr(ps),
                                                _ptr(workspace), _stream(stream)), "attention_fwd_debug")
     return out, lse, pc, ps
+
+
+def attention_fwd_ex(packed: PackedQKV, sm_scale: float | None = None, causal: bool = False,
+                     norm="p_reorder", out_dtype=torch.bfloat16, out=None, lse=None, workspace=None, stream=None,
+                     split_kv: bool = False, s_bias=None, want_p: bool = False, want_tile_sums: bool = False,
+                     tile_sums=None):
+    """attention_fwd with the extras of hifa4_attention_fwd_ex: the score bias
+    s_bias [B,Hq,Nkv] (Q-Mean), and optionally the P_hat dump and the
+    per-(row, kv tile) sums (sum P_hat, sum P) [B,Hq,Nq,Nkv/128,2] (written
+    into ``tile_sums`` when given, else into a zeroed new tensor).
+    Returns dict(o, lse, p_codes, p_scales, tile_sums)."""
+    sm_scale, flags, nm, out, lse, workspace = _attn_args(packed, sm_scale, causal, norm, out_dtype, out, lse,
+                                                          workspace, True, split_kv)
+    B, Hq, Hkv, Nq, Nkv, D = packed.shape
+    dev = out.device
+    pc = torch.zeros(B, Hq, Nq, Nkv // 2, dtype=torch.uint8, device=dev) if want_p else None
+    ps = torch.zeros(B, Hq, Nq, Nkv // 16, dtype=torch.uint8, device=dev) if want_p else None
+    ts = tile_sums
+    if ts is None and want_tile_sums:
+        ts = torch.zeros(B, Hq, Nq, Nkv // 128, 2, dtype=torch.float32, device=dev)
+    if ts is not None and (ts.shape != (B, Hq, Nq, Nkv // 128, 2) or ts.dtype != torch.float32
+                           or not ts.is_contiguous() or not ts.is_cuda):
+        raise ValueError("tile_sums must be a contiguous float32 CUDA tensor [B, Hq, Nq, Nkv/128, 2]")
+    if s_bias is not None and (s_bias.shape != (B, Hq, Nkv) or s_bias.dtype != torch.float32
+                               or not s_bias.is_contiguous()):
+        raise ValueError("s_bias must be a contiguous float32 [B, Hq, Nkv] tensor")
+    ex = L.AttentionExtras(_ptr(s_bias), _ptr(pc), _ptr(ps), _ptr(ts))
+    st = packed.struct()
+    L.check(L.load().hifa4_attention_fwd_ex(ctypes.byref(st), B, Hq, Hkv, Nq, Nkv, D, float(sm_scale), flags, nm,
+                                            _ptr(out), _DT[out.dtype], _ptr(lse), ctypes.byref(ex), _ptr(workspace),
+                                            _stream(stream)), "attention_fwd_ex")
+    return dict(o=out, lse=lse, p_codes=pc, p_scales=ps, tile_sums=ts)
+
+
+def tile_stats(tile_sums: torch.Tensor, out=None, stream=None) -> torch.Tensor:
+    """Per-tile epsilon-bar [B,Hq,ceil(Nq/128),Nkv/128] (NaN: tile without mass)
+    from the tile sums of attention_fwd_ex."""
+    _check_input(tile_sums, "tile_sums", 5)
+    B, Hq, Nq, T, two = tile_sums.shape
+    if two != 2 or tile_sums.dtype != torch.float32:
+        raise ValueError("tile_sums must be float32 [B, Hq, Nq, Nkv/128, 2]")
+    if out is None:
+        out = torch.empty(B, Hq, (Nq + 127) // 128, T, dtype=torch.float32, device=tile_sums.device)
+    L.check(L.load().hifa4_tile_stats(_ptr(tile_sums), B, Hq, Nq, T * 128, _ptr(out), _stream(stream)), "tile_stats")
+    return out
 
 
 def get_status(workspace: torch.Tensor, stream=None) -> int:

@@ -87,6 +87,34 @@ bool decode_mode(int Hq, int Hkv, int Nq, int Nkv, int D, unsigned flags) {
            Nkv / 128 >= kDecodeSplits;
 }
 
+// Checks of the optional steps before quantization; want_q / want_k: the
+// call quantizes Q / K (their positions are then needed with RoPE).
+hifa4_status check_prequant(const hifa4_prequant& x, bool want_q, bool want_k) {
+    if ((x.s == nullptr) != (x.s_inv == nullptr)) return HIFA4_ERR_INVALID_ARG;
+    if (!aligned16(x.s) || !aligned16(x.s_inv)) return HIFA4_ERR_INVALID_ARG;
+    if ((x.rope_cos == nullptr) != (x.rope_sin == nullptr)) return HIFA4_ERR_INVALID_ARG;
+    if (x.rope_cos != nullptr) {
+        if (!aligned16(x.rope_cos) || !aligned16(x.rope_sin) || x.n_pos <= 0) return HIFA4_ERR_INVALID_ARG;
+        if (want_q && (x.q_pos == nullptr || (reinterpret_cast<uintptr_t>(x.q_pos) & 3u))) return HIFA4_ERR_INVALID_ARG;
+        if (want_k && (x.k_pos == nullptr || (reinterpret_cast<uintptr_t>(x.k_pos) & 3u))) return HIFA4_ERR_INVALID_ARG;
+    }
+    if ((x.q_mean == nullptr) != (x.s_bias == nullptr)) return HIFA4_ERR_INVALID_ARG;
+    if (!aligned16(x.q_mean) || !aligned16(x.s_bias)) return HIFA4_ERR_INVALID_ARG;
+    return HIFA4_OK;
+}
+
+void set_prequant(QuantArgs& a, const hifa4_prequant& x) {
+    a.s = x.s;
+    a.s_inv = x.s_inv;
+    a.rope_cos = x.rope_cos;
+    a.rope_sin = x.rope_sin;
+    a.q_pos = x.q_pos;
+    a.k_pos = x.k_pos;
+    a.n_pos = x.n_pos;
+    a.q_mean = x.q_mean;
+    a.s_bias = x.s_bias;
+}
+
 }  // namespace
 
 hifa4_status hifa4::from_cuda(cudaError_t e) {
@@ -121,12 +149,16 @@ namespace {
 
 hifa4_status attention_impl(const hifa4_packed* in, int B, int Hq, int Hkv, int Nq, int Nkv, int D, float sm_scale,
                             unsigned flags, hifa4_norm_mode norm, void* o, hifa4_dtype o_dtype, float* lse,
-                            uint8_t* p_codes, uint8_t* p_sf, bool dump, void* workspace, hifa4_stream_t stream) {
+                            const hifa4_attention_extras* ex, void* workspace, hifa4_stream_t stream) {
     const hifa4_status chk = check_attention_args(in, B, Hq, Hkv, Nq, Nkv, D, sm_scale, flags, norm, o, o_dtype, lse);
     if (chk != HIFA4_OK) return chk;
     if (workspace == nullptr || !aligned16(workspace)) return HIFA4_ERR_INVALID_ARG;
-    if (dump && (p_codes == nullptr || p_sf == nullptr || !aligned16(p_codes) || !aligned16(p_sf)))
+    hifa4_attention_extras x{};
+    if (ex != nullptr) x = *ex;
+    if ((x.p_codes == nullptr) != (x.p_scales == nullptr)) return HIFA4_ERR_INVALID_ARG;
+    if (!aligned16(x.p_codes) || !aligned16(x.p_scales) || !aligned16(x.s_bias) || !aligned16(x.tile_sums))
         return HIFA4_ERR_INVALID_ARG;
+    const bool extras = x.p_codes != nullptr || x.s_bias != nullptr || x.tile_sums != nullptr;
     const bool causal = (flags & HIFA4_CAUSAL) != 0;
     const long long rows_q = (long long)B * Hq * Nq, rows_k = (long long)B * Hkv * Nkv, rows_v = (long long)B * Hkv * D;
     const Sizes sz = sizes_of(B, Hq, Hkv, Nq, Nkv, D);
@@ -148,8 +180,10 @@ hifa4_status attention_impl(const hifa4_packed* in, int B, int Hq, int Hkv, int 
     p.vts = static_cast<const uint8_t*>(in->vts);
     p.o = o;
     p.lse = lse;
-    p.p_codes = p_codes;
-    p.p_sf = p_sf;
+    p.s_bias = x.s_bias;
+    p.p_codes = x.p_codes;
+    p.p_sf = x.p_scales;
+    p.tile_sums = reinterpret_cast<float2*>(x.tile_sums);
     p.status = static_cast<uint32_t*>(workspace);
     p.B = B;
     p.Hq = Hq;
@@ -166,7 +200,7 @@ hifa4_status attention_impl(const hifa4_packed* in, int B, int Hq, int Hkv, int 
     p.wait_limit_ns = lim > 0 ? (unsigned long long)lim : kDefaultWaitNs;
     p.stall_loads = g_stall_loads.load();
     const int out = o_dtype == HIFA4_F16 ? 0 : (o_dtype == HIFA4_BF16 ? 1 : 2);
-    return from_cuda(launch_attention(&tq, &tk, &tv, p, D, (int)norm, causal, out, dump, dec,
+    return from_cuda(launch_attention(&tq, &tk, &tv, p, D, (int)norm, causal, out, extras, dec,
                                       reinterpret_cast<cudaStream_t>(stream)));
 }
 
@@ -211,27 +245,38 @@ hifa4_status hifa4_calibrate_smooth(const void* q, const void* k, hifa4_dtype dt
                                       reinterpret_cast<cudaStream_t>(stream)));
 }
 
-hifa4_status hifa4_quantize_kv(const void* k, const void* v, hifa4_dtype dtype, int B, int Hkv, int Nkv, int D,
-                               const float* s_inv, const hifa4_packed* out, hifa4_stream_t stream) {
-    if (k == nullptr || v == nullptr || out == nullptr) return HIFA4_ERR_INVALID_ARG;
+hifa4_status hifa4_quantize_qkv_ex(const void* q, const void* k, const void* v, hifa4_dtype dtype, int B, int Hq,
+                                   int Hkv, int Nq, int Nkv, int D, const hifa4_prequant* pre,
+                                   const hifa4_packed* out, hifa4_stream_t stream) {
+    if (q == nullptr || k == nullptr || v == nullptr || out == nullptr) return HIFA4_ERR_INVALID_ARG;
     if (dtype != HIFA4_F16 && dtype != HIFA4_BF16) return HIFA4_ERR_INVALID_ARG;
-    if (!shape_ok(B, Hkv, Hkv, 16, Nkv, D)) return HIFA4_ERR_UNSUPPORTED;
-    const void* ptrs[6] = {k, v, out->kc, out->ks, out->vtc, out->vts};
-    for (const void* q : ptrs)
-        if (q == nullptr || !aligned16(q)) return HIFA4_ERR_INVALID_ARG;
-    if (s_inv != nullptr && !aligned16(s_inv)) return HIFA4_ERR_INVALID_ARG;
+    if (!shape_ok(B, Hq, Hkv, Nq, Nkv, D)) return HIFA4_ERR_UNSUPPORTED;
+    const void* ptrs[9] = {q, k, v, out->qc, out->qs, out->kc, out->ks, out->vtc, out->vts};
+    for (const void* p : ptrs)
+        if (p == nullptr || !aligned16(p)) return HIFA4_ERR_INVALID_ARG;
+    hifa4_prequant x{};
+    if (pre != nullptr) x = *pre;
+    const hifa4_status pc = check_prequant(x, true, true);
+    if (pc != HIFA4_OK) return pc;
+    if ((long long)B * Hq * Nq > INT32_MAX || (long long)B * Hkv * Nkv > INT32_MAX) return HIFA4_ERR_UNSUPPORTED;
+    const Sizes sz = sizes_of(B, Hq, Hkv, Nq, Nkv, D);
     QuantArgs a{};
     a.bf16 = dtype == HIFA4_BF16;
     a.D = D;
-    a.G = 1;
+    a.G = Hq / Hkv;
     a.hkv = Hkv;
-    a.nq = 0;
+    a.nq = Nq;
     a.nkv = Nkv;
-    a.tiles_q = 0;
+    a.nkv_in = Nkv;
+    a.kv_start = 0;
+    a.tiles_q = sz.Tq;
     a.n_groups = (long long)B * Hkv;
+    a.q = q;
     a.k = k;
     a.v = v;
-    a.s_inv = s_inv;
+    set_prequant(a, x);
+    a.qc = static_cast<uint8_t*>(out->qc);
+    a.qs = static_cast<uint8_t*>(out->qs);
     a.kc = static_cast<uint8_t*>(out->kc);
     a.ks = static_cast<uint8_t*>(out->ks);
     a.vtc = static_cast<uint8_t*>(out->vtc);
@@ -242,51 +287,126 @@ hifa4_status hifa4_quantize_kv(const void* k, const void* v, hifa4_dtype dtype, 
 hifa4_status hifa4_quantize_qkv(const void* q, const void* k, const void* v, hifa4_dtype dtype, int B, int Hq, int Hkv,
                                 int Nq, int Nkv, int D, const float* s, const float* s_inv, const hifa4_packed* out,
                                 hifa4_stream_t stream) {
-    if (q == nullptr || k == nullptr || v == nullptr || out == nullptr) return HIFA4_ERR_INVALID_ARG;
-    if ((s == nullptr) != (s_inv == nullptr)) return HIFA4_ERR_INVALID_ARG;
+    hifa4_prequant x{};
+    x.s = s;
+    x.s_inv = s_inv;
+    return hifa4_quantize_qkv_ex(q, k, v, dtype, B, Hq, Hkv, Nq, Nkv, D, &x, out, stream);
+}
+
+hifa4_status hifa4_append_kv(const void* k, const void* v, hifa4_dtype dtype, int B, int Hkv, int n_new, int D,
+                             const hifa4_prequant* pre, const hifa4_packed* cache, int cache_tokens, int start,
+                             hifa4_stream_t stream) {
+    if (k == nullptr || v == nullptr || cache == nullptr) return HIFA4_ERR_INVALID_ARG;
     if (dtype != HIFA4_F16 && dtype != HIFA4_BF16) return HIFA4_ERR_INVALID_ARG;
-    if (!shape_ok(B, Hq, Hkv, Nq, Nkv, D)) return HIFA4_ERR_UNSUPPORTED;
-    const void* ptrs[9] = {q, k, v, out->qc, out->qs, out->kc, out->ks, out->vtc, out->vts};
+    if (!shape_ok(B, Hkv, Hkv, 16, cache_tokens, D)) return HIFA4_ERR_UNSUPPORTED;
+    if (n_new <= 0 || n_new % 16 != 0 || start < 0 || start % 16 != 0 || (long long)start + n_new > cache_tokens)
+        return HIFA4_ERR_INVALID_ARG;
+    const void* ptrs[6] = {k, v, cache->kc, cache->ks, cache->vtc, cache->vts};
     for (const void* p : ptrs)
         if (p == nullptr || !aligned16(p)) return HIFA4_ERR_INVALID_ARG;
-    if ((s != nullptr && !aligned16(s)) || (s_inv != nullptr && !aligned16(s_inv))) return HIFA4_ERR_INVALID_ARG;
-    const Sizes sz = sizes_of(B, Hq, Hkv, Nq, Nkv, D);
+    hifa4_prequant x{};
+    if (pre != nullptr) x = *pre;
+    if (x.q_mean != nullptr || x.s_bias != nullptr) return HIFA4_ERR_INVALID_ARG;
+    x.s = x.s_inv;                                  // only s_inv applies to K (pairing checked on s_inv alone)
+    const hifa4_status pc = check_prequant(x, false, true);
+    if (pc != HIFA4_OK) return pc;
+    x.s = nullptr;
+    if ((long long)B * Hkv * cache_tokens > INT32_MAX) return HIFA4_ERR_UNSUPPORTED;
     QuantArgs a{};
     a.bf16 = dtype == HIFA4_BF16;
     a.D = D;
-    a.G = Hq / Hkv;
+    a.G = 1;
     a.hkv = Hkv;
-    a.nq = Nq;
-    a.nkv = Nkv;
-    a.tiles_q = sz.Tq;
+    a.nq = 0;
+    a.nkv = cache_tokens;
+    a.nkv_in = n_new;
+    a.kv_start = start;
+    a.tiles_q = 0;
     a.n_groups = (long long)B * Hkv;
-    a.q = q;
     a.k = k;
     a.v = v;
-    a.s = s;
-    a.s_inv = s_inv;
-    a.qc = static_cast<uint8_t*>(out->qc);
-    a.qs = static_cast<uint8_t*>(out->qs);
-    a.kc = static_cast<uint8_t*>(out->kc);
-    a.ks = static_cast<uint8_t*>(out->ks);
-    a.vtc = static_cast<uint8_t*>(out->vtc);
-    a.vts = static_cast<uint8_t*>(out->vts);
+    set_prequant(a, x);
+    a.kc = static_cast<uint8_t*>(cache->kc);
+    a.ks = static_cast<uint8_t*>(cache->ks);
+    a.vtc = static_cast<uint8_t*>(cache->vtc);
+    a.vts = static_cast<uint8_t*>(cache->vts);
     return from_cuda(launch_quantize_qkv(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+hifa4_status hifa4_quantize_kv(const void* k, const void* v, hifa4_dtype dtype, int B, int Hkv, int Nkv, int D,
+                               const float* s_inv, const hifa4_packed* out, hifa4_stream_t stream) {
+    if (out == nullptr) return HIFA4_ERR_INVALID_ARG;
+    hifa4_prequant x{};
+    x.s_inv = s_inv;
+    return hifa4_append_kv(k, v, dtype, B, Hkv, Nkv, D, &x, out, Nkv, 0, stream);
+}
+
+hifa4_status hifa4_q_mean(const void* q, hifa4_dtype dtype, int B, int Hq, int Hkv, int Nq, int D,
+                          const hifa4_prequant* pre, float* q_mean, hifa4_stream_t stream) {
+    if (q == nullptr || q_mean == nullptr) return HIFA4_ERR_INVALID_ARG;
+    if (dtype != HIFA4_F16 && dtype != HIFA4_BF16) return HIFA4_ERR_INVALID_ARG;
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || Nq <= 0 || Hq % Hkv != 0) return HIFA4_ERR_INVALID_ARG;
+    if (D != 64 && D != 128 && D != 256) return HIFA4_ERR_UNSUPPORTED;
+    if (!aligned16(q) || !aligned16(q_mean)) return HIFA4_ERR_INVALID_ARG;
+    hifa4_prequant x{};
+    if (pre != nullptr) x = *pre;
+    x.s_inv = x.s;                                  // only s applies to Q (pairing checked on s alone)
+    x.q_mean = nullptr;
+    x.s_bias = nullptr;
+    const hifa4_status pc = check_prequant(x, true, false);
+    if (pc != HIFA4_OK) return pc;
+    if ((long long)B * Hq > INT32_MAX) return HIFA4_ERR_UNSUPPORTED;
+    QMeanArgs a{};
+    a.bf16 = dtype == HIFA4_BF16;
+    a.B = B;
+    a.Hq = Hq;
+    a.Hkv = Hkv;
+    a.Nq = Nq;
+    a.D = D;
+    a.q = q;
+    a.s = x.s;
+    a.rope_cos = x.rope_cos;
+    a.rope_sin = x.rope_sin;
+    a.q_pos = x.q_pos;
+    a.n_pos = x.n_pos;
+    a.mean = q_mean;
+    return from_cuda(launch_q_mean(a, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 hifa4_status hifa4_attention_fwd(const hifa4_packed* in, int B, int Hq, int Hkv, int Nq, int Nkv, int D,
                                  float sm_scale, unsigned flags, hifa4_norm_mode norm, void* o, hifa4_dtype o_dtype,
                                  float* lse, void* workspace, hifa4_stream_t stream) {
-    return attention_impl(in, B, Hq, Hkv, Nq, Nkv, D, sm_scale, flags, norm, o, o_dtype, lse, nullptr, nullptr, false,
-                          workspace, stream);
+    return attention_impl(in, B, Hq, Hkv, Nq, Nkv, D, sm_scale, flags, norm, o, o_dtype, lse, nullptr, workspace,
+                          stream);
+}
+
+hifa4_status hifa4_attention_fwd_ex(const hifa4_packed* in, int B, int Hq, int Hkv, int Nq, int Nkv, int D,
+                                    float sm_scale, unsigned flags, hifa4_norm_mode norm, void* o,
+                                    hifa4_dtype o_dtype, float* lse, const hifa4_attention_extras* extras,
+                                    void* workspace, hifa4_stream_t stream) {
+    return attention_impl(in, B, Hq, Hkv, Nq, Nkv, D, sm_scale, flags, norm, o, o_dtype, lse, extras, workspace,
+                          stream);
 }
 
 hifa4_status hifa4_attention_fwd_debug(const hifa4_packed* in, int B, int Hq, int Hkv, int Nq, int Nkv, int D,
                                        float sm_scale, unsigned flags, hifa4_norm_mode norm, void* o,
                                        hifa4_dtype o_dtype, float* lse, uint8_t* p_codes, uint8_t* p_scales,
                                        void* workspace, hifa4_stream_t stream) {
-    return attention_impl(in, B, Hq, Hkv, Nq, Nkv, D, sm_scale, flags, norm, o, o_dtype, lse, p_codes, p_scales, true,
-                          workspace, stream);
+    if (p_codes == nullptr || p_scales == nullptr) return HIFA4_ERR_INVALID_ARG;
+    hifa4_attention_extras x{};
+    x.p_codes = p_codes;
+    x.p_scales = p_scales;
+    return attention_impl(in, B, Hq, Hkv, Nq, Nkv, D, sm_scale, flags, norm, o, o_dtype, lse, &x, workspace, stream);
+}
+
+hifa4_status hifa4_tile_stats(const float* tile_sums, int B, int Hq, int Nq, int Nkv, float* eps_bar,
+                              hifa4_stream_t stream) {
+    if (tile_sums == nullptr || eps_bar == nullptr) return HIFA4_ERR_INVALID_ARG;
+    if (B <= 0 || Hq <= 0 || Nq <= 0 || Nkv <= 0 || Nkv % 128 != 0) return HIFA4_ERR_INVALID_ARG;
+    if (!aligned16(tile_sums) || (reinterpret_cast<uintptr_t>(eps_bar) & 3u)) return HIFA4_ERR_INVALID_ARG;
+    if ((long long)B * Hq > INT32_MAX) return HIFA4_ERR_UNSUPPORTED;
+    return from_cuda(launch_tile_stats(reinterpret_cast<const float2*>(tile_sums), B * Hq, Nq, Nkv / 128, eps_bar,
+                                       reinterpret_cast<cudaStream_t>(stream)));
 }
 
 hifa4_status hifa4_get_status(void* workspace, hifa4_stream_t stream) {

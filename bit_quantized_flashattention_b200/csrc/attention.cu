@@ -41,6 +41,10 @@
 //
 // TMEM (512 columns): S [0,128), O tiles [128, 128 + NQT*NO), then the
 // scale-factor regions of Q, K, P and V.
+// The EXTRAS variant also takes an additive score term per (head, key)
+// (the Q-Mean bias) and writes, where asked, each row's P_hat codes and
+// scales and its per-tile sums (sum P_hat, sum P) for the epsilon statistics.
+//
 // Every mbarrier wait is bounded; when one gives up the CTA records
 // HIFA4_ERR_TIMEOUT in the workspace, drains its copies and MMAs, frees TMEM
 // and exits; the warps then keep meeting at the named barriers (doing no
@@ -183,7 +187,7 @@ __device__ __forceinline__ void store_out(void* dst, const float* v) {
     }
 }
 
-template <int D, bool PREORDER, bool CAUSAL, int OUT, bool DUMP, bool DEC>
+template <int D, bool PREORDER, bool CAUSAL, int OUT, bool EXTRAS, bool DEC>
 __global__ void __launch_bounds__(Cfg<D, PREORDER, DEC>::THREADS, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
@@ -674,6 +678,9 @@ __global__ void __launch_bounds__(Cfg<D, PREORDER, DEC>::THREADS, 1)
         const float one_sixth = rn_one_sixth();
         const uint32_t lut_s = smem_u32(lut);
         float m_old = -INFINITY, mc_old = 0.0f, l_hp = 0.0f;
+        const float* bias_row = nullptr;                    // score term of this row's head (EXTRAS)
+        if constexpr (EXTRAS)
+            if (p.s_bias != nullptr && valid) bias_row = p.s_bias + (out_row / (size_t)p.Nq) * (size_t)p.Nkv;
         bool ok = true;                                     // false once a wait gave up (then no more work)
         for (int j = 0; j < nt; ++j) {
             HIFA4_TRACE_POINT(qt, j, 0);
@@ -704,6 +711,17 @@ __global__ void __launch_bounds__(Cfg<D, PREORDER, DEC>::THREADS, 1)
                 // (decode: a row whose range has ended masks the whole step)
                 const int n0 = (kt0 + j) * 128;
                 const int lim = j < own_steps ? last : -1;
+                if constexpr (EXTRAS) {
+                    if (bias_row != nullptr && j < own_steps) {
+                        const float4* bp = reinterpret_cast<const float4*>(bias_row + n0);
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) {
+                            const float4 b4 = __ldg(bp + e);
+                            S[2 * e] = make_float2(__fadd_rn(S[2 * e].x, b4.x), __fadd_rn(S[2 * e].y, b4.y));
+                            S[2 * e + 1] = make_float2(__fadd_rn(S[2 * e + 1].x, b4.z), __fadd_rn(S[2 * e + 1].y, b4.w));
+                        }
+                    }
+                }
                 if (n0 + 127 > lim) {
 #pragma unroll
                     for (int e = 0; e < 64; ++e) {
@@ -737,7 +755,7 @@ __global__ void __launch_bounds__(Cfg<D, PREORDER, DEC>::THREADS, 1)
                         for (int e = 0; e < 4; ++e) {
                             const float2 t = __ffma2_rn(S[8 * b + 4 * h + e], c2, nmc2);
                             const float2 P = make_float2(ex2_approx(t.x), ex2_approx(t.y));
-                            if constexpr (!PREORDER) lsum2 = __fadd2_rn(lsum2, P);
+                            if constexpr (!PREORDER || EXTRAS) lsum2 = __fadd2_rn(lsum2, P);
                             const float2 yy = __fmul2_rn(P, r2);
                             y[2 * e] = yy.x;
                             y[2 * e + 1] = yy.y;
@@ -790,9 +808,19 @@ __global__ void __launch_bounds__(Cfg<D, PREORDER, DEC>::THREADS, 1)
                     tmem_st1(tl + C::COL_SFP + qt * 8 + wq, sfw[0]);
                     tmem_st1(tl + C::COL_SFP + qt * 8 + 4 + wq, sfw[1]);
                     tmem_wait_st();
-                    if constexpr (DUMP) {
-                        // debug copy of this row's P_hat codes and scales
-                        if (valid && j < own_steps) {
+                    if constexpr (EXTRAS) {
+                        // per-tile mass of P_hat (codes x scales) and of P
+                        if (p.tile_sums != nullptr && valid && j < own_steps) {
+                            float sh = 0.0f;
+#pragma unroll
+                            for (int b = 0; b < 8; ++b) {
+                                const uint32_t sf = (sfw[b >> 2] >> (8 * (b & 3))) & 0xFFu;
+                                sh = __fmaf_rn(e4m3_to_f32(sf), e2m1x8_sum(code[2 * b]) + e2m1x8_sum(code[2 * b + 1]), sh);
+                            }
+                            p.tile_sums[out_row * (size_t)p.n_kv_tiles + (kt0 + j)] = make_float2(sh, lsum2.x + lsum2.y);
+                        }
+                        // copy of this row's P_hat codes and scales
+                        if (p.p_codes != nullptr && valid && j < own_steps) {
                             uint4* dc = reinterpret_cast<uint4*>(p.p_codes + out_row * (size_t)(p.Nkv / 2) + n0 / 2);
 #pragma unroll
                             for (int q = 0; q < 4; ++q)
@@ -920,11 +948,11 @@ __global__ void __launch_bounds__(Cfg<D, PREORDER, DEC>::THREADS, 1)
     if (threadIdx.x == 0) HIFA4_TRACE_POINT(4, 63, 2);
 }
 
-template <int D, bool PRE, bool CAUSAL, int OUT, bool DUMP, bool DEC>
+template <int D, bool PRE, bool CAUSAL, int OUT, bool EXTRAS, bool DEC>
 static cudaError_t launch_one(const CUtensorMap* q, const CUtensorMap* k, const CUtensorMap* v, const AttnParams& p,
                               cudaStream_t st) {
     using C = Cfg<D, PRE, DEC>;
-    auto kern = attn_fwd_kernel<D, PRE, CAUSAL, OUT, DUMP, DEC>;
+    auto kern = attn_fwd_kernel<D, PRE, CAUSAL, OUT, EXTRAS, DEC>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t lc{};
@@ -940,51 +968,51 @@ static cudaError_t launch_one(const CUtensorMap* q, const CUtensorMap* k, const 
     return cudaLaunchKernelEx(&lc, kern, *q, *k, *v, p);
 }
 
-template <int D, bool PRE, bool CAUSAL, int OUT, bool DUMP>
+template <int D, bool PRE, bool CAUSAL, int OUT, bool EXTRAS>
 static cudaError_t launch_dec(const CUtensorMap* q, const CUtensorMap* k, const CUtensorMap* v, const AttnParams& p,
                               bool dec, cudaStream_t st) {
     if constexpr (D <= 128) {
-        if (dec) return launch_one<D, PRE, CAUSAL, OUT, DUMP, true>(q, k, v, p, st);
+        if (dec) return launch_one<D, PRE, CAUSAL, OUT, EXTRAS, true>(q, k, v, p, st);
     } else {
         if (dec) return cudaErrorInvalidValue;
     }
-    return launch_one<D, PRE, CAUSAL, OUT, DUMP, false>(q, k, v, p, st);
+    return launch_one<D, PRE, CAUSAL, OUT, EXTRAS, false>(q, k, v, p, st);
 }
 
 template <int D, bool PRE, bool CAUSAL, int OUT>
-static cudaError_t launch_dump(const CUtensorMap* q, const CUtensorMap* k, const CUtensorMap* v, const AttnParams& p,
-                               bool dump, bool dec, cudaStream_t st) {
-    return dump ? launch_dec<D, PRE, CAUSAL, OUT, true>(q, k, v, p, dec, st)
-                : launch_dec<D, PRE, CAUSAL, OUT, false>(q, k, v, p, dec, st);
+static cudaError_t launch_extras(const CUtensorMap* q, const CUtensorMap* k, const CUtensorMap* v,
+                                 const AttnParams& p, bool extras, bool dec, cudaStream_t st) {
+    return extras ? launch_dec<D, PRE, CAUSAL, OUT, true>(q, k, v, p, dec, st)
+                  : launch_dec<D, PRE, CAUSAL, OUT, false>(q, k, v, p, dec, st);
 }
 
 template <int D, bool PRE, bool CAUSAL>
 static cudaError_t launch_out(const CUtensorMap* q, const CUtensorMap* k, const CUtensorMap* v, const AttnParams& p,
-                              int out, bool dump, bool dec, cudaStream_t st) {
+                              int out, bool extras, bool dec, cudaStream_t st) {
     switch (out) {
-        case 0: return launch_dump<D, PRE, CAUSAL, 0>(q, k, v, p, dump, dec, st);
-        case 1: return launch_dump<D, PRE, CAUSAL, 1>(q, k, v, p, dump, dec, st);
-        default: return launch_dump<D, PRE, CAUSAL, 2>(q, k, v, p, dump, dec, st);
+        case 0: return launch_extras<D, PRE, CAUSAL, 0>(q, k, v, p, extras, dec, st);
+        case 1: return launch_extras<D, PRE, CAUSAL, 1>(q, k, v, p, extras, dec, st);
+        default: return launch_extras<D, PRE, CAUSAL, 2>(q, k, v, p, extras, dec, st);
     }
 }
 
 template <int D>
 static cudaError_t launch_d(const CUtensorMap* q, const CUtensorMap* k, const CUtensorMap* v, const AttnParams& p,
-                            int norm, bool causal, int out, bool dump, bool dec, cudaStream_t st) {
+                            int norm, bool causal, int out, bool extras, bool dec, cudaStream_t st) {
     if (norm == 0)
-        return causal ? launch_out<D, true, true>(q, k, v, p, out, dump, dec, st)
-                      : launch_out<D, true, false>(q, k, v, p, out, dump, dec, st);
-    return causal ? launch_out<D, false, true>(q, k, v, p, out, dump, dec, st)
-                  : launch_out<D, false, false>(q, k, v, p, out, dump, dec, st);
+        return causal ? launch_out<D, true, true>(q, k, v, p, out, extras, dec, st)
+                      : launch_out<D, true, false>(q, k, v, p, out, extras, dec, st);
+    return causal ? launch_out<D, false, true>(q, k, v, p, out, extras, dec, st)
+                  : launch_out<D, false, false>(q, k, v, p, out, extras, dec, st);
 }
 
 cudaError_t launch_attention(const CUtensorMap* tmQ, const CUtensorMap* tmK, const CUtensorMap* tmV,
-                             const AttnParams& p, int D, int norm, bool causal, int out_dtype, bool dump, bool dec,
+                             const AttnParams& p, int D, int norm, bool causal, int out_dtype, bool extras, bool dec,
                              cudaStream_t st) {
     switch (D) {
-        case 64: return launch_d<64>(tmQ, tmK, tmV, p, norm, causal, out_dtype, dump, dec, st);
-        case 128: return launch_d<128>(tmQ, tmK, tmV, p, norm, causal, out_dtype, dump, dec, st);
-        case 256: return launch_d<256>(tmQ, tmK, tmV, p, norm, causal, out_dtype, dump, dec, st);
+        case 64: return launch_d<64>(tmQ, tmK, tmV, p, norm, causal, out_dtype, extras, dec, st);
+        case 128: return launch_d<128>(tmQ, tmK, tmV, p, norm, causal, out_dtype, extras, dec, st);
+        case 256: return launch_d<256>(tmQ, tmK, tmV, p, norm, causal, out_dtype, extras, dec, st);
         default: return cudaErrorInvalidValue;
     }
 }

@@ -343,6 +343,17 @@ __device__ __forceinline__ float e4m3_to_f32(uint32_t code) {
     return __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu)));
 }
 
+// Sum of the eight non-negative E2M1 values packed in 32 bits (the sign bit of
+// each nibble is ignored: probability codes are never negative). Twice the
+// magnitude of code m = 0..7 is 0, 1, 2, 3, 4, 6, 8, 12: hex digit m of
+// 0xC8643210. The integer sum is exact; the result is half of it.
+__device__ __forceinline__ float e2m1x8_sum(uint32_t w) {
+    uint32_t twice = 0;
+#pragma unroll
+    for (int n = 0; n < 8; ++n) twice += (0xC8643210u >> (4u * ((w >> (4 * n)) & 7u))) & 0xFu;
+    return 0.5f * (float)twice;
+}
+
 __device__ __forceinline__ float ex2_approx(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));

@@ -7,21 +7,48 @@
 
 namespace hifa4 {
 
-// One pass over Q (optional), K and V: smooth, quantize, write codes and
-// MMA-ready scales.
+// One pass over Q (optional), K and V: quantize, write codes and MMA-ready
+// scales. Before quantization, in order: RoPE (rope_cos non-null), the Smooth-QK
+// multiply (s / s_inv non-null), the Q-Mean subtraction on Q (q_mean
+// non-null; the K pass then writes the score bias s_bias). The K and V input
+// tokens [0, nkv_in) land at tokens [kv_start, kv_start + nkv_in) of an output
+// of nkv tokens (a KV-cache append; the plain pass has nkv_in = nkv, kv_start = 0).
 struct QuantArgs {
     bool bf16;
     int D, G, hkv, nq, nkv, tiles_q;
+    int nkv_in, kv_start;
     long long n_groups;           // B * Hkv
     const void* q;                // null: K and V only
     const void* k;
     const void* v;
     const float* s;
     const float* s_inv;
+    const float* rope_cos;        // [n_pos, D/2] or null
+    const float* rope_sin;
+    const int* q_pos;             // [nq]
+    const int* k_pos;             // [nkv_in]
+    int n_pos;
+    const float* q_mean;          // [B*Hq, D] or null
+    float* s_bias;                // [B*Hq, nkv]
     uint8_t *qc, *qs, *kc, *ks, *vtc, *vts;
 };
 
 cudaError_t launch_quantize_qkv(const QuantArgs& a, cudaStream_t st);
+
+// Q-Mean: mean [B*Hq, D] of the pre-quantization Q (RoPE, smoothing as above).
+struct QMeanArgs {
+    bool bf16;
+    int B, Hq, Hkv, Nq, D;
+    const void* q;
+    const float* s;
+    const float* rope_cos;
+    const float* rope_sin;
+    const int* q_pos;
+    int n_pos;
+    float* mean;
+};
+
+cudaError_t launch_q_mean(const QMeanArgs& a, cudaStream_t st);
 
 cudaError_t launch_calibrate(bool bf16, const void* q, const void* k, int B, int Hq, int Hkv, int N, int D, float alpha,
                              float* s, float* s_inv, cudaStream_t st);
@@ -32,8 +59,11 @@ struct AttnParams {
     const uint8_t* vts;      // ... of V^T
     void* o;                 // [B,Hq,Nq,D] output
     float* lse;              // [B,Hq,Nq] or null
-    uint8_t* p_codes;        // P_hat dump (debug variant only)
-    uint8_t* p_sf;
+    // optional outputs and inputs of the extras variant (each may be null)
+    const float* s_bias;     // [B*Hq, Nkv] added to the scores of head (b, h)
+    uint8_t* p_codes;        // P_hat dump [B*Hq*Nq, Nkv/2]
+    uint8_t* p_sf;           // ... and its scales [B*Hq*Nq, Nkv/16]
+    float2* tile_sums;       // (sum P_hat, sum P) per (row, kv tile) [B*Hq*Nq, Nkv/128]
     uint32_t* status;        // workspace status word
     int B, Hq, Hkv, Nq, Nkv, G;
     int Tq;                  // 128-row tiles per (b, kv head) group
@@ -46,11 +76,15 @@ struct AttnParams {
 };
 
 // D in {64,128,256}; norm 0 = P-Reordering, 1 = high-precision l;
-// out_dtype 0 = f16, 1 = bf16, 2 = f32; dec: split-kv decode mode (D <= 128,
+// out_dtype 0 = f16, 1 = bf16, 2 = f32; extras: the variant that reads s_bias
+// and writes p_codes / p_sf / tile_sums where they are non-null; dec: split-kv decode mode (D <= 128,
 // G*Nq <= 64, at least 4 kv tiles; one CTA per group).
 cudaError_t launch_attention(const CUtensorMap* tmQ, const CUtensorMap* tmK, const CUtensorMap* tmV,
-                             const AttnParams& p, int D, int norm, bool causal, int out_dtype, bool dump, bool dec,
+                             const AttnParams& p, int D, int norm, bool causal, int out_dtype, bool extras, bool dec,
                              cudaStream_t st);
+
+// Per-tile epsilon-bar from the attention kernel's tile sums.
+cudaError_t launch_tile_stats(const float2* sums, int BH, int Nq, int T, float* eps_bar, cudaStream_t st);
 
 // Number of contiguous kv ranges the decode mode cuts the keys into.
 constexpr int kDecodeSplits = 4;

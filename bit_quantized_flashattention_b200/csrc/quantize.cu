@@ -59,28 +59,98 @@ __device__ __forceinline__ uint32_t quant_block16_lut(const float (&x)[16], cons
     return sf;
 }
 
+// ------------------------------------------------- before quantization
+
+// RoPE tables of one 8-channel chunk: cos and sin of the chunk's channel pairs
+// at the row's position (clamped to the table).
+struct RopeChunk {
+    float4 c0, c1, s0, s1;
+};
+
+template <int D>
+__device__ __forceinline__ RopeChunk load_rope(const float* cos_t, const float* sin_t, const int* pos, unsigned tok,
+                                               int n_pos, unsigned chunk) {
+    constexpr unsigned HALF = D / 16;                     // chunks per half row
+    int ps = __ldg(pos + tok);
+    ps = ps < 0 ? 0 : (ps >= n_pos ? n_pos - 1 : ps);
+    const size_t off = (size_t)ps * (D / 2) + (chunk % HALF) * 8;
+    const float4* c4 = reinterpret_cast<const float4*>(cos_t + off);
+    const float4* s4 = reinterpret_cast<const float4*>(sin_t + off);
+    return RopeChunk{__ldg(c4), __ldg(c4 + 1), __ldg(s4), __ldg(s4 + 1)};
+}
+
+// The rotation of one chunk, rotate-half pairing: channel d < D/2 pairs with
+// d + D/2, which sits in chunk c ^ (D/16) of the same row (a neighbouring lane
+// group: the row's D/8 chunks are consecutive lanes). Each product and sum is
+// rounded on its own (no fused multiply-add):
+//   first half   x <- RN(RN(x*cos) - RN(x_pair*sin))
+//   second half  x <- RN(RN(x*cos) + RN(x_pair*sin))
+// Every lane of the warp calls this (it shuffles).
+template <typename T, int D>
+__device__ __forceinline__ void rope_chunk(const uint4& raw, unsigned chunk, const RopeChunk& t, float (&v)[8]) {
+    constexpr unsigned HALF = D / 16;
+    uint4 pr;
+    pr.x = __shfl_xor_sync(0xFFFFFFFFu, raw.x, HALF);
+    pr.y = __shfl_xor_sync(0xFFFFFFFFu, raw.y, HALF);
+    pr.z = __shfl_xor_sync(0xFFFFFFFFu, raw.z, HALF);
+    pr.w = __shfl_xor_sync(0xFFFFFFFFu, raw.w, HALF);
+    float w[8];
+    unpack8<T>(pr, w);
+    const float cs[8] = {t.c0.x, t.c0.y, t.c0.z, t.c0.w, t.c1.x, t.c1.y, t.c1.z, t.c1.w};
+    const float sn[8] = {t.s0.x, t.s0.y, t.s0.z, t.s0.w, t.s1.x, t.s1.y, t.s1.z, t.s1.w};
+    if (chunk < HALF) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[i] = __fsub_rn(__fmul_rn(v[i], cs[i]), __fmul_rn(w[i], sn[i]));
+    } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[i] = __fadd_rn(__fmul_rn(v[i], cs[i]), __fmul_rn(w[i], sn[i]));
+    }
+}
+
+__device__ __forceinline__ void load8(const float* p, float (&f)[8]) {
+    const float4 a = __ldg(reinterpret_cast<const float4*>(p)), b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+    f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w;
+    f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+}
+
 // ---------------------------------------------------------------- Q and K
 
-// One row-quantization job (Q or K, quantized along D). A group is the G*N
-// consecutive input rows that share a kv head (G = q heads per kv head for Q,
-// 1 for K), padded to whole 128-row tiles; padding rows only receive zero
-// scale words.
+// One row-quantization job (Q or K, quantized along D). A group holds the rows
+// that share a kv head: for Q the G*Nq rows of its q heads stacked head after
+// head (row p = head_in_group * n_tok + token), padded to whole 128-row tiles
+// whose padding rows only receive zero scale words; for K the group's tokens.
+// K rows may land at an offset of a larger output (a KV-cache append).
 struct RowJob {
     const void* x;
     const float* scale;       // smoothing factors [Hkv, D] or null
+    const float* rope_cos;    // RoPE tables [n_pos, D/2] (used by the RoPE variant)
+    const float* rope_sin;
+    const int* pos;           // position of each input token [n_tok]
+    int n_pos;
+    const float* mean;        // Q-Mean: subtract row (group*G + head_in_group) of [B*Hq, D], or null
+    const float* bias_mean;   // Q-Mean on K rows: means [B*Hq, D] the score bias is taken from, or null
+    float* bias;              // [B*Hq, rows_out] score bias output (with bias_mean)
     uint8_t* codes;
     uint8_t* sfs;
-    unsigned rows_per_group;
-    unsigned tiles_per_group;
+    unsigned n_tok;           // tokens per head in the input
+    unsigned rows_in;         // input rows per group
+    unsigned rows_out;        // output rows per group
+    unsigned row0;            // output row of input row 0
+    unsigned tiles_out;       // 128-row scale tiles per group in the output
+    unsigned padded;          // rows [0, padded) are visited; [rows_in, padded) get zero scale words
     unsigned hkv;
-    unsigned blocks_per_group;  // CTAs sharing one group's rows
+    unsigned G;               // q heads per kv head
+    unsigned blocks_per_group;
 };
 
 struct VJob {
     const void* v;
     uint8_t* vtc;
     uint8_t* vts;
-    int nkv;
+    int n_in;                 // input tokens per group
+    int nkv;                  // output tokens per group
+    int start;                // output token of input token 0 (a multiple of 16)
+    unsigned half0;           // first 64-token half of the output the job touches
     unsigned warps_per_group;
 };
 
@@ -90,8 +160,11 @@ struct VJob {
 // lane's 8 smoothing factors stay in registers. The two halves of a
 // 16-element block sit in neighbouring lanes (one shuffle for the maximum),
 // and the 4 scale bytes of a 64-element K step are gathered by shuffles into
-// one 32-bit word of the MMA-ready atom.
-template <typename T, int D>
+// one 32-bit word of the MMA-ready atom. Before quantization, in order: RoPE
+// (ROPE variant), the smoothing multiply, the Q-Mean subtraction; on K rows
+// with bias_mean the Q-Mean score bias mean . K' of every head of the group is
+// reduced across the row's lanes from the same pre-quantization values.
+template <typename T, int D, bool ROPE>
 __device__ __forceinline__ void quantize_rows_cta(const RowJob& jb, unsigned cta, const float* lut) {
     constexpr unsigned CPR = D / 8;                        // chunks per row
     constexpr unsigned RPB = 256 / CPR;                    // rows per CTA step
@@ -100,40 +173,58 @@ __device__ __forceinline__ void quantize_rows_cta(const RowJob& jb, unsigned cta
     const unsigned grp = cta / jb.blocks_per_group;
     const unsigned part = cta % jb.blocks_per_group;
     const unsigned c = threadIdx.x % CPR;
-    const unsigned padded = jb.tiles_per_group * 128;
-    const unsigned steps = (padded + RPB - 1) / RPB;
+    const unsigned steps = (jb.padded + RPB - 1) / RPB;
     const unsigned s0 = (unsigned)(((unsigned long long)steps * part) / jb.blocks_per_group);
     const unsigned s1 = (unsigned)(((unsigned long long)steps * (part + 1)) / jb.blocks_per_group);
     float sc[8];
-    if (jb.scale != nullptr) {
-        const float4* s4 = reinterpret_cast<const float4*>(jb.scale + (size_t)(grp % jb.hkv) * D + c * 8);
-        const float4 a = __ldg(s4), b = __ldg(s4 + 1);
-        sc[0] = a.x; sc[1] = a.y; sc[2] = a.z; sc[3] = a.w;
-        sc[4] = b.x; sc[5] = b.y; sc[6] = b.z; sc[7] = b.w;
-    }
-    const T* xg = static_cast<const T*>(jb.x) + (size_t)grp * jb.rows_per_group * D;
-    uint8_t* cg = jb.codes + (size_t)grp * jb.rows_per_group * (D / 2);
-    uint8_t* sg = jb.sfs + (size_t)grp * jb.tiles_per_group * KS * 512;
+    if (jb.scale != nullptr) load8(jb.scale + (size_t)(grp % jb.hkv) * D + c * 8, sc);
+    const T* xg = static_cast<const T*>(jb.x) + (size_t)grp * jb.rows_in * D;
+    uint8_t* cg = jb.codes + ((size_t)grp * jb.rows_out + jb.row0) * (D / 2);
+    uint8_t* sg = jb.sfs + (size_t)grp * jb.tiles_out * KS * 512;
     const unsigned r_in = threadIdx.x / CPR;
     for (unsigned st = s0; st < s1; st += UNROLL) {
         uint4 raw[UNROLL];
+        RopeChunk rc[ROPE ? UNROLL : 1];
 #pragma unroll
         for (unsigned u = 0; u < UNROLL; ++u) {
             const unsigned pp = (st + u) * RPB + r_in;
-            raw[u] = (st + u < s1 && pp < jb.rows_per_group)
-                         ? *reinterpret_cast<const uint4*>(xg + (size_t)pp * D + c * 8)
-                         : make_uint4(0u, 0u, 0u, 0u);
+            const bool real = st + u < s1 && pp < jb.rows_in;
+            raw[u] = real ? *reinterpret_cast<const uint4*>(xg + (size_t)pp * D + c * 8) : make_uint4(0u, 0u, 0u, 0u);
+            if constexpr (ROPE)
+                rc[u] = load_rope<D>(jb.rope_cos, jb.rope_sin, jb.pos, real ? pp % jb.n_tok : 0u, jb.n_pos, c);
         }
 #pragma unroll
         for (unsigned u = 0; u < UNROLL; ++u) {
             const unsigned p = (st + u) * RPB + r_in;
             const bool in_range = st + u < s1;             // warp-uniform
-            const bool real = in_range && p < jb.rows_per_group;
+            const bool real = in_range && p < jb.rows_in;
             float v[8];
             unpack8<T>(raw[u], v);
+            if constexpr (ROPE) rope_chunk<T, D>(raw[u], c, rc[u], v);
             if (jb.scale != nullptr) {
 #pragma unroll
                 for (int i = 0; i < 8; ++i) v[i] = __fmul_rn(v[i], sc[i]);
+            }
+            if (jb.mean != nullptr && real) {
+                float m[8];
+                load8(jb.mean + ((size_t)grp * jb.G + p / jb.n_tok) * D + c * 8, m);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) v[i] = __fsub_rn(v[i], m[i]);
+            }
+            if (jb.bias_mean != nullptr) {
+                // score bias of this key for every q head of the group
+                for (unsigned hl = 0; hl < jb.G; ++hl) {
+                    float acc = 0.0f;
+                    if (real) {
+                        float m[8];
+                        load8(jb.bias_mean + ((size_t)grp * jb.G + hl) * D + c * 8, m);
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) acc = __fmaf_rn(m[i], v[i], acc);
+                    }
+#pragma unroll
+                    for (unsigned o = CPR / 2; o >= 1; o >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, o);
+                    if (real && c == 0) jb.bias[((size_t)grp * jb.G + hl) * jb.rows_out + jb.row0 + p] = acc;
+                }
             }
             float amax = 0.0f;
 #pragma unroll
@@ -149,8 +240,9 @@ __device__ __forceinline__ void quantize_rows_cta(const RowJob& jb, unsigned cta
             uint32_t word = ((c & 1u) == 0u) ? (sf << (8u * ((c >> 1) & 3u))) : 0u;
             word |= __shfl_xor_sync(0xFFFFFFFFu, word, 2);
             word |= __shfl_xor_sync(0xFFFFFFFFu, word, 4);
-            if (in_range && p < padded && (c & 7u) == 0u)
-                *reinterpret_cast<uint32_t*>(sg + ((size_t)(p >> 7) * KS + c / 8) * 512 + atom_offset(p & 127u)) =
+            const unsigned q = jb.row0 + p;                // output row
+            if (in_range && p < jb.padded && (c & 7u) == 0u)
+                *reinterpret_cast<uint32_t*>(sg + ((size_t)(q >> 7) * KS + c / 8) * 512 + atom_offset(q & 127u)) =
                     real ? word : 0u;
         }
     }
@@ -160,11 +252,13 @@ __device__ __forceinline__ void quantize_rows_cta(const RowJob& jb, unsigned cta
 
 // V quantized along tokens, written transposed and tiled (each 128-token tile
 // of V^T is one contiguous D x 64-byte block). A warp covers 32 channels x 64
-// tokens of one group; lane (cc, tb) owns 4 channels (cc = 0..7) x one 16-token
-// block (tb = 0..3): it reads 16 rows of 8 bytes (each load instruction reads 4
-// rows of 64 contiguous bytes), quantizes one block per channel and writes 8
-// code bytes per channel; the 4 scale bytes of a channel for the 64-token half
-// come from the lanes tb = 0..3 and are gathered by shuffles. For D = 64 one
+// output tokens of one group; lane (cc, tb) owns 4 channels (cc = 0..7) x one
+// 16-token block (tb = 0..3): it reads 16 rows of 8 bytes (each load
+// instruction reads 4 rows of 64 contiguous bytes), quantizes one block per
+// channel and writes 8 code bytes per channel. The 4 scale bytes of a channel
+// for the 64-token half are gathered by shuffles into one word when the job
+// covers the whole half; a job that covers part of it (an append) writes its
+// blocks' scale bytes one by one and leaves the others alone. For D = 64 one
 // warp per half also fills the padding rows of the scale atoms (row 64 = 1.0
 // for the normalizer column of P-Reordering, the rest 0).
 template <typename T, int D>
@@ -176,14 +270,21 @@ __device__ __forceinline__ void quantize_v_warp(const VJob& jb, unsigned gw_all,
     const unsigned gw = gw_all % jb.warps_per_group;
     const int nkv = jb.nkv;
     const unsigned cw = gw % CWARPS;
-    const unsigned hh = gw / CWARPS;                       // 64-token half over the sequence
+    const unsigned hh = jb.half0 + gw / CWARPS;            // 64-token half of the output
     const unsigned cc = lane >> 2, tb = lane & 3u;
     const unsigned d0 = cw * 32 + cc * 4;
-    const unsigned tok0 = hh * 64 + tb * 16;
-    const T* src = static_cast<const T*>(jb.v) + ((size_t)grp * nkv + tok0) * D + d0;
+    const int tok0 = (int)(hh * 64 + tb * 16);             // output token of this lane's block
+    const bool active = tok0 >= jb.start && tok0 < jb.start + jb.n_in;
+    const bool whole = (int)(hh * 64) >= jb.start && (int)(hh * 64 + 64) <= jb.start + jb.n_in;   // warp-uniform
     uint2 raw[16];
+    if (active) {
+        const T* src = static_cast<const T*>(jb.v) + ((size_t)grp * jb.n_in + (tok0 - jb.start)) * D + d0;
 #pragma unroll
-    for (int i = 0; i < 16; ++i) raw[i] = *reinterpret_cast<const uint2*>(src + (size_t)i * D);
+        for (int i = 0; i < 16; ++i) raw[i] = *reinterpret_cast<const uint2*>(src + (size_t)i * D);
+    } else {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) raw[i] = make_uint2(0u, 0u);
+    }
     const unsigned j = hh / 2, half = hh % 2;
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
@@ -194,14 +295,17 @@ __device__ __forceinline__ void quantize_v_warp(const VJob& jb, unsigned gw_all,
         const uint32_t sf = quant_block16_lut(x, lut, lo, hi);
         const unsigned d = d0 + k;
         // tiled V^T codes: the 64 bytes of channel d for kv tile tok0/128
-        *reinterpret_cast<uint2*>(jb.vtc + (((size_t)grp * (nkv / 128) + tok0 / 128) * D + d) * 64 + (tok0 % 128) / 2) =
-            make_uint2(lo, hi);
-        uint32_t word = sf << (8u * tb);
-        word |= __shfl_xor_sync(0xFFFFFFFFu, word, 1);
-        word |= __shfl_xor_sync(0xFFFFFFFFu, word, 2);
-        if (tb == 0) {
-            const size_t atom = (((size_t)grp * (nkv / 128) + j) * NRB + (d >> 7)) * 2 + half;
-            *reinterpret_cast<uint32_t*>(jb.vts + atom * 512 + atom_offset(d & 127u)) = word;
+        if (active)
+            *reinterpret_cast<uint2*>(jb.vtc + (((size_t)grp * (nkv / 128) + tok0 / 128) * D + d) * 64 +
+                                      (tok0 % 128) / 2) = make_uint2(lo, hi);
+        const size_t atom = (((size_t)grp * (nkv / 128) + j) * NRB + (d >> 7)) * 2 + half;
+        if (whole) {
+            uint32_t word = sf << (8u * tb);
+            word |= __shfl_xor_sync(0xFFFFFFFFu, word, 1);
+            word |= __shfl_xor_sync(0xFFFFFFFFu, word, 2);
+            if (tb == 0) *reinterpret_cast<uint32_t*>(jb.vts + atom * 512 + atom_offset(d & 127u)) = word;
+        } else if (active) {
+            jb.vts[atom * 512 + atom_offset(d & 127u) + tb] = (uint8_t)sf;
         }
     }
     if constexpr (D == 64) {
@@ -215,7 +319,7 @@ __device__ __forceinline__ void quantize_v_warp(const VJob& jb, unsigned gw_all,
 
 // One launch for the whole pass: CTAs [0, nq) quantize Q rows, [nq, nq + nk)
 // K rows, the rest V (8 warps per CTA).
-template <typename T, int D>
+template <typename T, int D, bool ROPE>
 __global__ void __launch_bounds__(256) quantize_qkv_kernel(RowJob q, RowJob k, VJob v, unsigned nq, unsigned nk,
                                                            unsigned v_warps) {
     __shared__ float lut[128];
@@ -225,12 +329,72 @@ __global__ void __launch_bounds__(256) quantize_qkv_kernel(RowJob q, RowJob k, V
     build_rcp_lut(lut);
     const unsigned b = blockIdx.x;
     if (b < nq) {
-        quantize_rows_cta<T, D>(q, b, lut);
+        quantize_rows_cta<T, D, ROPE>(q, b, lut);
     } else if (b < nq + nk) {
-        quantize_rows_cta<T, D>(k, b - nq, lut);
+        quantize_rows_cta<T, D, ROPE>(k, b - nq, lut);
     } else {
         const unsigned gw = (b - nq - nk) * 8 + (threadIdx.x >> 5);
         if (gw < v_warps) quantize_v_warp<T, D>(v, gw, lut);
+    }
+}
+
+// ----------------------------------------------------------------- Q-Mean
+
+// Per-(batch, head, channel) mean of the pre-quantization Q (after RoPE and
+// smoothing) over the head's Nq tokens: the sum is accumulated in fp64, then
+// divided in fp64 and rounded once to fp32. One CTA per (b, h); lane chunk
+// c = tid % (D/8) of token lane tid / (D/8); token lanes are reduced through
+// shared memory in a fixed order.
+struct QMeanJob {
+    const void* q;
+    const float* scale;       // smoothing factors [Hkv, D] or null
+    const float* rope_cos;
+    const float* rope_sin;
+    const int* pos;
+    int n_pos;
+    float* mean;              // [B*Hq, D]
+    int Hq, G, Hkv, Nq;
+};
+
+template <typename T, int D, bool ROPE>
+__global__ void __launch_bounds__(256) q_mean_kernel(QMeanJob jb) {
+    constexpr unsigned CPR = D / 8, TL = 256 / CPR;
+    __shared__ double red[TL][D];
+    const unsigned bh = blockIdx.x;
+    const unsigned c = threadIdx.x % CPR, tl = threadIdx.x / CPR;
+    const unsigned g = (bh % (unsigned)jb.Hq) / (unsigned)jb.G;
+    float sc[8];
+    if (jb.scale != nullptr) load8(jb.scale + (size_t)g * D + c * 8, sc);
+    const T* xb = static_cast<const T*>(jb.q) + (size_t)bh * jb.Nq * D;
+    double acc[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i] = 0.0;
+    for (unsigned base = 0; base < (unsigned)jb.Nq; base += TL) {      // warp-uniform trip count
+        const unsigned i = base + tl;
+        const bool real = i < (unsigned)jb.Nq;
+        const uint4 raw = real ? *reinterpret_cast<const uint4*>(xb + (size_t)i * D + c * 8) : make_uint4(0u, 0u, 0u, 0u);
+        float v[8];
+        unpack8<T>(raw, v);
+        if constexpr (ROPE) {
+            const RopeChunk rc = load_rope<D>(jb.rope_cos, jb.rope_sin, jb.pos, real ? i : 0u, jb.n_pos, c);
+            rope_chunk<T, D>(raw, c, rc, v);
+        }
+        if (jb.scale != nullptr) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) v[e] = __fmul_rn(v[e], sc[e]);
+        }
+        if (real) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) acc[e] = __dadd_rn(acc[e], (double)v[e]);
+        }
+    }
+#pragma unroll
+    for (int e = 0; e < 8; ++e) red[tl][c * 8 + e] = acc[e];
+    __syncthreads();
+    for (unsigned d = threadIdx.x; d < (unsigned)D; d += 256) {
+        double sum = 0.0;
+        for (unsigned t = 0; t < TL; ++t) sum = __dadd_rn(sum, red[t][d]);
+        jb.mean[(size_t)bh * D + d] = __double2float_rn(__ddiv_rn(sum, (double)jb.Nq));
     }
 }
 
@@ -277,13 +441,6 @@ __global__ void calib_finalize_kernel(float* __restrict__ s, float* __restrict__
 
 template <typename T, int D>
 static cudaError_t launch_qkv_t(const QuantArgs& a, cudaStream_t st) {
-    int dev = 0, sms = 148, occ = 1;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, quantize_qkv_kernel<T, D>, 256, 0) != cudaSuccess || occ < 1)
-        occ = 1;
-    (void)occ;
-    (void)sms;
     const long long n_grp = a.n_groups;
     // small CTAs (at most 8 row steps of 256/(D/8) rows each): many CTAs per SM
     // overlap one CTA's loads with another's arithmetic
@@ -293,21 +450,64 @@ static cudaError_t launch_qkv_t(const QuantArgs& a, cudaStream_t st) {
         const long long steps = (padded_rows + rows_per_step - 1) / rows_per_step;
         return (steps + 7) / 8;
     };
-    const long long rows_q = a.q != nullptr ? (long long)a.tiles_q * 128 : 0;
-    const long long rows_k = a.nkv;
-    const long long v_warps = n_grp * (a.nkv / 64) * (D / 32);
+    const bool rope = a.rope_cos != nullptr;
+    RowJob jq{};
+    jq.x = a.q;
+    jq.scale = a.s;
+    jq.rope_cos = a.rope_cos;
+    jq.rope_sin = a.rope_sin;
+    jq.pos = a.q_pos;
+    jq.n_pos = a.n_pos;
+    jq.mean = a.q_mean;
+    jq.codes = a.qc;
+    jq.sfs = a.qs;
+    jq.n_tok = (unsigned)a.nq;
+    jq.rows_in = jq.rows_out = (unsigned)(a.G * a.nq);
+    jq.tiles_out = (unsigned)a.tiles_q;
+    jq.padded = (unsigned)a.tiles_q * 128u;
+    jq.hkv = (unsigned)a.hkv;
+    jq.G = (unsigned)a.G;
+    jq.blocks_per_group = (unsigned)per_group(a.q != nullptr ? jq.padded : 0);
+    RowJob jk{};
+    jk.x = a.k;
+    jk.scale = a.s_inv;
+    jk.rope_cos = a.rope_cos;
+    jk.rope_sin = a.rope_sin;
+    jk.pos = a.k_pos;
+    jk.n_pos = a.n_pos;
+    jk.bias_mean = a.q_mean;
+    jk.bias = a.s_bias;
+    jk.codes = a.kc;
+    jk.sfs = a.ks;
+    jk.n_tok = jk.rows_in = jk.padded = (unsigned)a.nkv_in;
+    jk.rows_out = (unsigned)a.nkv;
+    jk.row0 = (unsigned)a.kv_start;
+    jk.tiles_out = (unsigned)(a.nkv / 128);
+    jk.hkv = (unsigned)a.hkv;
+    jk.G = (unsigned)a.G;
+    jk.blocks_per_group = (unsigned)per_group(jk.padded);
+    VJob jv{};
+    jv.v = a.v;
+    jv.vtc = a.vtc;
+    jv.vts = a.vts;
+    jv.n_in = a.nkv_in;
+    jv.nkv = a.nkv;
+    jv.start = a.kv_start;
+    jv.half0 = (unsigned)(a.kv_start / 64);
+    const unsigned halves = (unsigned)((a.kv_start + a.nkv_in - 1) / 64 - a.kv_start / 64 + 1);
+    jv.warps_per_group = halves * (D / 32);
+    const long long v_warps = n_grp * jv.warps_per_group;
     const long long v_ctas = (v_warps + 7) / 8;
-    RowJob jq{a.q, a.s, a.qc, a.qs, (unsigned)(a.G * a.nq), (unsigned)a.tiles_q, (unsigned)a.hkv,
-              (unsigned)per_group(rows_q)};
-    RowJob jk{a.k, a.s_inv, a.kc, a.ks, (unsigned)a.nkv, (unsigned)(a.nkv / 128), (unsigned)a.hkv,
-              (unsigned)per_group(rows_k)};
-    VJob jv{a.v, a.vtc, a.vts, a.nkv, (unsigned)((a.nkv / 64) * (D / 32))};
     const long long nq = a.q != nullptr ? n_grp * jq.blocks_per_group : 0;
     const long long nk = n_grp * jk.blocks_per_group;
     const long long total = nq + nk + v_ctas;
     if (total > 0x7FFFFFFFLL) return cudaErrorInvalidConfiguration;
-    quantize_qkv_kernel<T, D><<<(unsigned)total, 256, 0, st>>>(jq, jk, jv, (unsigned)nq, (unsigned)nk,
-                                                                (unsigned)v_warps);
+    if (rope)
+        quantize_qkv_kernel<T, D, true><<<(unsigned)total, 256, 0, st>>>(jq, jk, jv, (unsigned)nq, (unsigned)nk,
+                                                                          (unsigned)v_warps);
+    else
+        quantize_qkv_kernel<T, D, false><<<(unsigned)total, 256, 0, st>>>(jq, jk, jv, (unsigned)nq, (unsigned)nk,
+                                                                           (unsigned)v_warps);
     return cudaGetLastError();
 }
 
@@ -316,6 +516,27 @@ cudaError_t launch_quantize_qkv(const QuantArgs& a, cudaStream_t st) {
         case 64: return a.bf16 ? launch_qkv_t<__nv_bfloat16, 64>(a, st) : launch_qkv_t<__half, 64>(a, st);
         case 128: return a.bf16 ? launch_qkv_t<__nv_bfloat16, 128>(a, st) : launch_qkv_t<__half, 128>(a, st);
         case 256: return a.bf16 ? launch_qkv_t<__nv_bfloat16, 256>(a, st) : launch_qkv_t<__half, 256>(a, st);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+template <typename T, int D>
+static cudaError_t launch_q_mean_t(const QMeanArgs& a, cudaStream_t st) {
+    QMeanJob jb{a.q, a.s, a.rope_cos, a.rope_sin, a.q_pos, a.n_pos, a.mean, a.Hq, a.Hq / a.Hkv, a.Hkv, a.Nq};
+    const long long n = (long long)a.B * a.Hq;
+    if (n > 0x7FFFFFFFLL) return cudaErrorInvalidConfiguration;
+    if (a.rope_cos != nullptr)
+        q_mean_kernel<T, D, true><<<(unsigned)n, 256, 0, st>>>(jb);
+    else
+        q_mean_kernel<T, D, false><<<(unsigned)n, 256, 0, st>>>(jb);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_q_mean(const QMeanArgs& a, cudaStream_t st) {
+    switch (a.D) {
+        case 64: return a.bf16 ? launch_q_mean_t<__nv_bfloat16, 64>(a, st) : launch_q_mean_t<__half, 64>(a, st);
+        case 128: return a.bf16 ? launch_q_mean_t<__nv_bfloat16, 128>(a, st) : launch_q_mean_t<__half, 128>(a, st);
+        case 256: return a.bf16 ? launch_q_mean_t<__nv_bfloat16, 256>(a, st) : launch_q_mean_t<__half, 256>(a, st);
         default: return cudaErrorInvalidValue;
     }
 }

@@ -150,6 +150,66 @@ hifa4_status hifa4_quantize_kv(const void* k, const void* v, hifa4_dtype dtype,
                                int B, int Hkv, int Nkv, int D, const float* s_inv,
                                const hifa4_packed* out, hifa4_stream_t stream);
 
+/* The steps before quantization, each optional, applied in this order to the
+ * pre-quantization fp32 values (no rounding to the storage type between them):
+ *  1. RoPE (rope_cos != NULL), rotate-half pairing: channel d < D/2 pairs with
+ *     d + D/2; with c = rope_cos[pos, d], s = rope_sin[pos, d] (tables fp32
+ *     [n_pos, D/2]): x[d] <- RN(RN(x[d]*c) - RN(x[d+D/2]*s)),
+ *     x[d+D/2] <- RN(RN(x[d+D/2]*c) + RN(x[d]*s)), each product and sum rounded
+ *     to fp32 (no fused multiply-add). Applied to Q and K, never to V. The
+ *     abstract applies Smooth-QK "after RoPE"; fusing the two removes a pass.
+ *  2. Smooth-QK: x <- RN(x*s[g]) for Q, RN(x*s_inv[g]) for K (both NULL: off).
+ *  3. Q-Mean auxiliary (q_mean != NULL; the abstract adopts it with
+ *     P-Reordering on models where Smooth-QK is disabled, without defining it;
+ *     this library reads it as Q smoothing by the mean): Q <- RN(Q - q_mean[b,h])
+ *     before quantization, and the rank-one score term that subtraction
+ *     removes, s_bias[b,h,j] = sum_d q_mean[b,h,d] * K'[b,g,j,d], is written
+ *     from the keys K' as they enter quantization (after steps 1-2, before
+ *     4-bit rounding), accumulated in fp32. hifa4_attention_fwd_ex adds s_bias
+ *     to the scores.
+ * Positions: query token i of every batch and head sits at q_pos[i] (int32
+ * [Nq]); key token j at k_pos[j] (int32 [Nkv], or [n_new] for an append).
+ * Positions outside [0, n_pos) are clamped into it. */
+typedef struct {
+    const float* s;          /* Smooth-QK factors [Hkv, D] or NULL */
+    const float* s_inv;      /* their reciprocals [Hkv, D]; NULL exactly when s is NULL */
+    const float* rope_cos;   /* [n_pos, D/2] fp32, or NULL (then rope_sin is NULL too) */
+    const float* rope_sin;
+    const int32_t* q_pos;    /* [Nq] */
+    const int32_t* k_pos;    /* [Nkv] or [n_new] */
+    int n_pos;
+    const float* q_mean;     /* Q-Mean auxiliary [B,Hq,D] (see hifa4_q_mean) or NULL */
+    float* s_bias;           /* [B,Hq,Nkv] fp32 output, required exactly when q_mean is set */
+} hifa4_prequant;
+
+/* hifa4_quantize_qkv with the steps of hifa4_prequant (pre may be NULL: none).
+ * Table and bias pointers must be 16-byte aligned, positions 4-byte aligned. */
+hifa4_status hifa4_quantize_qkv_ex(const void* q, const void* k, const void* v, hifa4_dtype dtype,
+                                   int B, int Hq, int Hkv, int Nq, int Nkv, int D,
+                                   const hifa4_prequant* pre, const hifa4_packed* out, hifa4_stream_t stream);
+
+/* Q-Mean: q_mean[b,h,d] (fp32 [B,Hq,D]) = mean over the Nq tokens of Q after
+ * RoPE and smoothing (pre: uses s, rope_cos, rope_sin, q_pos, n_pos; may be
+ * NULL), summed in fp64 and rounded once to fp32 after an fp64 division. The
+ * order of the fp64 additions is unspecified: results can differ from another
+ * fp64 summation only when the exact mean lies within about 1e-16 (relative)
+ * of an fp32 rounding boundary. */
+hifa4_status hifa4_q_mean(const void* q, hifa4_dtype dtype, int B, int Hq, int Hkv, int Nq, int D,
+                          const hifa4_prequant* pre, float* q_mean, hifa4_stream_t stream);
+
+/* KV-cache append: quantize n_new new K and V tokens ([B, Hkv, n_new, D]) into
+ * token slots [start, start + n_new) of a packed cache that holds
+ * cache_tokens tokens (cache->kc, ks, vtc, vts sized by hifa4_packed_bytes
+ * with Nkv = cache_tokens; qc / qs ignored). Codes and scales equal those of
+ * quantizing the whole cache at once; slots outside the range are untouched.
+ * Needs start % 16 == 0 and n_new % 16 == 0 (a V scale covers 16 tokens;
+ * decoding keeps the last, partial 16 tokens unquantized or re-appends them),
+ * start + n_new <= cache_tokens, cache_tokens % 128 == 0. pre: s_inv and RoPE
+ * (k_pos has n_new entries) may be set; q_mean must be NULL. */
+hifa4_status hifa4_append_kv(const void* k, const void* v, hifa4_dtype dtype, int B, int Hkv, int n_new, int D,
+                             const hifa4_prequant* pre, const hifa4_packed* cache, int cache_tokens, int start,
+                             hifa4_stream_t stream);
+
 /* 4-bit attention forward (HiFA4 abstract). For each query row, one pass over
  * 128-key tiles in ascending order: S = Q_hat K_hat^T (block-scaled FP4 MMA,
  * fp32 accumulate), running max m updated every tile, c = RN(sm_scale*log2 e),
@@ -180,6 +240,41 @@ hifa4_status hifa4_attention_fwd_debug(const hifa4_packed* in, int B, int Hq, in
                                        void* o, hifa4_dtype o_dtype, float* lse,
                                        uint8_t* p_codes, uint8_t* p_scales,
                                        void* workspace, hifa4_stream_t stream);
+
+/* Optional inputs and outputs of hifa4_attention_fwd_ex (any field may be NULL).
+ *  s_bias     [B,Hq,Nkv] fp32, added to every score of head (b,h) and key j
+ *             before the softmax: S = RN(Q_hat K_hat^T + s_bias) (the Q-Mean
+ *             term written by hifa4_quantize_qkv_ex).
+ *  p_codes    [B,Hq,Nq,Nkv/2], p_scales [B,Hq,Nq,Nkv/16]: P_hat as in
+ *             hifa4_attention_fwd_debug (set both or neither).
+ *  tile_sums  [B,Hq,Nq,Nkv/128,2] fp32: for each query row and 128-key tile the
+ *             row visits, (sum of P_hat = codes x scales, sum of P before
+ *             quantization), both relative to the row's running max at that
+ *             tile. The abstract's epsilon_bar statistic is built from these
+ *             (hifa4_tile_stats). Tiles a row does not visit are not written.
+ * Each set field makes the call run the kernel's slower extras variant. */
+typedef struct {
+    const float* s_bias;
+    uint8_t* p_codes;
+    uint8_t* p_scales;
+    float* tile_sums;
+} hifa4_attention_extras;
+
+/* hifa4_attention_fwd with the extras above (extras may be NULL: the plain call). */
+hifa4_status hifa4_attention_fwd_ex(const hifa4_packed* in, int B, int Hq, int Hkv, int Nq, int Nkv, int D,
+                                    float sm_scale, unsigned flags, hifa4_norm_mode norm,
+                                    void* o, hifa4_dtype o_dtype, float* lse,
+                                    const hifa4_attention_extras* extras, void* workspace, hifa4_stream_t stream);
+
+/* Epsilon-bar per tile (HiFA4 abstract: the net probability-mass change of
+ * quantizing P, median -0.064 over the Qwen3-8B trace's tiles). A tile is 128
+ * query rows (the last one of a head may be shorter) of one (b,h) x one
+ * 128-key tile: eps_bar = mean over the tile's rows with sum P > 0 of
+ * (sum P_hat / sum P - 1) in fp32, NaN when no row of the tile has mass.
+ * tile_sums as written by hifa4_attention_fwd_ex, zeroed before that call so
+ * that unvisited tiles read as empty; eps_bar fp32 [B,Hq,ceil(Nq/128),Nkv/128]. */
+hifa4_status hifa4_tile_stats(const float* tile_sums, int B, int Hq, int Nq, int Nkv, float* eps_bar,
+                              hifa4_stream_t stream);
 
 /* hifa4_attention_fwd without a caller-provided workspace, for callers that
  * cannot allocate device memory: for example a plugin inside a host runtime

@@ -110,3 +110,54 @@ def test_noalloc_checks_arguments_before_any_cuda_call(lib):
     assert call(scale=0.0) == L.ERR_INVALID_ARG
     assert call(flags=8) == L.ERR_INVALID_ARG
     assert call(o=None) == L.ERR_INVALID_ARG
+
+
+def test_extension_calls_validate_on_the_host(lib):
+    """RoPE / Q-Mean / append / extras / tile-statistics calls reject bad
+    arguments before any CUDA call (a CUDA call would fail without a GPU)."""
+    from bit_quantized_flashattention_b200 import _lib as L
+    fake = ctypes.c_void_p(1 << 20)
+    odd = ctypes.c_void_p((1 << 20) + 4)
+    pk = L.Packed(*([fake] * 6))
+
+    def pre(**kw):
+        p = L.Prequant()
+        for k, v in kw.items():
+            setattr(p, k, v)
+        return ctypes.byref(p)
+
+    def qx(p):
+        return lib.hifa4_quantize_qkv_ex(fake, fake, fake, L.BF16, 1, 2, 1, 128, 128, 128, p, ctypes.byref(pk), None)
+
+    assert qx(pre(s=fake)) == L.ERR_INVALID_ARG                            # s without s_inv
+    assert qx(pre(rope_cos=fake)) == L.ERR_INVALID_ARG                     # cos without sin
+    assert qx(pre(rope_cos=fake, rope_sin=fake, n_pos=8, k_pos=fake)) == L.ERR_INVALID_ARG   # no q_pos
+    assert qx(pre(rope_cos=fake, rope_sin=fake, n_pos=0, q_pos=fake, k_pos=fake)) == L.ERR_INVALID_ARG
+    assert qx(pre(rope_cos=odd, rope_sin=fake, n_pos=8, q_pos=fake, k_pos=fake)) == L.ERR_INVALID_ARG
+    assert qx(pre(q_mean=fake)) == L.ERR_INVALID_ARG                       # q_mean without s_bias
+    assert qx(pre(q_mean=fake, s_bias=odd)) == L.ERR_INVALID_ARG
+
+    def app(n_new=16, start=0, cap=128, p=None):
+        return lib.hifa4_append_kv(fake, fake, L.BF16, 1, 1, n_new, 128, p, ctypes.byref(pk), cap, start, None)
+
+    assert app(n_new=8) == L.ERR_INVALID_ARG                               # not a multiple of 16
+    assert app(start=8) == L.ERR_INVALID_ARG
+    assert app(start=120) == L.ERR_INVALID_ARG                             # past the end of the cache
+    assert app(n_new=0) == L.ERR_INVALID_ARG
+    assert app(cap=100) == L.ERR_UNSUPPORTED
+    assert app(p=pre(q_mean=fake, s_bias=fake)) == L.ERR_INVALID_ARG       # no Q-Mean on an append
+    assert app(p=pre(rope_cos=fake, rope_sin=fake, n_pos=4)) == L.ERR_INVALID_ARG   # no k_pos
+
+    assert lib.hifa4_q_mean(fake, L.BF16, 1, 2, 1, 128, 96, None, fake, None) == L.ERR_UNSUPPORTED
+    assert lib.hifa4_q_mean(fake, L.BF16, 1, 3, 2, 128, 128, None, fake, None) == L.ERR_INVALID_ARG
+    assert lib.hifa4_q_mean(fake, L.BF16, 1, 2, 1, 128, 128, None, odd, None) == L.ERR_INVALID_ARG
+
+    def ax(ex):
+        return lib.hifa4_attention_fwd_ex(ctypes.byref(pk), 1, 2, 1, 128, 128, 128, ctypes.c_float(0.1), 0, 0, fake,
+                                          L.F32, None, ex, fake, None)
+
+    assert ax(ctypes.byref(L.AttentionExtras(None, fake, None, None))) == L.ERR_INVALID_ARG   # codes, no scales
+    assert ax(ctypes.byref(L.AttentionExtras(odd, None, None, None))) == L.ERR_INVALID_ARG
+    assert ax(ctypes.byref(L.AttentionExtras(None, None, None, odd))) == L.ERR_INVALID_ARG
+    assert lib.hifa4_tile_stats(fake, 1, 2, 128, 100, fake, None) == L.ERR_INVALID_ARG
+    assert lib.hifa4_tile_stats(None, 1, 2, 128, 128, fake, None) == L.ERR_INVALID_ARG

@@ -26,7 +26,7 @@ from dataclasses import dataclass, field
 
 import numpy as np
 
-__all__ = ["Config", "CONFIGS", "get", "k_gains", "q_slice", "k_slice",
+__all__ = ["Config", "CONFIGS", "get", "k_gains", "q_slice", "k_slice", "rope_tables",
            "v_slice", "qcal_slice", "kcal_slice", "full", "calib_full",
            "round_to_dtype", "to_bits"]
 
@@ -221,3 +221,12 @@ def calib_full(cfg: Config):
     qc = np.stack([qcal_slice(cfg, h) for h in range(cfg.Hq)])[None]
     kc = np.stack([kcal_slice(cfg, g, gains) for g in range(cfg.Hkv)])[None]
     return qc, kc
+
+
+def rope_tables(n_pos: int, D: int, base: float = 10000.0):
+    """Caller-side RoPE tables for the fused RoPE option: cos and sin of
+    pos * base^(-2d/D) for d < D/2, evaluated in float64 and rounded to float32
+    ([n_pos, D/2] each), the usual frequency schedule of rotary embeddings."""
+    inv = base ** (-np.arange(0, D // 2, dtype=np.float64) * 2.0 / D)
+    ang = np.arange(n_pos, dtype=np.float64)[:, None] * inv[None, :]
+    return np.cos(ang).astype(np.float32), np.sin(ang).astype(np.float32)
