@@ -672,6 +672,22 @@ def roofline(cfg, H, attn_ms, fp4_peak, hbm_peak):
             "frac": round(achieved / fp4_peak, 4), "algorithmic_flops": flops}
 
 
+def mufu_roofline(cfg, attn_ms, dev, clocks):
+    """The softmax's own bound: every visible (query, key) pair needs one exp2
+    and every 16 keys one more for the block scale; MUFU ex2 runs at 16 per clock
+    per SM (measured on this GPU), at the SM clock sampled during the run."""
+    import torch
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    mhz = (clocks or {}).get("sm_max_mhz") or 1965.0
+    pairs = cfg.flops() / (4.0 * cfg.D)
+    ex2 = pairs * (1.0 + 1.0 / 16.0)
+    peak = 16.0 * sms * mhz * 1e6
+    achieved = ex2 / (attn_ms * 1e-3)
+    return {"bound": "alu", "unit": "ex2/s", "achieved": round(achieved / 1e12, 4), "peak": round(peak / 1e12, 4),
+            "scale": "1e12", "frac": round(achieved / peak, 4), "ex2_per_launch": int(ex2),
+            "floor_us": round(ex2 / peak * 1e6, 2)}
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -733,6 +749,7 @@ def run_ours(args):
         "breakdown_ms": {"quantize": round(r["quant_ms"], 5), "attention": round(r["attn_ms"], 5)},
         "attention_only_tflops": round(attn_tflops, 2),
         "roofline": roof,
+        "alu_roofline": mufu_roofline(cfg, r["attn_ms"], dev, r["clocks"]),
         "e2e": {"value": round(ws * flops * n / (r["e2e_ms"] * 1e-3) / 1e12, 3), "unit": "TFLOPS",
                 "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"],
                 "ms_per_step": round(r["e2e_ms"] / n, 4),
@@ -779,7 +796,8 @@ def run_all_configs(args, dev, rank, ws, H, pk, fp4_peak):
                    "step_tflops": round(cfg.flops() / (r["total_ms"] / args.steps * 1e-3) / 1e12, 2),
                    "attention_ms": round(r["attn_ms"], 5),
                    "attention_tflops": round(cfg.flops() / (r["attn_ms"] * 1e-3) / 1e12, 2),
-                   "quantize_ms": round(r["quant_ms"], 5), "roofline": roof, "clocks": r["clocks"]}
+                   "quantize_ms": round(r["quant_ms"], 5), "roofline": roof,
+                   "alu_roofline": mufu_roofline(cfg, r["attn_ms"], dev, r["clocks"]), "clocks": r["clocks"]}
             if rank == 0 and not args.no_extras:
                 rec["sdpa_bf16_tflops"] = sdpa_context(r["q"], r["k"], r["v"], cfg, r["flush"])
                 rec["error_vs_fp32"] = error_vs_fp32(H, r["packed"], r["q"], r["k"], r["v"], cfg, norm, r["split_kv"])

@@ -41,8 +41,8 @@
 //
 // TMEM (512 columns): S [0,128), O tiles [128, 128 + NQT*NO), then the
 // scale-factor regions of Q, K, P and V.
-// The EXTRAS variant also takes an additive score term per (head, key)
-// (the Q-Mean bias) and writes, where asked, each row's P_hat codes and
+// Variants by XT: 0 the plain path; 1 also adds a score term per (head, key)
+// (the Q-Mean bias); 2 also writes, where asked, each row's P_hat codes and
 // scales and its per-tile sums (sum P_hat, sum P) for the epsilon statistics.
 //
 // Every mbarrier wait is bounded; when one gives up the CTA records
@@ -115,7 +115,9 @@ struct Cfg {
     static constexpr int OFF_ONES = OFF_SFV + STV * SFV_BYTES;
     static constexpr int OFF_LUT = OFF_ONES + 512;                        // float [128]
     static constexpr int OFF_BAR = OFF_LUT + 128 * 4;
-    static constexpr int OFF_MISC = OFF_BAR + 1024;
+    static constexpr int OFF_BIAS = OFF_BAR + 1024;                      // score-bias staging (XT >= 1)
+    static constexpr int BIAS_BYTES = 4 * NQT * 2 * 2 * 512;             // per softmax warp: 2 steps x 2 heads x 128 fp32
+    static constexpr int OFF_MISC = OFF_BIAS + BIAS_BYTES;
     static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;              // + alignment slack
     static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
     // decode merge scratch, after the loop: partial O rows (fp32, rows padded by
@@ -187,7 +189,7 @@ __device__ __forceinline__ void store_out(void* dst, const float* v) {
     }
 }
 
-template <int D, bool PREORDER, bool CAUSAL, int OUT, bool EXTRAS, bool DEC>
+template <int D, bool PREORDER, bool CAUSAL, int OUT, int XT, bool DEC>
 __global__ void __launch_bounds__(Cfg<D, PREORDER, DEC>::THREADS, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
@@ -678,10 +680,41 @@ __global__ void __launch_bounds__(Cfg<D, PREORDER, DEC>::THREADS, 1)
         const float one_sixth = rn_one_sixth();
         const uint32_t lut_s = smem_u32(lut);
         float m_old = -INFINITY, mc_old = 0.0f, l_hp = 0.0f;
-        const float* bias_row = nullptr;                    // score term of this row's head (EXTRAS)
-        if constexpr (EXTRAS)
-            if (p.s_bias != nullptr && valid) bias_row = p.s_bias + (out_row / (size_t)p.Nq) * (size_t)p.Nkv;
         bool ok = true;                                     // false once a wait gave up (then no more work)
+        // XT >= 1: the score bias of a step's kv tile is staged in shared memory
+        // one step ahead, a warp at a time: lane l loads 4 of the 128 values of
+        // each head the warp's rows belong to (at most two: Nq >= 16), and every
+        // row then reads its head's 128 values back as broadcast loads.
+        const bool use_bias = XT >= 1 && p.s_bias != nullptr;
+        const int my_head = valid ? (int)(out_row / (size_t)p.Nq) : -1;
+        const int head0 = __shfl_sync(0xFFFFFFFFu, my_head, 0);
+        const int head1 = __reduce_max_sync(0xFFFFFFFFu, my_head);
+        const uint32_t bias_s = sbase + C::OFF_BIAS + (uint32_t)(warp - kSmWarp0) * 2048u;   // [step & 1][head 0/1][128]
+        float4 bias_next[2];
+        auto load_bias = [&](int jn) {                      // this lane's part of step jn's rows
+            if (use_bias && head0 >= 0 && jn < own_steps) {
+                const size_t col = (size_t)(kt0 + jn) * 128 + 4 * lane;
+                bias_next[0] = __ldg(reinterpret_cast<const float4*>(p.s_bias + (size_t)head0 * p.Nkv + col));
+                bias_next[1] = head1 != head0
+                                   ? __ldg(reinterpret_cast<const float4*>(p.s_bias + (size_t)head1 * p.Nkv + col))
+                                   : bias_next[0];
+            }
+        };
+        auto stage_bias = [&](int jn) {
+            if (use_bias && head0 >= 0 && jn < own_steps) {
+                __syncwarp();
+                const uint32_t b = bias_s + (uint32_t)(jn & 1) * 1024u + 16u * lane;
+                sts_v4(b, __float_as_uint(bias_next[0].x), __float_as_uint(bias_next[0].y),
+                       __float_as_uint(bias_next[0].z), __float_as_uint(bias_next[0].w));
+                sts_v4(b + 512u, __float_as_uint(bias_next[1].x), __float_as_uint(bias_next[1].y),
+                       __float_as_uint(bias_next[1].z), __float_as_uint(bias_next[1].w));
+                __syncwarp();
+            }
+        };
+        if constexpr (XT >= 1) {
+            load_bias(0);
+            stage_bias(0);
+        }
         for (int j = 0; j < nt; ++j) {
             HIFA4_TRACE_POINT(qt, j, 0);
             ok = __all_sync(0xFFFFFFFFu, ok && mbar_wait(&bars->s_full[qt], j & 1, ctl));
@@ -711,12 +744,13 @@ __global__ void __launch_bounds__(Cfg<D, PREORDER, DEC>::THREADS, 1)
                 // (decode: a row whose range has ended masks the whole step)
                 const int n0 = (kt0 + j) * 128;
                 const int lim = j < own_steps ? last : -1;
-                if constexpr (EXTRAS) {
-                    if (bias_row != nullptr && j < own_steps) {
-                        const float4* bp = reinterpret_cast<const float4*>(bias_row + n0);
+                if constexpr (XT >= 1) {
+                    load_bias(j + 1);
+                    if (use_bias && my_head >= 0 && j < own_steps) {
+                        const uint32_t bp = bias_s + (uint32_t)(j & 1) * 1024u + (my_head != head0 ? 512u : 0u);
 #pragma unroll
                         for (int e = 0; e < 32; ++e) {
-                            const float4 b4 = __ldg(bp + e);
+                            const float4 b4 = lds_v4f(bp + 16u * e);
                             S[2 * e] = make_float2(__fadd_rn(S[2 * e].x, b4.x), __fadd_rn(S[2 * e].y, b4.y));
                             S[2 * e + 1] = make_float2(__fadd_rn(S[2 * e + 1].x, b4.z), __fadd_rn(S[2 * e + 1].y, b4.w));
                         }
@@ -755,7 +789,7 @@ __global__ void __launch_bounds__(Cfg<D, PREORDER, DEC>::THREADS, 1)
                         for (int e = 0; e < 4; ++e) {
                             const float2 t = __ffma2_rn(S[8 * b + 4 * h + e], c2, nmc2);
                             const float2 P = make_float2(ex2_approx(t.x), ex2_approx(t.y));
-                            if constexpr (!PREORDER || EXTRAS) lsum2 = __fadd2_rn(lsum2, P);
+                            if constexpr (!PREORDER || XT == 2) lsum2 = __fadd2_rn(lsum2, P);
                             const float2 yy = __fmul2_rn(P, r2);
                             y[2 * e] = yy.x;
                             y[2 * e + 1] = yy.y;
@@ -808,7 +842,7 @@ __global__ void __launch_bounds__(Cfg<D, PREORDER, DEC>::THREADS, 1)
                     tmem_st1(tl + C::COL_SFP + qt * 8 + wq, sfw[0]);
                     tmem_st1(tl + C::COL_SFP + qt * 8 + 4 + wq, sfw[1]);
                     tmem_wait_st();
-                    if constexpr (EXTRAS) {
+                    if constexpr (XT == 2) {
                         // per-tile mass of P_hat (codes x scales) and of P
                         if (p.tile_sums != nullptr && valid && j < own_steps) {
                             float sh = 0.0f;
@@ -834,6 +868,7 @@ __global__ void __launch_bounds__(Cfg<D, PREORDER, DEC>::THREADS, 1)
                 tc_fence_before();
                 m_old = m_new;
                 mc_old = mc_new;
+                if constexpr (XT >= 1) stage_bias(j + 1);
             }
             // every row's P_hat is in shared memory and its O is rescaled: PV
             if (ok) named_barrier_arrive(id_p, 160); else named_barrier_sync(id_p, 160);
@@ -948,11 +983,11 @@ __global__ void __launch_bounds__(Cfg<D, PREORDER, DEC>::THREADS, 1)
     if (threadIdx.x == 0) HIFA4_TRACE_POINT(4, 63, 2);
 }
 
-template <int D, bool PRE, bool CAUSAL, int OUT, bool EXTRAS, bool DEC>
+template <int D, bool PRE, bool CAUSAL, int OUT, int XT, bool DEC>
 static cudaError_t launch_one(const CUtensorMap* q, const CUtensorMap* k, const CUtensorMap* v, const AttnParams& p,
                               cudaStream_t st) {
     using C = Cfg<D, PRE, DEC>;
-    auto kern = attn_fwd_kernel<D, PRE, CAUSAL, OUT, EXTRAS, DEC>;
+    auto kern = attn_fwd_kernel<D, PRE, CAUSAL, OUT, XT, DEC>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t lc{};
@@ -968,22 +1003,23 @@ static cudaError_t launch_one(const CUtensorMap* q, const CUtensorMap* k, const 
     return cudaLaunchKernelEx(&lc, kern, *q, *k, *v, p);
 }
 
-template <int D, bool PRE, bool CAUSAL, int OUT, bool EXTRAS>
+template <int D, bool PRE, bool CAUSAL, int OUT, int XT>
 static cudaError_t launch_dec(const CUtensorMap* q, const CUtensorMap* k, const CUtensorMap* v, const AttnParams& p,
                               bool dec, cudaStream_t st) {
     if constexpr (D <= 128) {
-        if (dec) return launch_one<D, PRE, CAUSAL, OUT, EXTRAS, true>(q, k, v, p, st);
+        if (dec) return launch_one<D, PRE, CAUSAL, OUT, XT, true>(q, k, v, p, st);
     } else {
         if (dec) return cudaErrorInvalidValue;
     }
-    return launch_one<D, PRE, CAUSAL, OUT, EXTRAS, false>(q, k, v, p, st);
+    return launch_one<D, PRE, CAUSAL, OUT, XT, false>(q, k, v, p, st);
 }
 
 template <int D, bool PRE, bool CAUSAL, int OUT>
 static cudaError_t launch_extras(const CUtensorMap* q, const CUtensorMap* k, const CUtensorMap* v,
                                  const AttnParams& p, bool extras, bool dec, cudaStream_t st) {
-    return extras ? launch_dec<D, PRE, CAUSAL, OUT, true>(q, k, v, p, dec, st)
-                  : launch_dec<D, PRE, CAUSAL, OUT, false>(q, k, v, p, dec, st);
+    if (!extras) return launch_dec<D, PRE, CAUSAL, OUT, 0>(q, k, v, p, dec, st);
+    if (p.p_codes == nullptr && p.tile_sums == nullptr) return launch_dec<D, PRE, CAUSAL, OUT, 1>(q, k, v, p, dec, st);
+    return launch_dec<D, PRE, CAUSAL, OUT, 2>(q, k, v, p, dec, st);
 }
 
 template <int D, bool PRE, bool CAUSAL>

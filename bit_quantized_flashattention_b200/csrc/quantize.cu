@@ -342,9 +342,11 @@ __global__ void __launch_bounds__(256) quantize_qkv_kernel(RowJob q, RowJob k, V
 
 // Per-(batch, head, channel) mean of the pre-quantization Q (after RoPE and
 // smoothing) over the head's Nq tokens: the sum is accumulated in fp64, then
-// divided in fp64 and rounded once to fp32. One CTA per (b, h); lane chunk
-// c = tid % (D/8) of token lane tid / (D/8); token lanes are reduced through
-// shared memory in a fixed order.
+// divided in fp64 and rounded once to fp32. A thread-block cluster of CL CTAs
+// serves one (b, h): CTA rank r sums the tokens [r*Nq/CL, (r+1)*Nq/CL) (lane
+// chunk c = tid % (D/8) of token lane tid / (D/8)), reduces its token lanes
+// through shared memory in a fixed order, and rank 0 adds the CL partial sums
+// from the other CTAs' shared memory (distributed shared memory), in rank order.
 struct QMeanJob {
     const void* q;
     const float* scale;       // smoothing factors [Hkv, D] or null
@@ -356,22 +358,48 @@ struct QMeanJob {
     int Hq, G, Hkv, Nq;
 };
 
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ uint32_t cluster_size() {
+    uint32_t n;
+    asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(n));
+    return n;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// fp64 load from the shared memory of CTA `rank` of this cluster
+__device__ __forceinline__ double ld_cluster_f64(const double* local, uint32_t rank) {
+    uint32_t remote;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(local)), "r"(rank));
+    double v;
+    asm volatile("ld.shared::cluster.f64 %0, [%1];" : "=d"(v) : "r"(remote) : "memory");
+    return v;
+}
+
 template <typename T, int D, bool ROPE>
 __global__ void __launch_bounds__(256) q_mean_kernel(QMeanJob jb) {
     constexpr unsigned CPR = D / 8, TL = 256 / CPR;
     __shared__ double red[TL][D];
-    const unsigned bh = blockIdx.x;
+    __shared__ double part[D];
+    const unsigned cl = cluster_size(), rank = cluster_rank();
+    const unsigned bh = blockIdx.x / cl;
     const unsigned c = threadIdx.x % CPR, tl = threadIdx.x / CPR;
     const unsigned g = (bh % (unsigned)jb.Hq) / (unsigned)jb.G;
     float sc[8];
     if (jb.scale != nullptr) load8(jb.scale + (size_t)g * D + c * 8, sc);
+    const unsigned t_begin = (unsigned)(((unsigned long long)jb.Nq * rank) / cl);
+    const unsigned t_end = (unsigned)(((unsigned long long)jb.Nq * (rank + 1)) / cl);
     const T* xb = static_cast<const T*>(jb.q) + (size_t)bh * jb.Nq * D;
     double acc[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) acc[i] = 0.0;
-    for (unsigned base = 0; base < (unsigned)jb.Nq; base += TL) {      // warp-uniform trip count
+    for (unsigned base = t_begin; base < t_end; base += TL) {        // warp-uniform trip count
         const unsigned i = base + tl;
-        const bool real = i < (unsigned)jb.Nq;
+        const bool real = i < t_end;
         const uint4 raw = real ? *reinterpret_cast<const uint4*>(xb + (size_t)i * D + c * 8) : make_uint4(0u, 0u, 0u, 0u);
         float v[8];
         unpack8<T>(raw, v);
@@ -394,8 +422,17 @@ __global__ void __launch_bounds__(256) q_mean_kernel(QMeanJob jb) {
     for (unsigned d = threadIdx.x; d < (unsigned)D; d += 256) {
         double sum = 0.0;
         for (unsigned t = 0; t < TL; ++t) sum = __dadd_rn(sum, red[t][d]);
-        jb.mean[(size_t)bh * D + d] = __double2float_rn(__ddiv_rn(sum, (double)jb.Nq));
+        part[d] = sum;
     }
+    cluster_sync_all();                       // every CTA's partial sums are in its shared memory
+    if (rank == 0) {
+        for (unsigned d = threadIdx.x; d < (unsigned)D; d += 256) {
+            double sum = part[d];
+            for (unsigned r = 1; r < cl; ++r) sum = __dadd_rn(sum, ld_cluster_f64(&part[d], r));
+            jb.mean[(size_t)bh * D + d] = __double2float_rn(__ddiv_rn(sum, (double)jb.Nq));
+        }
+    }
+    cluster_sync_all();                       // rank 0 has read the others' shared memory
 }
 
 // ------------------------------------------------------------ calibration
@@ -523,13 +560,26 @@ cudaError_t launch_quantize_qkv(const QuantArgs& a, cudaStream_t st) {
 template <typename T, int D>
 static cudaError_t launch_q_mean_t(const QMeanArgs& a, cudaStream_t st) {
     QMeanJob jb{a.q, a.s, a.rope_cos, a.rope_sin, a.q_pos, a.n_pos, a.mean, a.Hq, a.Hq / a.Hkv, a.Hkv, a.Nq};
-    const long long n = (long long)a.B * a.Hq;
+    // one cluster per (b, h); more CTAs per cluster for long heads (at least
+    // 256 tokens each), at most the portable cluster size of 8
+    unsigned cl = 1;
+    while (cl < 8 && (long long)a.Nq >= 256LL * cl * 2) cl *= 2;
+    const long long n = (long long)a.B * a.Hq * cl;
     if (n > 0x7FFFFFFFLL) return cudaErrorInvalidConfiguration;
-    if (a.rope_cos != nullptr)
-        q_mean_kernel<T, D, true><<<(unsigned)n, 256, 0, st>>>(jb);
-    else
-        q_mean_kernel<T, D, false><<<(unsigned)n, 256, 0, st>>>(jb);
-    return cudaGetLastError();
+    cudaLaunchConfig_t lc{};
+    lc.gridDim = dim3((unsigned)n);
+    lc.blockDim = dim3(256);
+    lc.dynamicSmemBytes = 0;
+    lc.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = cl;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    lc.attrs = attr;
+    lc.numAttrs = 1;
+    if (a.rope_cos != nullptr) return cudaLaunchKernelEx(&lc, q_mean_kernel<T, D, true>, jb);
+    return cudaLaunchKernelEx(&lc, q_mean_kernel<T, D, false>, jb);
 }
 
 cudaError_t launch_q_mean(const QMeanArgs& a, cudaStream_t st) {

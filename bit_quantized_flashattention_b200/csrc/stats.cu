@@ -25,11 +25,18 @@ __global__ void __launch_bounds__(256) tile_stats_kernel(const float2* __restric
     const int i0 = 128 * a, i1 = min(128 * a + 128, Nq);
     float acc = 0.0f;
     int cnt = 0;
-    for (int i = i0; i < i1; ++i) {
-        const float2 s = sums[((size_t)bh * Nq + i) * T + t];
-        if (s.y > 0.0f) {
-            acc = __fadd_rn(acc, __fsub_rn(__fdiv_rn(s.x, s.y), 1.0f));
-            ++cnt;
+    const float2* row0 = sums + ((size_t)bh * Nq) * T + t;
+    // rows in order; eight loads in flight
+    for (int i = i0; i < i1; i += 8) {
+        float2 s[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) s[u] = i + u < i1 ? row0[(size_t)(i + u) * T] : make_float2(0.0f, 0.0f);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            if (s[u].y > 0.0f) {
+                acc = __fadd_rn(acc, __fsub_rn(__fdiv_rn(s[u].x, s[u].y), 1.0f));
+                ++cnt;
+            }
         }
     }
     eps_bar[idx] = cnt > 0 ? __fdiv_rn(acc, (float)cnt) : __int_as_float(0x7FC00000);
