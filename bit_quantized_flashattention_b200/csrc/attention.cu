@@ -479,7 +479,9 @@ __global__ void __launch_bounds__(Cfg<D, PREORDER, DEC>::THREADS, 1)
             };
             int ik = 0, iv = 0;
             bool ok = true;
-            uint64_t t_last = global_timer_ns();
+            // start of the current run of iterations without progress (0: none);
+            // the timer is read only while idle (a read costs hundreds of cycles)
+            uint64_t t_idle = 0;
             while ((ik < n_loads || iv < n_loads) && ok) {
                 bool progressed = false;
                 if (ik < n_loads && slot_free(bars->k_empty, ik, STK)) {
@@ -512,12 +514,14 @@ __global__ void __launch_bounds__(Cfg<D, PREORDER, DEC>::THREADS, 1)
                     progressed = true;
                 }
                 if (progressed) {
-                    t_last = global_timer_ns();
+                    t_idle = 0;
                 } else {
                     __nanosleep(128);
+                    const uint64_t now = global_timer_ns();
+                    if (t_idle == 0) t_idle = now;
                     if (*abort_flag) {
                         ok = false;
-                    } else if (global_timer_ns() - t_last > p.wait_limit_ns) {
+                    } else if (now - t_idle > p.wait_limit_ns) {
                         *abort_flag = 1;
                         atomicExch(p.status, kStatusTimeout);
                         ok = false;
@@ -772,10 +776,19 @@ __global__ void __launch_bounds__(Cfg<D, PREORDER, DEC>::THREADS, 1)
                 const float mc_new = (m_new == -INFINITY) ? 0.0f : __fmul_rn(m_new, c);
                 const float alpha = (m_old == -INFINITY) ? 0.0f : ex2_approx(mc_old - mc_new);
                 const float2 nmc2 = make_float2(-mc_new, -mc_new);
-                // P = 2^(S*c - mc), 8 blocks of 16 keys to E2M1 codes + E4M3 scales
+                // P = 2^(S*c - mc) in place: one stream of independent FFMA2 +
+                // ex2 pairs that keeps the MUFU busy; then 8 blocks of 16 keys to
+                // E4M3 scales and E2M1 codes (no MUFU on that chain but the 8
+                // block-scale exponentials)
+                float2 lsum2 = make_float2(0.0f, 0.0f);
+#pragma unroll
+                for (int e = 0; e < 64; ++e) {
+                    const float2 t = __ffma2_rn(S[e], c2, nmc2);
+                    S[e] = make_float2(ex2_approx(t.x), ex2_approx(t.y));
+                    if constexpr (!PREORDER || XT == 2) lsum2 = __fadd2_rn(lsum2, S[e]);
+                }
                 uint32_t code[16];
                 uint32_t sfw[2] = {0u, 0u};
-                float2 lsum2 = make_float2(0.0f, 0.0f);
 #pragma unroll
                 for (int b = 0; b < 8; ++b) {
                     const float pm = ex2_approx(__fmaf_rn(bm[b], c, -mc_new));
@@ -787,10 +800,7 @@ __global__ void __launch_bounds__(Cfg<D, PREORDER, DEC>::THREADS, 1)
                         float y[8];
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
-                            const float2 t = __ffma2_rn(S[8 * b + 4 * h + e], c2, nmc2);
-                            const float2 P = make_float2(ex2_approx(t.x), ex2_approx(t.y));
-                            if constexpr (!PREORDER || XT == 2) lsum2 = __fadd2_rn(lsum2, P);
-                            const float2 yy = __fmul2_rn(P, r2);
+                            const float2 yy = __fmul2_rn(S[8 * b + 4 * h + e], r2);
                             y[2 * e] = yy.x;
                             y[2 * e + 1] = yy.y;
                         }
