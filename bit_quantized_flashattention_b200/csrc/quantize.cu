@@ -164,7 +164,7 @@ struct VJob {
 // (ROPE variant), the smoothing multiply, the Q-Mean subtraction; on K rows
 // with bias_mean the Q-Mean score bias mean . K' of every head of the group is
 // reduced across the row's lanes from the same pre-quantization values.
-template <typename T, int D, bool ROPE>
+template <typename T, int D, bool ROPE, bool QM>
 __device__ __forceinline__ void quantize_rows_cta(const RowJob& jb, unsigned cta, const float* lut) {
     constexpr unsigned CPR = D / 8;                        // chunks per row
     constexpr unsigned RPB = 256 / CPR;                    // rows per CTA step
@@ -184,14 +184,11 @@ __device__ __forceinline__ void quantize_rows_cta(const RowJob& jb, unsigned cta
     const unsigned r_in = threadIdx.x / CPR;
     for (unsigned st = s0; st < s1; st += UNROLL) {
         uint4 raw[UNROLL];
-        RopeChunk rc[ROPE ? UNROLL : 1];
 #pragma unroll
         for (unsigned u = 0; u < UNROLL; ++u) {
             const unsigned pp = (st + u) * RPB + r_in;
             const bool real = st + u < s1 && pp < jb.rows_in;
             raw[u] = real ? *reinterpret_cast<const uint4*>(xg + (size_t)pp * D + c * 8) : make_uint4(0u, 0u, 0u, 0u);
-            if constexpr (ROPE)
-                rc[u] = load_rope<D>(jb.rope_cos, jb.rope_sin, jb.pos, real ? pp % jb.n_tok : 0u, jb.n_pos, c);
         }
 #pragma unroll
         for (unsigned u = 0; u < UNROLL; ++u) {
@@ -200,18 +197,22 @@ __device__ __forceinline__ void quantize_rows_cta(const RowJob& jb, unsigned cta
             const bool real = in_range && p < jb.rows_in;
             float v[8];
             unpack8<T>(raw[u], v);
-            if constexpr (ROPE) rope_chunk<T, D>(raw[u], c, rc[u], v);
+            if constexpr (ROPE) {
+                // the table rows are cache hits: loaded where they are used
+                const RopeChunk rc = load_rope<D>(jb.rope_cos, jb.rope_sin, jb.pos, real ? p % jb.n_tok : 0u, jb.n_pos, c);
+                rope_chunk<T, D>(raw[u], c, rc, v);
+            }
             if (jb.scale != nullptr) {
 #pragma unroll
                 for (int i = 0; i < 8; ++i) v[i] = __fmul_rn(v[i], sc[i]);
             }
-            if (jb.mean != nullptr && real) {
+            if (QM && jb.mean != nullptr && real) {
                 float m[8];
                 load8(jb.mean + ((size_t)grp * jb.G + p / jb.n_tok) * D + c * 8, m);
 #pragma unroll
                 for (int i = 0; i < 8; ++i) v[i] = __fsub_rn(v[i], m[i]);
             }
-            if (jb.bias_mean != nullptr) {
+            if (QM && jb.bias_mean != nullptr) {
                 // score bias of this key for every q head of the group
                 for (unsigned hl = 0; hl < jb.G; ++hl) {
                     float acc = 0.0f;
@@ -319,7 +320,7 @@ __device__ __forceinline__ void quantize_v_warp(const VJob& jb, unsigned gw_all,
 
 // One launch for the whole pass: CTAs [0, nq) quantize Q rows, [nq, nq + nk)
 // K rows, the rest V (8 warps per CTA).
-template <typename T, int D, bool ROPE>
+template <typename T, int D, bool ROPE, bool QM>
 __global__ void __launch_bounds__(256) quantize_qkv_kernel(RowJob q, RowJob k, VJob v, unsigned nq, unsigned nk,
                                                            unsigned v_warps) {
     __shared__ float lut[128];
@@ -329,9 +330,9 @@ __global__ void __launch_bounds__(256) quantize_qkv_kernel(RowJob q, RowJob k, V
     build_rcp_lut(lut);
     const unsigned b = blockIdx.x;
     if (b < nq) {
-        quantize_rows_cta<T, D, ROPE>(q, b, lut);
+        quantize_rows_cta<T, D, ROPE, QM>(q, b, lut);
     } else if (b < nq + nk) {
-        quantize_rows_cta<T, D, ROPE>(k, b - nq, lut);
+        quantize_rows_cta<T, D, ROPE, QM>(k, b - nq, lut);
     } else {
         const unsigned gw = (b - nq - nk) * 8 + (threadIdx.x >> 5);
         if (gw < v_warps) quantize_v_warp<T, D>(v, gw, lut);
@@ -539,12 +540,11 @@ static cudaError_t launch_qkv_t(const QuantArgs& a, cudaStream_t st) {
     const long long nk = n_grp * jk.blocks_per_group;
     const long long total = nq + nk + v_ctas;
     if (total > 0x7FFFFFFFLL) return cudaErrorInvalidConfiguration;
-    if (rope)
-        quantize_qkv_kernel<T, D, true><<<(unsigned)total, 256, 0, st>>>(jq, jk, jv, (unsigned)nq, (unsigned)nk,
-                                                                          (unsigned)v_warps);
-    else
-        quantize_qkv_kernel<T, D, false><<<(unsigned)total, 256, 0, st>>>(jq, jk, jv, (unsigned)nq, (unsigned)nk,
-                                                                           (unsigned)v_warps);
+    // variants: RoPE or not, Q-Mean or not (the plain pass carries neither)
+    const bool qm = a.q_mean != nullptr;
+    auto kern = rope ? (qm ? quantize_qkv_kernel<T, D, true, true> : quantize_qkv_kernel<T, D, true, false>)
+                     : (qm ? quantize_qkv_kernel<T, D, false, true> : quantize_qkv_kernel<T, D, false, false>);
+    kern<<<(unsigned)total, 256, 0, st>>>(jq, jk, jv, (unsigned)nq, (unsigned)nk, (unsigned)v_warps);
     return cudaGetLastError();
 }
 
