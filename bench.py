@@ -108,10 +108,12 @@ def profiled_traffic(cfg):
     return rec.get("dram_bytes_per_launch")
 
 
-def ingest_ncu(csv_path, workload, command):
+def ingest_ncu(csv_path, workload, command, scale=1.0):
     """Sum dram__bytes_read/write of the attention kernel's captured launches in an
     ncu CSV (``ncu --csv --metrics dram__bytes_read.sum,dram__bytes_write.sum ...``)
-    and record the per-launch mean, with the kernel-source hash, in the JSON."""
+    and record the per-launch mean, with the kernel-source hash, in the JSON.
+    scale > 1: the capture ran a smaller batch of the workload whose traffic grows
+    in proportion to the batch; the recorded bytes are scaled to the full launch."""
     import csv
     per_launch = {}
     with open(csv_path) as f:
@@ -120,10 +122,10 @@ def ingest_ncu(csv_path, workload, command):
         if "attn_fwd_kernel" not in row.get("Kernel Name", ""):
             continue
         name, unit, val = row["Metric Name"], row.get("Metric Unit", ""), row["Metric Value"].replace(",", "")
-        scale = {"byte": 1, "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9}.get(unit, 1)
+        unit_scale = {"byte": 1, "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9}.get(unit, 1)
         if name in ("dram__bytes_read.sum", "dram__bytes_write.sum"):
             per_launch.setdefault(row["ID"], 0.0)
-            per_launch[row["ID"]] += float(val) * scale
+            per_launch[row["ID"]] += float(val) * unit_scale
     if not per_launch:
         raise SystemExit(f"no attn_fwd_kernel DRAM counters in {csv_path}")
     rec = {}
@@ -132,8 +134,10 @@ def ingest_ncu(csv_path, workload, command):
             rec = json.load(f)
     except (OSError, ValueError):
         pass
-    rec[workload] = {"dram_bytes_per_launch": int(round(statistics.mean(per_launch.values()))),
+    rec[workload] = {"dram_bytes_per_launch": int(round(statistics.mean(per_launch.values()) * scale)),
                      "launches": len(per_launch), "source_sha256": attention_source_hash(), "command": command}
+    if scale != 1.0:
+        rec[workload]["scaled_from_capture_by"] = scale
     os.makedirs(os.path.dirname(TRAFFIC_JSON), exist_ok=True)
     with open(TRAFFIC_JSON, "w") as f:
         json.dump(rec, f, indent=1, sort_keys=True)
@@ -874,9 +878,11 @@ def main():
     ap.add_argument("--ingest-ncu", help="record DRAM bytes per attention launch from this ncu CSV")
     ap.add_argument("--workload", help="with --ingest-ncu: the workload name the capture ran")
     ap.add_argument("--ncu-command", default="", help="with --ingest-ncu: the command that made the capture")
+    ap.add_argument("--ncu-scale", type=float, default=1.0,
+                    help="with --ingest-ncu: the capture ran 1/scale of the workload's batch")
     args = ap.parse_args()
     if args.ingest_ncu:
-        ingest_ncu(args.ingest_ncu, args.workload or W.get(args.config).name, args.ncu_command)
+        ingest_ncu(args.ingest_ncu, args.workload or W.get(args.config).name, args.ncu_command, args.ncu_scale)
     elif args.impl == "reference":
         run_reference(args)
     else:
