@@ -268,6 +268,34 @@ __global__ void __launch_bounds__(Cfg<D, PREORDER, DEC>::THREADS, 1)
         return false;
     };
 
+    // One load of the K or V ring (a null load, which nothing reads, only
+    // arrives on its barrier); issued by the producer thread alone.
+    auto issue_k = [&](int i) {
+        const int st = i % STK;
+        if (load_users(i) == 0) {
+            mbar_arrive(&bars->k_full[st]);
+            return;
+        }
+        const int j = load_tile(i);
+        mbar_arrive_expect_tx(&bars->k_full[st], C::K_BYTES + C::SFQK_BYTES);
+        tma_load_2d(smem + C::OFF_K + st * C::K_BYTES, &tmK, 0, grp * p.Nkv + j * 128, &bars->k_full[st]);
+        bulk_load(smem + C::OFF_SFK + st * C::SFQK_BYTES, p.ks + ((size_t)grp * T + j) * C::SFQK_BYTES,
+                  C::SFQK_BYTES, &bars->k_full[st]);
+    };
+    auto issue_v = [&](int i) {
+        const int st = i % STV;
+        if (load_users(i) == 0) {
+            mbar_arrive(&bars->v_full[st]);
+            return;
+        }
+        const int j = load_tile(i);
+        mbar_arrive_expect_tx(&bars->v_full[st], C::V_TMA_BYTES + C::SFV_BYTES);
+        tma_load_2d(smem + C::OFF_V + st * C::V_STRIDE, &tmV, 0, (grp * T + j) * D, &bars->v_full[st]);
+        bulk_load(smem + C::OFF_SFV + st * C::SFV_BYTES, p.vts + ((size_t)grp * T + j) * C::SFV_BYTES,
+                  C::SFV_BYTES, &bars->v_full[st]);
+    };
+    int ik = 0, iv = 0;                     // K / V loads issued so far (producer thread)
+
     // --------------------------------------------------------------- setup
     if (threadIdx.x == 0) {
         HIFA4_TRACE_POINT(4, 63, 0);
@@ -287,6 +315,31 @@ __global__ void __launch_bounds__(Cfg<D, PREORDER, DEC>::THREADS, 1)
         for (int k = 0; k < 3; ++k) mbar_init(&bars->drain[k], 1);
         *abort_flag = 0;
         fence_barrier_init();
+        // This thread is also the producer. It starts the loads now, so that
+        // their latency overlaps the rest of the set-up: once the previous
+        // kernel of the stream has completed (programmatic dependent launch),
+        // Q_hat and the first ring-full of K_hat and V_hat^T tiles (every slot
+        // is free). The packed operands are read only after that wait.
+        if (!p.stall_loads) {
+            grid_dependency_wait();
+            const int nq_load = DEC ? 1 : n_qt;
+            mbar_arrive_expect_tx(&bars->q_full, nq_load * (C::Q_BYTES + C::SFQK_BYTES));
+            for (int qt = 0; qt < nq_load; ++qt) {
+                tma_load_2d(smem + C::OFF_Q + qt * C::Q_BYTES, &tmQ, 0, grp * rows_in_grp + (t0 + qt) * 128,
+                            &bars->q_full);
+                bulk_load(smem + C::OFF_SFQ + qt * C::SFQK_BYTES,
+                          p.qs + ((size_t)grp * p.Tq + t0 + qt) * C::SFQK_BYTES, C::SFQK_BYTES, &bars->q_full);
+            }
+            const int k0 = min(STK, n_loads), v0 = min(STV, n_loads);
+            while (ik < k0 || iv < v0) {
+                if (ik < k0) {
+                    issue_k(ik);
+                    HIFA4_TRACE_POINT(4, ik, 1);
+                    ++ik;
+                }
+                if (iv < v0) issue_v(iv++);
+            }
+        }
     }
     if (threadIdx.x >= 128 && threadIdx.x < 256) {
         const uint32_t i = threadIdx.x - 128;
@@ -450,21 +503,11 @@ __global__ void __launch_bounds__(Cfg<D, PREORDER, DEC>::THREADS, 1)
 
     if (warp == 0) {
         // ---------------------------------------------------------- producer
-        // The set-up above overlaps the end of the previous kernel in the
-        // stream (programmatic dependent launch); the packed operands are read
-        // only after it has completed. Every other read of those operands
-        // goes through this warp's copies. A slot is refilled once every query
-        // tile that read the previous load in it has released it.
-        grid_dependency_wait();
+        // Q_hat and the first ring-full of loads were issued during the set-up
+        // (above). Every other read of the packed operands goes through this
+        // warp's copies. A slot is refilled once every query tile that read
+        // the previous load in it has released it.
         if (lane == 0 && !p.stall_loads) {
-            const int nq_load = DEC ? 1 : n_qt;
-            mbar_arrive_expect_tx(&bars->q_full, nq_load * (C::Q_BYTES + C::SFQK_BYTES));
-            for (int qt = 0; qt < nq_load; ++qt) {
-                tma_load_2d(smem + C::OFF_Q + qt * C::Q_BYTES, &tmQ, 0, grp * rows_in_grp + (t0 + qt) * 128,
-                            &bars->q_full);
-                bulk_load(smem + C::OFF_SFQ + qt * C::SFQK_BYTES,
-                          p.qs + ((size_t)grp * p.Tq + t0 + qt) * C::SFQK_BYTES, C::SFQK_BYTES, &bars->q_full);
-            }
             // K and V go through their rings independently: a K slot is free
             // once the S MMAs that read it finished, a V slot once the PV MMAs
             // did, so K runs a step further ahead than V needs to.
@@ -477,7 +520,6 @@ __global__ void __launch_bounds__(Cfg<D, PREORDER, DEC>::THREADS, 1)
                     if (((users >> x) & 1) && !mbar_test(&empty[ip % stages][x], ph)) return false;
                 return true;
             };
-            int ik = 0, iv = 0;
             bool ok = true;
             // start of the current run of iterations without progress (0: none);
             // the timer is read only while idle (a read costs hundreds of cycles)
@@ -485,31 +527,13 @@ __global__ void __launch_bounds__(Cfg<D, PREORDER, DEC>::THREADS, 1)
             while ((ik < n_loads || iv < n_loads) && ok) {
                 bool progressed = false;
                 if (ik < n_loads && slot_free(bars->k_empty, ik, STK)) {
-                    const int st = ik % STK;
-                    if (load_users(ik) == 0) {
-                        mbar_arrive(&bars->k_full[st]);              // null load: nothing reads it
-                    } else {
-                        const int j = load_tile(ik);
-                        mbar_arrive_expect_tx(&bars->k_full[st], C::K_BYTES + C::SFQK_BYTES);
-                        tma_load_2d(smem + C::OFF_K + st * C::K_BYTES, &tmK, 0, grp * p.Nkv + j * 128, &bars->k_full[st]);
-                        bulk_load(smem + C::OFF_SFK + st * C::SFQK_BYTES,
-                                  p.ks + ((size_t)grp * T + j) * C::SFQK_BYTES, C::SFQK_BYTES, &bars->k_full[st]);
-                    }
+                    issue_k(ik);
                     HIFA4_TRACE_POINT(4, ik, 1);
                     ++ik;
                     progressed = true;
                 }
                 if (iv < n_loads && slot_free(bars->v_empty, iv, STV)) {
-                    const int st = iv % STV;
-                    if (load_users(iv) == 0) {
-                        mbar_arrive(&bars->v_full[st]);
-                    } else {
-                        const int j = load_tile(iv);
-                        mbar_arrive_expect_tx(&bars->v_full[st], C::V_TMA_BYTES + C::SFV_BYTES);
-                        tma_load_2d(smem + C::OFF_V + st * C::V_STRIDE, &tmV, 0, (grp * T + j) * D, &bars->v_full[st]);
-                        bulk_load(smem + C::OFF_SFV + st * C::SFV_BYTES,
-                                  p.vts + ((size_t)grp * T + j) * C::SFV_BYTES, C::SFV_BYTES, &bars->v_full[st]);
-                    }
+                    issue_v(iv);
                     ++iv;
                     progressed = true;
                 }
@@ -716,6 +740,9 @@ __global__ void __launch_bounds__(Cfg<D, PREORDER, DEC>::THREADS, 1)
             }
         };
         if constexpr (XT >= 1) {
+            // the bias is written by the previous kernel of the stream: read it
+            // only once that kernel has completed (programmatic dependent launch)
+            if (use_bias) grid_dependency_wait();
             load_bias(0);
             stage_bias(0);
         }
