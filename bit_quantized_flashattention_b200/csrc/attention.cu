@@ -315,31 +315,6 @@ __global__ void __launch_bounds__(Cfg<D, PREORDER, DEC>::THREADS, 1)
         for (int k = 0; k < 3; ++k) mbar_init(&bars->drain[k], 1);
         *abort_flag = 0;
         fence_barrier_init();
-        // This thread is also the producer. It starts the loads now, so that
-        // their latency overlaps the rest of the set-up: once the previous
-        // kernel of the stream has completed (programmatic dependent launch),
-        // Q_hat and the first ring-full of K_hat and V_hat^T tiles (every slot
-        // is free). The packed operands are read only after that wait.
-        if (!p.stall_loads) {
-            grid_dependency_wait();
-            const int nq_load = DEC ? 1 : n_qt;
-            mbar_arrive_expect_tx(&bars->q_full, nq_load * (C::Q_BYTES + C::SFQK_BYTES));
-            for (int qt = 0; qt < nq_load; ++qt) {
-                tma_load_2d(smem + C::OFF_Q + qt * C::Q_BYTES, &tmQ, 0, grp * rows_in_grp + (t0 + qt) * 128,
-                            &bars->q_full);
-                bulk_load(smem + C::OFF_SFQ + qt * C::SFQK_BYTES,
-                          p.qs + ((size_t)grp * p.Tq + t0 + qt) * C::SFQK_BYTES, C::SFQK_BYTES, &bars->q_full);
-            }
-            const int k0 = min(STK, n_loads), v0 = min(STV, n_loads);
-            while (ik < k0 || iv < v0) {
-                if (ik < k0) {
-                    issue_k(ik);
-                    HIFA4_TRACE_POINT(4, ik, 1);
-                    ++ik;
-                }
-                if (iv < v0) issue_v(iv++);
-            }
-        }
     }
     if (threadIdx.x >= 128 && threadIdx.x < 256) {
         const uint32_t i = threadIdx.x - 128;
@@ -503,11 +478,21 @@ __global__ void __launch_bounds__(Cfg<D, PREORDER, DEC>::THREADS, 1)
 
     if (warp == 0) {
         // ---------------------------------------------------------- producer
-        // Q_hat and the first ring-full of loads were issued during the set-up
-        // (above). Every other read of the packed operands goes through this
-        // warp's copies. A slot is refilled once every query tile that read
-        // the previous load in it has released it.
+        // The set-up above overlaps the end of the previous kernel in the
+        // stream (programmatic dependent launch); the packed operands are read
+        // only after it has completed. Every other read of those operands
+        // goes through this warp's copies. A slot is refilled once every query
+        // tile that read the previous load in it has released it.
+        grid_dependency_wait();
         if (lane == 0 && !p.stall_loads) {
+            const int nq_load = DEC ? 1 : n_qt;
+            mbar_arrive_expect_tx(&bars->q_full, nq_load * (C::Q_BYTES + C::SFQK_BYTES));
+            for (int qt = 0; qt < nq_load; ++qt) {
+                tma_load_2d(smem + C::OFF_Q + qt * C::Q_BYTES, &tmQ, 0, grp * rows_in_grp + (t0 + qt) * 128,
+                            &bars->q_full);
+                bulk_load(smem + C::OFF_SFQ + qt * C::SFQK_BYTES,
+                          p.qs + ((size_t)grp * p.Tq + t0 + qt) * C::SFQK_BYTES, C::SFQK_BYTES, &bars->q_full);
+            }
             // K and V go through their rings independently: a K slot is free
             // once the S MMAs that read it finished, a V slot once the PV MMAs
             // did, so K runs a step further ahead than V needs to.
