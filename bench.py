@@ -510,6 +510,31 @@ def run_extensions(args, dev, H):
     del q, k, v, packed, o, ts, eb
     torch.cuda.empty_cache()
 
+    # the step with Q quantized inside the attention kernel (quantize K/V only)
+    for ci in (2, 4):
+        cfg = W.get(ci)
+        q, k, v, cal = make_inputs(cfg, dev)
+        s = s_inv = None
+        if cal is not None:
+            s, s_inv = H.calibrate_smooth(cal[0], cal[1], cfg.alpha)
+        packed = H.alloc_packed(cfg.B, cfg.Hq, cfg.Hkv, cfg.Nq, cfg.Nkv, cfg.D, dev)
+        o = torch.empty(cfg.B, cfg.Hq, cfg.Nq, cfg.D, dtype=torch.bfloat16, device=dev)
+        lse = torch.empty(cfg.B, cfg.Hq, cfg.Nq, dtype=torch.float32, device=dev)
+        wsp = H.alloc_workspace(cfg.B, cfg.Hq, cfg.Hkv, cfg.Nq, cfg.Nkv, cfg.D, dev)
+        tq = time_fn(lambda: H.quantize_qkv(q, k, v, s, s_inv, out=packed), n, flush, stream)
+        ta = time_fn(lambda: H.attention_fwd(packed, causal=cfg.causal, out=o, lse=lse, workspace=wsp), n, flush,
+                     stream)
+        tkv = time_fn(lambda: H.quantize_kv(k, v, s_inv, out=packed), n, flush, stream)
+        taq = time_fn(lambda: H.attention_fwd_q(q, packed, s, causal=cfg.causal, out=o, lse=lse, workspace=wsp), n,
+                      flush, stream)
+        emit({"extension": "in_kernel_q_quantization", "workload": cfg.name,
+              "packed_path_ms": {"quantize_qkv": round(tq, 5), "attention_fwd": round(ta, 5),
+                                 "sum": round(tq + ta, 5)},
+              "fused_path_ms": {"quantize_kv": round(tkv, 5), "attention_fwd_q": round(taq, 5),
+                                "sum": round(tkv + taq, 5)}})
+        del q, k, v, packed, o, lse
+        torch.cuda.empty_cache()
+
     # KV-cache append on the decode workload (B = 64, 8 kv heads, 8192 slots)
     cfg = W.get(5)
     cache = H.alloc_packed(cfg.B, cfg.Hq, cfg.Hkv, cfg.Nq, cfg.Nkv, cfg.D, dev)
@@ -546,9 +571,27 @@ def measure(cfg, norm, args, dev, rank, ws, H, want_e2e=True):
     flush = L2Flush(dev)
     stream = torch.cuda.current_stream()
 
+    # fused_q: the attention kernel quantizes Q itself (D = 128 outside the
+    # decode mode; same result, bit for bit) and the quantize pass covers K and
+    # V only. Measured a tie on the Qwen3-8B step, so the step keeps the packed
+    # path; --extensions times both.
+    fused_q = getattr(args, "fused_q", False) and cfg.D == 128 and n_splits == 1
+
+    def quant():
+        if fused_q:
+            H.quantize_kv(k, v, s_inv, out=packed)
+        else:
+            H.quantize_qkv(q, k, v, s, s_inv, out=packed)
+
+    def attn():
+        if fused_q:
+            H.attention_fwd_q(q, packed, s, causal=cfg.causal, norm=norm, out=o, lse=lse, workspace=wsp)
+        else:
+            H.attention_fwd(packed, causal=cfg.causal, norm=norm, out=o, lse=lse, workspace=wsp, split_kv=split_kv)
+
     def step():
-        H.quantize_qkv(q, k, v, s, s_inv, out=packed)
-        H.attention_fwd(packed, causal=cfg.causal, norm=norm, out=o, lse=lse, workspace=wsp, split_kv=split_kv)
+        quant()
+        attn()
 
     for _ in range(max(args.warmup, 3)):
         step()
@@ -566,9 +609,9 @@ def measure(cfg, norm, args, dev, rank, ws, H, want_e2e=True):
     with torch.cuda.graph(g_step):
         step()
     with torch.cuda.graph(g_quant):
-        H.quantize_qkv(q, k, v, s, s_inv, out=packed)
+        quant()
     with torch.cuda.graph(g_attn):
-        H.attention_fwd(packed, causal=cfg.causal, norm=norm, out=o, lse=lse, workspace=wsp, split_kv=split_kv)
+        attn()
     for g in (g_step, g_quant, g_attn):
         g.replay()
     torch.cuda.synchronize()
@@ -605,9 +648,11 @@ def measure(cfg, norm, args, dev, rank, ws, H, want_e2e=True):
     st = max_over_ranks(H.get_status(wsp), dev)
     if st != 0:
         raise RuntimeError(f"kernel status {int(st)} in the timed region (max over ranks)")
+    if fused_q:
+        H.quantize_qkv(q, k, v, s, s_inv, out=packed)      # packed Q_hat for the untimed extras
     res = dict(q=q, k=k, v=v, s=s, s_inv=s_inv, packed=packed, o=o, lse=lse, wsp=wsp, flush=flush,
                total_ms=total_ms, attn_ms=statistics.mean(attn_ms), quant_ms=statistics.mean(quant_ms),
-               clocks=clk.summary(), n_splits=n_splits, split_kv=split_kv)
+               clocks=clk.summary(), n_splits=n_splits, split_kv=split_kv, fused_q=fused_q)
     del g_step, g_quant, g_attn
     if not want_e2e:
         return res
@@ -643,9 +688,14 @@ def measure(cfg, norm, args, dev, rank, ws, H, want_e2e=True):
             s_cp.wait_event(ev_in[b])
             if i >= nb:
                 s_cp.wait_event(ev_out[b])         # step i-2's results have left this output buffer
-            H.quantize_qkv(dq[b], dk[b], dv[b], s, s_inv, out=dpk[b], stream=s_cp)
-            H.attention_fwd(dpk[b], causal=cfg.causal, norm=norm, out=do[b], lse=dl[b], workspace=dws[b],
-                            stream=s_cp, split_kv=split_kv)
+            if fused_q:
+                H.quantize_kv(dk[b], dv[b], s_inv, out=dpk[b], stream=s_cp)
+                H.attention_fwd_q(dq[b], dpk[b], s, causal=cfg.causal, norm=norm, out=do[b], lse=dl[b],
+                                  workspace=dws[b], stream=s_cp)
+            else:
+                H.quantize_qkv(dq[b], dk[b], dv[b], s, s_inv, out=dpk[b], stream=s_cp)
+                H.attention_fwd(dpk[b], causal=cfg.causal, norm=norm, out=do[b], lse=dl[b], workspace=dws[b],
+                                stream=s_cp, split_kv=split_kv)
             ev_cp[b].record(s_cp)
         with torch.cuda.stream(s_out):
             s_out.wait_event(ev_cp[b])
@@ -762,7 +812,8 @@ def run_ours(args):
                    "kv_splits": r["n_splits"],
                    "inputs": cfg.dtype, "output": "bf16", "parallelism": f"replicas{ws}" if ws > 1 else "single",
                    "l2": "cold and clean between steps (256 MiB write, then 256 MiB read)",
-                   "step": "quantize_qkv + attention_fwd (calibration offline)",
+                   "step": ("quantize_kv + attention_fwd_q (Q quantized inside the attention kernel; "
+                            "calibration offline)" if r["fused_q"] else "quantize_qkv + attention_fwd (calibration offline)"),
                    "launch": "the step replayed from a CUDA graph (programmatic dependent launch between its two kernels)"},
         "fp4_tensor_pct": round(100.0 * value / ws / fp4_peak, 2),
         "breakdown_ms": {"quantize": round(r["quant_ms"], 5), "attention": round(r["attn_ms"], 5)},
@@ -777,7 +828,7 @@ def run_ours(args):
         "clocks": r["clocks"],
     }
     # the HBM-bound quantize pass: algorithmic bytes (read 2 B/elem, write 0.5625 B/elem)
-    elems = cfg.B * cfg.Hq * cfg.Nq * cfg.D + 2 * cfg.B * cfg.Hkv * cfg.Nkv * cfg.D
+    elems = (0 if r["fused_q"] else cfg.B * cfg.Hq * cfg.Nq * cfg.D) + 2 * cfg.B * cfg.Hkv * cfg.Nkv * cfg.D
     line["quantize_gbs"] = round(elems * (2 + 0.5625) / (r["quant_ms"] * 1e-3) / 1e9, 1)
     if rank == 0 and not args.no_extras:
         line["sdpa_bf16_tflops"] = sdpa_context(r["q"], r["k"], r["v"], cfg, r["flush"])
@@ -887,6 +938,8 @@ def main():
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle samples")
     ap.add_argument("--no-extras", action="store_true", help="skip SDPA, fp32-error and FP4-GEMM context")
     ap.add_argument("--all-configs", action="store_true", help="time every workload (one JSON line each)")
+    ap.add_argument("--fused-q", action="store_true",
+                    help="time the step as quantize_kv + attention_fwd_q (Q quantized in the attention kernel)")
     ap.add_argument("--extensions", action="store_true",
                     help="time Q-Mean, fused RoPE quantize, KV appends and the epsilon statistics")
     ap.add_argument("--table", help="with --all-configs: also write a markdown table here")

@@ -17,7 +17,7 @@ EXPORTS = ["hifa4_packed_bytes", "hifa4_workspace_bytes", "hifa4_calibrate_smoot
            "hifa4_quantize_kv", "hifa4_attention_fwd", "hifa4_attention_fwd_debug", "hifa4_get_status",
            "hifa4_debug_set_wait_limit", "hifa4_status_string", "hifa4_version", "hifa4_attention_fwd_noalloc",
            "hifa4_last_cuda_error", "hifa4_attention_splits", "hifa4_quantize_qkv_ex", "hifa4_q_mean",
-           "hifa4_append_kv", "hifa4_attention_fwd_ex", "hifa4_tile_stats"]
+           "hifa4_append_kv", "hifa4_attention_fwd_ex", "hifa4_tile_stats", "hifa4_attention_fwd_q"]
 
 
 class Packed(ctypes.Structure):
@@ -83,6 +83,8 @@ def load():
     L.hifa4_attention_fwd_ex.argtypes = [pk] + [ci] * 6 + [cf, cu, ci, vp, ci, vp, ctypes.POINTER(AttentionExtras),
                                                            vp, vp]
     L.hifa4_attention_fwd_ex.restype = ci
+    L.hifa4_attention_fwd_q.argtypes = [vp, ci, vp, pk] + [ci] * 6 + [cf, cu, ci, vp, ci, vp, vp, vp]
+    L.hifa4_attention_fwd_q.restype = ci
     L.hifa4_tile_stats.argtypes = [vp, ci, ci, ci, ci, vp, vp]
     L.hifa4_tile_stats.restype = ci
     L.hifa4_get_status.argtypes = [vp, vp]

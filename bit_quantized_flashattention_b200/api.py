@@ -311,6 +311,34 @@ def attention_fwd_ex(packed: PackedQKV, sm_scale: float | None = None, causal: b
     return dict(o=out, lse=lse, p_codes=pc, p_scales=ps, tile_sums=ts)
 
 
+def attention_fwd_q(q: torch.Tensor, kv: PackedQKV, s=None, sm_scale: float | None = None, causal: bool = False,
+                    norm="p_reorder", out_dtype=torch.bfloat16, out=None, lse=None, workspace=None, stream=None):
+    """Attention from unquantized Q (bf16/fp16 [B,Hq,Nq,D], D = 128) and packed K/V
+    (``kv``: e.g. quantize_kv or append_kv): the kernel quantizes Q itself, with
+    the optional Smooth-QK factors ``s`` [Hkv,D]. Same result as quantize_qkv +
+    attention_fwd. Returns (O, LSE)."""
+    _check_input(q, "q")
+    B, Hq, Nq, D = q.shape
+    if (B, D) != (kv.B, kv.D):
+        raise ValueError("q does not match the packed K/V")
+    Hkv, Nkv = kv.Hkv, kv.Nkv
+    dev = q.device
+    if sm_scale is None:
+        sm_scale = 1.0 / math.sqrt(D)
+    if out is None:
+        out = torch.empty(B, Hq, Nq, D, dtype=out_dtype, device=dev)
+    if lse is None:
+        lse = torch.empty(B, Hq, Nq, dtype=torch.float32, device=dev)
+    if workspace is None:
+        workspace = alloc_workspace(B, Hq, Hkv, Nq, Nkv, D, dev)
+    st = kv.struct()
+    L.check(L.load().hifa4_attention_fwd_q(_ptr(q), _DT[q.dtype], _ptr(s), ctypes.byref(st), B, Hq, Hkv, Nq, Nkv, D,
+                                           float(sm_scale), L.CAUSAL if causal else 0, _NORM[norm], _ptr(out),
+                                           _DT[out.dtype], _ptr(lse), _ptr(workspace), _stream(stream)),
+            "attention_fwd_q")
+    return out, lse
+
+
 def tile_stats(tile_sums: torch.Tensor, out=None, stream=None) -> torch.Tensor:
     """Per-tile epsilon-bar [B,Hq,ceil(Nq/128),Nkv/128] (NaN: tile without mass)
     from the tile sums of attention_fwd_ex."""

@@ -158,7 +158,7 @@ hifa4_status attention_impl(const hifa4_packed* in, int B, int Hq, int Hkv, int 
     if ((x.p_codes == nullptr) != (x.p_scales == nullptr)) return HIFA4_ERR_INVALID_ARG;
     if (!aligned16(x.p_codes) || !aligned16(x.p_scales) || !aligned16(x.s_bias) || !aligned16(x.tile_sums))
         return HIFA4_ERR_INVALID_ARG;
-    const bool extras = x.p_codes != nullptr || x.s_bias != nullptr || x.tile_sums != nullptr;
+    const int xt = (x.p_codes != nullptr || x.tile_sums != nullptr) ? 2 : (x.s_bias != nullptr ? 1 : 0);
     const bool causal = (flags & HIFA4_CAUSAL) != 0;
     const long long rows_q = (long long)B * Hq * Nq, rows_k = (long long)B * Hkv * Nkv, rows_v = (long long)B * Hkv * D;
     const Sizes sz = sizes_of(B, Hq, Hkv, Nq, Nkv, D);
@@ -200,7 +200,7 @@ hifa4_status attention_impl(const hifa4_packed* in, int B, int Hq, int Hkv, int 
     p.wait_limit_ns = lim > 0 ? (unsigned long long)lim : kDefaultWaitNs;
     p.stall_loads = g_stall_loads.load();
     const int out = o_dtype == HIFA4_F16 ? 0 : (o_dtype == HIFA4_BF16 ? 1 : 2);
-    return from_cuda(launch_attention(&tq, &tk, &tv, p, D, (int)norm, causal, out, extras, dec,
+    return from_cuda(launch_attention(&tq, &tk, &tv, p, D, (int)norm, causal, out, xt, dec,
                                       reinterpret_cast<cudaStream_t>(stream)));
 }
 
@@ -397,6 +397,61 @@ hifa4_status hifa4_attention_fwd_debug(const hifa4_packed* in, int B, int Hq, in
     x.p_codes = p_codes;
     x.p_scales = p_scales;
     return attention_impl(in, B, Hq, Hkv, Nq, Nkv, D, sm_scale, flags, norm, o, o_dtype, lse, &x, workspace, stream);
+}
+
+hifa4_status hifa4_attention_fwd_q(const void* q, hifa4_dtype q_dtype, const float* s, const hifa4_packed* kv, int B,
+                                   int Hq, int Hkv, int Nq, int Nkv, int D, float sm_scale, unsigned flags,
+                                   hifa4_norm_mode norm, void* o, hifa4_dtype o_dtype, float* lse, void* workspace,
+                                   hifa4_stream_t stream) {
+    if (q == nullptr || kv == nullptr) return HIFA4_ERR_INVALID_ARG;
+    if (q_dtype != HIFA4_F16 && q_dtype != HIFA4_BF16) return HIFA4_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(s)) return HIFA4_ERR_INVALID_ARG;
+    // the Q entries of the packed struct are not read: stand-ins keep the shared checks
+    hifa4_packed in = *kv;
+    in.qc = in.kc;
+    in.qs = in.ks;
+    const hifa4_status chk = check_attention_args(&in, B, Hq, Hkv, Nq, Nkv, D, sm_scale, flags, norm, o, o_dtype, lse);
+    if (chk != HIFA4_OK) return chk;
+    if (D != 128 || decode_mode(Hq, Hkv, Nq, Nkv, D, flags)) return HIFA4_ERR_UNSUPPORTED;
+    if (workspace == nullptr || !aligned16(workspace)) return HIFA4_ERR_INVALID_ARG;
+    const bool causal = (flags & HIFA4_CAUSAL) != 0;
+    const long long rows_k = (long long)B * Hkv * Nkv, rows_v = (long long)B * Hkv * D;
+    const Sizes sz = sizes_of(B, Hq, Hkv, Nq, Nkv, D);
+    const int nqt = 2;
+    const long long n_work = (long long)B * Hkv * ((sz.Tq + nqt - 1) / nqt);
+    // Q as rows of D 16-bit elements (256 bytes), loaded as two 128-byte column
+    // halves per 128-row tile with the 128-byte swizzle
+    const long long rows_q = (long long)B * Hq * Nq;
+    CUtensorMap tq, tk, tv;
+    if (!make_map(&tq, q, (uint64_t)D * 2, (uint64_t)rows_q, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map(&tk, kv->kc, (uint64_t)D / 2, (uint64_t)rows_k, D / 2, 128, CU_TENSOR_MAP_SWIZZLE_64B) ||
+        !make_map(&tv, kv->vtc, 64, (uint64_t)rows_v * (Nkv / 128), 64, D, CU_TENSOR_MAP_SWIZZLE_64B))
+        return from_cuda(cudaErrorInvalidValue);
+    AttnParams p{};
+    p.ks = static_cast<const uint8_t*>(kv->ks);
+    p.vts = static_cast<const uint8_t*>(kv->vts);
+    p.o = o;
+    p.lse = lse;
+    p.q_scale = s;
+    p.q_bf16 = q_dtype == HIFA4_BF16 ? 1 : 0;
+    p.status = static_cast<uint32_t*>(workspace);
+    p.B = B;
+    p.Hq = Hq;
+    p.Hkv = Hkv;
+    p.Nq = Nq;
+    p.Nkv = Nkv;
+    p.G = Hq / Hkv;
+    p.Tq = sz.Tq;
+    p.n_kv_tiles = Nkv / 128;
+    p.n_work = (int)n_work;
+    p.heavy_first = (causal && Nq % (128 * nqt) == 0) ? 1 : 0;
+    p.c = (float)((double)sm_scale * 1.4426950408889634074);
+    const long long lim = g_wait_limit_ns.load();
+    p.wait_limit_ns = lim > 0 ? (unsigned long long)lim : kDefaultWaitNs;
+    p.stall_loads = g_stall_loads.load();
+    const int out = o_dtype == HIFA4_F16 ? 0 : (o_dtype == HIFA4_BF16 ? 1 : 2);
+    return from_cuda(launch_attention(&tq, &tk, &tv, p, D, (int)norm, causal, out, 3, false,
+                                      reinterpret_cast<cudaStream_t>(stream)));
 }
 
 hifa4_status hifa4_tile_stats(const float* tile_sums, int B, int Hq, int Nq, int Nkv, float* eps_bar,

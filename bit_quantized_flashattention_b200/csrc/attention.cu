@@ -43,7 +43,11 @@
 // scale-factor regions of Q, K, P and V.
 // Variants by XT: 0 the plain path; 1 also adds a score term per (head, key)
 // (the Q-Mean bias); 2 also writes, where asked, each row's P_hat codes and
-// scales and its per-tile sums (sum P_hat, sum P) for the epsilon statistics.
+// scales and its per-tile sums (sum P_hat, sum P) for the epsilon statistics;
+// 3 (D = 128, not decode) takes Q unquantized (bf16 / fp16) and quantizes it
+// itself: each softmax thread smooths and quantizes its own row into the
+// shared-memory Q_hat tile and scale atoms at the start, while the first K / V
+// loads are in flight, with the same rule and result as the quantize pass.
 //
 // Every mbarrier wait is bounded; when one gives up the CTA records
 // HIFA4_ERR_TIMEOUT in the workspace, drains its copies and MMAs, frees TMEM
@@ -61,7 +65,7 @@ constexpr int kSmWarp0 = 4;          // first softmax warp (0: loads, 1: TMEM ow
 constexpr int kMaxStages = 12;
 constexpr int kDecSplits = 4;        // kv ranges of the split-kv decode mode
 
-template <int D, bool PREORDER, bool DEC>
+template <int D, bool PREORDER, bool DEC, bool QR = false>
 struct Cfg {
     static_assert(!DEC || D <= 128, "decode mode needs two query tiles per CTA");
     static constexpr int NQT = D == 256 ? 1 : 2;          // 128-row query tiles per CTA
@@ -115,10 +119,14 @@ struct Cfg {
     static constexpr int OFF_ONES = OFF_SFV + STV * SFV_BYTES;
     static constexpr int OFF_LUT = OFF_ONES + 512;                        // float [128]
     static constexpr int OFF_BAR = OFF_LUT + 128 * 4;
-    static constexpr int OFF_BIAS = OFF_BAR + 1024;                      // score-bias staging (XT >= 1)
+    static constexpr int OFF_BIAS = OFF_BAR + 1024;                      // score-bias staging (XT = 1, 2)
     static constexpr int BIAS_BYTES = 4 * NQT * 2 * 2 * 512;             // per softmax warp: 2 steps x 2 heads x 128 fp32
     static constexpr int OFF_MISC = OFF_BIAS + BIAS_BYTES;
-    static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;              // + alignment slack
+    // in-kernel Q quantization: the caller's bf16 / fp16 Q tiles, two 128-byte
+    // column halves per tile (128-byte swizzle), staged by TMA
+    static constexpr int QRAW_HALF = 128 * 128;
+    static constexpr int OFF_QRAW = (OFF_MISC + 16 + 1023) / 1024 * 1024;  // + (qt * 2 + half) * QRAW_HALF
+    static constexpr int SMEM_BYTES = (QR ? OFF_QRAW + NQT * 2 * QRAW_HALF : OFF_MISC + 16) + 1024;   // + alignment slack
     static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
     // decode merge scratch, after the loop: partial O rows (fp32, rows padded by
     // 4 floats) in the K/V ring, the (mc, l) pairs in the P buffers
@@ -135,6 +143,7 @@ struct Bars {
     uint64_t s_full[2];                // S of query tile x is in TMEM
     uint64_t o_done[2];                // PV MMA of query tile x finished
     uint64_t drain[3];                 // teardown: MMAs issued by the S issuer / each PV issuer
+    uint64_t q_ready;                  // in-kernel Q quantization: every softmax thread wrote its Q_hat row
 };
 static_assert(sizeof(Bars) <= 1024, "barrier area");
 
@@ -193,8 +202,12 @@ template <int D, bool PREORDER, bool CAUSAL, int OUT, int XT, bool DEC>
 __global__ void __launch_bounds__(Cfg<D, PREORDER, DEC>::THREADS, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
-    using C = Cfg<D, PREORDER, DEC>;
+    using C = Cfg<D, PREORDER, DEC, XT == 3>;
     constexpr int NQT = C::NQT;
+    constexpr bool BIAS = XT == 1 || XT == 2;            // score bias
+    constexpr bool DIAG = XT == 2;                       // P_hat dump, tile sums
+    constexpr bool QRAW = XT == 3;                       // Q quantized in this kernel
+    static_assert(!QRAW || (D == 128 && !DEC), "in-kernel Q quantization: D = 128, plain mode");
     constexpr int STK = C::STK, STV = C::STV;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -300,6 +313,7 @@ __global__ void __launch_bounds__(Cfg<D, PREORDER, DEC>::THREADS, 1)
     if (threadIdx.x == 0) {
         HIFA4_TRACE_POINT(4, 63, 0);
         mbar_init(&bars->q_full, 1);
+        mbar_init(&bars->q_ready, 128 * NQT);
         for (int s = 0; s < kMaxStages; ++s) {
             mbar_init(&bars->k_full[s], 1);
             mbar_init(&bars->v_full[s], 1);
@@ -485,8 +499,18 @@ __global__ void __launch_bounds__(Cfg<D, PREORDER, DEC>::THREADS, 1)
         // tile that read the previous load in it has released it.
         grid_dependency_wait();
         if (lane == 0 && !p.stall_loads) {
-            const int nq_load = DEC ? 1 : n_qt;
-            mbar_arrive_expect_tx(&bars->q_full, nq_load * (C::Q_BYTES + C::SFQK_BYTES));
+            const int nq_load = QRAW ? 0 : (DEC ? 1 : n_qt);
+            if constexpr (QRAW) {
+                // the caller's Q tiles (rows of D = 128 bf16 / fp16, 256 bytes) as
+                // two 128-byte column halves each; rows past the tensor read as 0
+                mbar_arrive_expect_tx(&bars->q_full, n_qt * 2 * C::QRAW_HALF);
+                for (int qt = 0; qt < n_qt; ++qt)
+                    for (int h = 0; h < 2; ++h)
+                        tma_load_2d(smem + C::OFF_QRAW + (qt * 2 + h) * C::QRAW_HALF, &tmQ, 128 * h,
+                                    grp * rows_in_grp + (t0 + qt) * 128, &bars->q_full);
+            } else {
+                mbar_arrive_expect_tx(&bars->q_full, nq_load * (C::Q_BYTES + C::SFQK_BYTES));
+            }
             for (int qt = 0; qt < nq_load; ++qt) {
                 tma_load_2d(smem + C::OFF_Q + qt * C::Q_BYTES, &tmQ, 0, grp * rows_in_grp + (t0 + qt) * 128,
                             &bars->q_full);
@@ -553,7 +577,7 @@ __global__ void __launch_bounds__(Cfg<D, PREORDER, DEC>::THREADS, 1)
         // an S tile has loaded it (named barrier "scores loaded" of that
         // warpgroup, which arrives without waiting) the next S MMA is issued.
         // A warp blocked in a named barrier takes no issue slots.
-        bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(&bars->q_full, 0, ctl));
+        bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(QRAW ? &bars->q_ready : &bars->q_full, 0, ctl));
         int j = 0, x = 0;
         bool more = next_item(0, -1, j, x);
         // the loads the first step reads (plain: load 0; decode: loads 0..3)
@@ -694,11 +718,88 @@ __global__ void __launch_bounds__(Cfg<D, PREORDER, DEC>::THREADS, 1)
         const uint32_t lut_s = smem_u32(lut);
         float m_old = -INFINITY, mc_old = 0.0f, l_hp = 0.0f;
         bool ok = true;                                     // false once a wait gave up (then no more work)
-        // XT >= 1: the score bias of a step's kv tile is staged in shared memory
+        if constexpr (QRAW) {
+            // this row of the query tile, from the caller's Q staged in shared
+            // memory: RN(x * s), per 16 elements sf = E4M3(amax * RN(1/6)), codes
+            // E2M1(RN(x * RN(1/sf))) (the quantize pass's rule), into the Q_hat
+            // tile (64-byte K-major rows, 64B swizzle) and the MMA-ready scale
+            // atoms; then arrive on q_ready (also after a failed wait).
+            ok = __all_sync(0xFFFFFFFFu, mbar_wait(&bars->q_full, 0, ctl));
+            uint32_t w[16];
+            uint32_t sfa[2] = {0u, 0u};
+#pragma unroll
+            for (int i = 0; i < 16; ++i) w[i] = 0u;
+            if (ok && valid) {
+                const float* sc = p.q_scale != nullptr ? p.q_scale + (size_t)(grp % p.Hkv) * D : nullptr;
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {   // 64 elements (4 blocks) at a time
+                    // 128-byte swizzle: 16-byte chunk c of row r sits at chunk c ^ (r % 8)
+                    const uint32_t rb = sbase + C::OFF_QRAW + (qt * 2 + half) * C::QRAW_HALF + row * 128;
+                    uint4 raw[8];
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        const float4 f4 = lds_v4f(rb + ((c ^ (row & 7)) << 4));
+                        raw[c] = make_uint4(__float_as_uint(f4.x), __float_as_uint(f4.y), __float_as_uint(f4.z),
+                                            __float_as_uint(f4.w));
+                    }
+#pragma unroll
+                    for (int bb = 0; bb < 4; ++bb) {
+                        const int b = 4 * half + bb;
+                        float x[16];
+#pragma unroll
+                        for (int h = 0; h < 2; ++h) {
+                            const uint32_t* u = reinterpret_cast<const uint32_t*>(&raw[2 * bb + h]);
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                float2 f;
+                                if (p.q_bf16) {
+                                    f = make_float2(__uint_as_float(u[e] << 16), __uint_as_float(u[e] & 0xFFFF0000u));
+                                } else {
+                                    f = __half22float2(*reinterpret_cast<const __half2*>(&u[e]));
+                                }
+                                x[8 * h + 2 * e] = f.x;
+                                x[8 * h + 2 * e + 1] = f.y;
+                            }
+                        }
+                        if (sc != nullptr) {
+                            const float4* s4 = reinterpret_cast<const float4*>(sc + 16 * b);
+#pragma unroll
+                            for (int q = 0; q < 4; ++q) {
+                                const float4 v = __ldg(s4 + q);
+                                x[4 * q] = __fmul_rn(x[4 * q], v.x);
+                                x[4 * q + 1] = __fmul_rn(x[4 * q + 1], v.y);
+                                x[4 * q + 2] = __fmul_rn(x[4 * q + 2], v.z);
+                                x[4 * q + 3] = __fmul_rn(x[4 * q + 3], v.w);
+                            }
+                        }
+                        float amax = 0.0f;
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) amax = fmaxf(amax, fabsf(x[e]));
+                        const uint32_t sf = cvt_e4m3(__fmul_rn(amax, rn_one_sixth()));
+                        const float r = lds_f32(smem_u32(lut) + 4u * (sf & 127u));
+                        float y[16];
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) y[e] = __fmul_rn(x[e], r);
+                        w[2 * b] = cvt_e2m1x8(y[0], y[1], y[2], y[3], y[4], y[5], y[6], y[7]);
+                        w[2 * b + 1] = cvt_e2m1x8(y[8], y[9], y[10], y[11], y[12], y[13], y[14], y[15]);
+                        sfa[b >> 2] |= sf << (8 * (b & 3));
+                    }
+                }
+            }
+            const uint32_t qb = sbase + C::OFF_Q + qt * C::Q_BYTES;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) sts_v4(qb + p_swizzle64(row, q), w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+            const uint32_t ao = 16u * (row & 31) + 4u * (row >> 5);       // row's word in a scale atom
+#pragma unroll
+            for (int a = 0; a < 2; ++a) sts_u32(sbase + C::OFF_SFQ + qt * C::SFQK_BYTES + 512 * a + ao, sfa[a]);
+            fence_proxy_async_smem();
+            mbar_arrive(&bars->q_ready);
+        }
+        // XT = 1, 2: the score bias of a step's kv tile is staged in shared memory
         // one step ahead, a warp at a time: lane l loads 4 of the 128 values of
         // each head the warp's rows belong to (at most two: Nq >= 16), and every
         // row then reads its head's 128 values back as broadcast loads.
-        const bool use_bias = XT >= 1 && p.s_bias != nullptr;
+        const bool use_bias = BIAS && p.s_bias != nullptr;
         const int my_head = valid ? (int)(out_row / (size_t)p.Nq) : -1;
         const int head0 = __shfl_sync(0xFFFFFFFFu, my_head, 0);
         const int head1 = __reduce_max_sync(0xFFFFFFFFu, my_head);
@@ -724,7 +825,7 @@ __global__ void __launch_bounds__(Cfg<D, PREORDER, DEC>::THREADS, 1)
                 __syncwarp();
             }
         };
-        if constexpr (XT >= 1) {
+        if constexpr (BIAS) {
             // the bias is written by the previous kernel of the stream: read it
             // only once that kernel has completed (programmatic dependent launch)
             if (use_bias) grid_dependency_wait();
@@ -760,7 +861,7 @@ __global__ void __launch_bounds__(Cfg<D, PREORDER, DEC>::THREADS, 1)
                 // (decode: a row whose range has ended masks the whole step)
                 const int n0 = (kt0 + j) * 128;
                 const int lim = j < own_steps ? last : -1;
-                if constexpr (XT >= 1) {
+                if constexpr (BIAS) {
                     load_bias(j + 1);
                     if (use_bias && my_head >= 0 && j < own_steps) {
                         const uint32_t bp = bias_s + (uint32_t)(j & 1) * 1024u + (my_head != head0 ? 512u : 0u);
@@ -797,7 +898,7 @@ __global__ void __launch_bounds__(Cfg<D, PREORDER, DEC>::THREADS, 1)
                 for (int e = 0; e < 64; ++e) {
                     const float2 t = __ffma2_rn(S[e], c2, nmc2);
                     S[e] = make_float2(ex2_approx(t.x), ex2_approx(t.y));
-                    if constexpr (!PREORDER || XT == 2) lsum2 = __fadd2_rn(lsum2, S[e]);
+                    if constexpr (!PREORDER || DIAG) lsum2 = __fadd2_rn(lsum2, S[e]);
                 }
                 uint32_t code[16];
                 uint32_t sfw[2] = {0u, 0u};
@@ -864,7 +965,7 @@ __global__ void __launch_bounds__(Cfg<D, PREORDER, DEC>::THREADS, 1)
                     tmem_st1(tl + C::COL_SFP + qt * 8 + wq, sfw[0]);
                     tmem_st1(tl + C::COL_SFP + qt * 8 + 4 + wq, sfw[1]);
                     tmem_wait_st();
-                    if constexpr (XT == 2) {
+                    if constexpr (DIAG) {
                         // per-tile mass of P_hat (codes x scales) and of P
                         if (p.tile_sums != nullptr && valid && j < own_steps) {
                             float sh = 0.0f;
@@ -890,7 +991,7 @@ __global__ void __launch_bounds__(Cfg<D, PREORDER, DEC>::THREADS, 1)
                 tc_fence_before();
                 m_old = m_new;
                 mc_old = mc_new;
-                if constexpr (XT >= 1) stage_bias(j + 1);
+                if constexpr (BIAS) stage_bias(j + 1);
             }
             // every row's P_hat is in shared memory and its O is rescaled: PV
             if (ok) named_barrier_arrive(id_p, 160); else named_barrier_sync(id_p, 160);
@@ -1008,7 +1109,7 @@ __global__ void __launch_bounds__(Cfg<D, PREORDER, DEC>::THREADS, 1)
 template <int D, bool PRE, bool CAUSAL, int OUT, int XT, bool DEC>
 static cudaError_t launch_one(const CUtensorMap* q, const CUtensorMap* k, const CUtensorMap* v, const AttnParams& p,
                               cudaStream_t st) {
-    using C = Cfg<D, PRE, DEC>;
+    using C = Cfg<D, PRE, DEC, XT == 3>;
     auto kern = attn_fwd_kernel<D, PRE, CAUSAL, OUT, XT, DEC>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
@@ -1038,39 +1139,46 @@ static cudaError_t launch_dec(const CUtensorMap* q, const CUtensorMap* k, const 
 
 template <int D, bool PRE, bool CAUSAL, int OUT>
 static cudaError_t launch_extras(const CUtensorMap* q, const CUtensorMap* k, const CUtensorMap* v,
-                                 const AttnParams& p, bool extras, bool dec, cudaStream_t st) {
-    if (!extras) return launch_dec<D, PRE, CAUSAL, OUT, 0>(q, k, v, p, dec, st);
-    if (p.p_codes == nullptr && p.tile_sums == nullptr) return launch_dec<D, PRE, CAUSAL, OUT, 1>(q, k, v, p, dec, st);
-    return launch_dec<D, PRE, CAUSAL, OUT, 2>(q, k, v, p, dec, st);
+                                 const AttnParams& p, int xt, bool dec, cudaStream_t st) {
+    switch (xt) {
+        case 0: return launch_dec<D, PRE, CAUSAL, OUT, 0>(q, k, v, p, dec, st);
+        case 1: return launch_dec<D, PRE, CAUSAL, OUT, 1>(q, k, v, p, dec, st);
+        case 2: return launch_dec<D, PRE, CAUSAL, OUT, 2>(q, k, v, p, dec, st);
+        default:
+            if constexpr (D == 128) {
+                if (!dec) return launch_one<D, PRE, CAUSAL, OUT, 3, false>(q, k, v, p, st);
+            }
+            return cudaErrorInvalidValue;
+    }
 }
 
 template <int D, bool PRE, bool CAUSAL>
 static cudaError_t launch_out(const CUtensorMap* q, const CUtensorMap* k, const CUtensorMap* v, const AttnParams& p,
-                              int out, bool extras, bool dec, cudaStream_t st) {
+                              int out, int xt, bool dec, cudaStream_t st) {
     switch (out) {
-        case 0: return launch_extras<D, PRE, CAUSAL, 0>(q, k, v, p, extras, dec, st);
-        case 1: return launch_extras<D, PRE, CAUSAL, 1>(q, k, v, p, extras, dec, st);
-        default: return launch_extras<D, PRE, CAUSAL, 2>(q, k, v, p, extras, dec, st);
+        case 0: return launch_extras<D, PRE, CAUSAL, 0>(q, k, v, p, xt, dec, st);
+        case 1: return launch_extras<D, PRE, CAUSAL, 1>(q, k, v, p, xt, dec, st);
+        default: return launch_extras<D, PRE, CAUSAL, 2>(q, k, v, p, xt, dec, st);
     }
 }
 
 template <int D>
 static cudaError_t launch_d(const CUtensorMap* q, const CUtensorMap* k, const CUtensorMap* v, const AttnParams& p,
-                            int norm, bool causal, int out, bool extras, bool dec, cudaStream_t st) {
+                            int norm, bool causal, int out, int xt, bool dec, cudaStream_t st) {
     if (norm == 0)
-        return causal ? launch_out<D, true, true>(q, k, v, p, out, extras, dec, st)
-                      : launch_out<D, true, false>(q, k, v, p, out, extras, dec, st);
-    return causal ? launch_out<D, false, true>(q, k, v, p, out, extras, dec, st)
-                  : launch_out<D, false, false>(q, k, v, p, out, extras, dec, st);
+        return causal ? launch_out<D, true, true>(q, k, v, p, out, xt, dec, st)
+                      : launch_out<D, true, false>(q, k, v, p, out, xt, dec, st);
+    return causal ? launch_out<D, false, true>(q, k, v, p, out, xt, dec, st)
+                  : launch_out<D, false, false>(q, k, v, p, out, xt, dec, st);
 }
 
 cudaError_t launch_attention(const CUtensorMap* tmQ, const CUtensorMap* tmK, const CUtensorMap* tmV,
-                             const AttnParams& p, int D, int norm, bool causal, int out_dtype, bool extras, bool dec,
+                             const AttnParams& p, int D, int norm, bool causal, int out_dtype, int xt, bool dec,
                              cudaStream_t st) {
     switch (D) {
-        case 64: return launch_d<64>(tmQ, tmK, tmV, p, norm, causal, out_dtype, extras, dec, st);
-        case 128: return launch_d<128>(tmQ, tmK, tmV, p, norm, causal, out_dtype, extras, dec, st);
-        case 256: return launch_d<256>(tmQ, tmK, tmV, p, norm, causal, out_dtype, extras, dec, st);
+        case 64: return launch_d<64>(tmQ, tmK, tmV, p, norm, causal, out_dtype, xt, dec, st);
+        case 128: return launch_d<128>(tmQ, tmK, tmV, p, norm, causal, out_dtype, xt, dec, st);
+        case 256: return launch_d<256>(tmQ, tmK, tmV, p, norm, causal, out_dtype, xt, dec, st);
         default: return cudaErrorInvalidValue;
     }
 }

@@ -64,6 +64,9 @@ struct AttnParams {
     uint8_t* p_codes;        // P_hat dump [B*Hq*Nq, Nkv/2]
     uint8_t* p_sf;           // ... and its scales [B*Hq*Nq, Nkv/16]
     float2* tile_sums;       // (sum P_hat, sum P) per (row, kv tile) [B*Hq*Nq, Nkv/128]
+    // in-kernel Q quantization (variant 3; Q itself comes through the Q tensor map)
+    const float* q_scale;    // Smooth-QK factors [Hkv, D] or null
+    int q_bf16;
     uint32_t* status;        // workspace status word
     int B, Hq, Hkv, Nq, Nkv, G;
     int Tq;                  // 128-row tiles per (b, kv head) group
@@ -76,11 +79,12 @@ struct AttnParams {
 };
 
 // D in {64,128,256}; norm 0 = P-Reordering, 1 = high-precision l;
-// out_dtype 0 = f16, 1 = bf16, 2 = f32; extras: the variant that reads s_bias
-// and writes p_codes / p_sf / tile_sums where they are non-null; dec: split-kv decode mode (D <= 128,
+// out_dtype 0 = f16, 1 = bf16, 2 = f32; xt: 0 the plain variant, 1 adds
+// s_bias, 2 also writes p_codes / p_sf / tile_sums where they are non-null,
+// 3 quantizes Q itself, reading the caller's Q through tmQ (D = 128, not dec); dec: split-kv decode mode (D <= 128,
 // G*Nq <= 64, at least 4 kv tiles; one CTA per group).
 cudaError_t launch_attention(const CUtensorMap* tmQ, const CUtensorMap* tmK, const CUtensorMap* tmV,
-                             const AttnParams& p, int D, int norm, bool causal, int out_dtype, bool extras, bool dec,
+                             const AttnParams& p, int D, int norm, bool causal, int out_dtype, int xt, bool dec,
                              cudaStream_t st);
 
 // Per-tile epsilon-bar from the attention kernel's tile sums.

@@ -266,6 +266,22 @@ hifa4_status hifa4_attention_fwd_ex(const hifa4_packed* in, int B, int Hq, int H
                                     void* o, hifa4_dtype o_dtype, float* lse,
                                     const hifa4_attention_extras* extras, void* workspace, hifa4_stream_t stream);
 
+/* hifa4_attention_fwd with Q given unquantized: q [B,Hq,Nq,D] in q_dtype (F16
+ * or BF16) and, optionally, the Smooth-QK factors s [Hkv,D] (NULL: no
+ * smoothing). The kernel quantizes each query row itself when it starts, with
+ * the rule and result of hifa4_quantize_qkv (Q' = RN(Q*s), per 16 elements
+ * sf = E4M3(amax * RN(1/6)), code = E2M1(RN(x * RN(1/sf)))), so O and LSE
+ * equal those of hifa4_quantize_qkv + hifa4_attention_fwd bit for bit; the
+ * packed Q is never written to memory. kv: the packed K and V (kc, ks, vtc,
+ * vts; qc and qs are ignored), e.g. from hifa4_quantize_kv or a cache filled
+ * by hifa4_append_kv. D must be 128 and the call must not select the split-kv
+ * decode mode (HIFA4_ERR_UNSUPPORTED otherwise). Other arguments as for
+ * hifa4_attention_fwd. */
+hifa4_status hifa4_attention_fwd_q(const void* q, hifa4_dtype q_dtype, const float* s, const hifa4_packed* kv,
+                                   int B, int Hq, int Hkv, int Nq, int Nkv, int D, float sm_scale, unsigned flags,
+                                   hifa4_norm_mode norm, void* o, hifa4_dtype o_dtype, float* lse,
+                                   void* workspace, hifa4_stream_t stream);
+
 /* Epsilon-bar per tile (HiFA4 abstract: the net probability-mass change of
  * quantizing P, median -0.064 over the Qwen3-8B trace's tiles). A tile is 128
  * query rows (the last one of a head may be shorter) of one (b,h) x one

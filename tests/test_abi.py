@@ -161,3 +161,20 @@ def test_extension_calls_validate_on_the_host(lib):
     assert ax(ctypes.byref(L.AttentionExtras(None, None, None, odd))) == L.ERR_INVALID_ARG
     assert lib.hifa4_tile_stats(fake, 1, 2, 128, 100, fake, None) == L.ERR_INVALID_ARG
     assert lib.hifa4_tile_stats(None, 1, 2, 128, 128, fake, None) == L.ERR_INVALID_ARG
+
+
+def test_in_kernel_q_entry_point_validates_on_the_host(lib):
+    from bit_quantized_flashattention_b200 import _lib as L
+    fake = ctypes.c_void_p(1 << 20)
+    pk = L.Packed(*([fake] * 6))
+
+    def call(q=fake, dt=None, D=128, Nq=128, Nkv=256, flags=0, Hq=2, Hkv=1, B=1):
+        return lib.hifa4_attention_fwd_q(q, L.BF16 if dt is None else dt, None, ctypes.byref(pk), B, Hq, Hkv, Nq, Nkv,
+                                         D, ctypes.c_float(0.1), flags, 0, fake, L.F32, None, fake, None)
+
+    assert call(q=None) == L.ERR_INVALID_ARG
+    assert call(dt=L.F32) == L.ERR_INVALID_ARG
+    assert call(q=ctypes.c_void_p((1 << 20) + 8)) == L.ERR_INVALID_ARG
+    assert call(D=64) == L.ERR_UNSUPPORTED                                  # D = 128 only
+    assert call(Nkv=100) == L.ERR_UNSUPPORTED
+    assert call(Hq=8, Hkv=2, Nq=16, Nkv=512, flags=L.SPLIT_KV) == L.ERR_UNSUPPORTED   # would take the decode mode

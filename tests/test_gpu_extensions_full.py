@@ -12,6 +12,9 @@ sampled (batch, kv head) groups, query rows and tiles.
   KV-cache appends on the decode workload's cache (B = 64, 8192 slots):
       appended chunks byte-identical to the whole-cache quantization, and the
       oracle's codes on sampled groups.
+  Attention with Q quantized in the kernel on the Qwen3-8B workload: O and
+      LSE equal the packed path's bit for bit, every row (the packed path is
+      oracle-checked on every row in test_gpu_configs.py).
 """
 import numpy as np
 import pytest
@@ -174,3 +177,18 @@ def test_append_full_size(H):
         assert np.array_equal(ks_all[b, g], ks[0, 0])
         vt = U.canonical_vtc(cache.vtc.view(cfg.B, cfg.Hkv, -1)[b, g], 1, 1, cfg.Nkv, cfg.D)[0, 0]
         assert np.array_equal(vt, vtc[0, 0]) and np.array_equal(vts_all[b, g], vts[0, 0])
+
+
+def test_in_kernel_q_quantization_full_size(H):
+    """The Qwen3-8B workload through hifa4_attention_fwd_q (Q quantized in the
+    attention kernel) equals quantize_qkv + attention_fwd bit for bit, every row."""
+    cfg = W.get(2)
+    q, k, v, calib = U.upload_config(cfg)
+    s, s_inv = H.calibrate_smooth(calib[0], calib[1], cfg.alpha)
+    pk = H.quantize_qkv(q, k, v, s, s_inv)
+    kv = H.quantize_kv(k, v, s_inv, Hq=cfg.Hq, Nq=cfg.Nq)
+    for norm in cfg.modes:
+        o_ref, l_ref = H.attention_fwd(pk, causal=True, norm=norm)
+        o, lse = H.attention_fwd_q(q, kv, s, causal=True, norm=norm)
+        torch.cuda.synchronize()
+        assert torch.equal(o, o_ref) and torch.equal(lse, l_ref), norm

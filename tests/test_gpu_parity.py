@@ -275,3 +275,37 @@ def test_attention_split_kv_matches_oracle(H, shape, causal, norm):
     ref = oracle.attention_rows(shape, oracle.all_rows(B, Hq, Nq), packed=ref_p, causal=causal,
                                 norm_mode=0 if norm == "p_reorder" else 1, want_p=True, n_splits=n_splits)
     _check_attention(o, lse, pc, ps, ref, D)
+
+
+@pytest.mark.parametrize("shape,causal,dtype,smooth", [
+    ((1, 4, 2, 384, 384, 128), True, "bf16", True),
+    ((2, 4, 2, 176, 512, 128), True, "bf16", False),       # G*Nq = 352: tiles mix heads, ragged last tile
+    ((1, 2, 1, 256, 384, 128), False, "fp16", True),
+    ((1, 8, 2, 16, 512, 128), False, "bf16", True),         # decode-style rows, one pass
+])
+@pytest.mark.parametrize("norm", ["p_reorder", "high_precision_l"])
+def test_attention_with_in_kernel_q_quantization(H, shape, causal, dtype, smooth, norm):
+    """hifa4_attention_fwd_q quantizes Q inside the attention kernel with the
+    quantize pass's rule: O and LSE equal those of quantize_qkv + attention_fwd
+    bit for bit, and therefore the oracle within the attention bars."""
+    B, Hq, Hkv, Nq, Nkv, D = shape
+    rng = np.random.default_rng(19)
+    q = W.round_to_dtype(_rand(rng, (B, Hq, Nq, D), 1.5), dtype)
+    k = W.round_to_dtype(_rand(rng, (B, Hkv, Nkv, D)) * rng.lognormal(0, 1, (1, Hkv, 1, D)).astype(np.float32), dtype)
+    v = W.round_to_dtype(_rand(rng, (B, Hkv, Nkv, D)), dtype)
+    s, si = oracle.calibrate(q, k) if smooth else (None, None)
+    dq, dk, dv = (U.to_device(x, dtype) for x in (q, k, v))
+    ds = None if s is None else torch.from_numpy(s).cuda()
+    dsi = None if si is None else torch.from_numpy(si).cuda()
+    pk = H.quantize_qkv(dq, dk, dv, ds, dsi)
+    o_ref, l_ref = H.attention_fwd(pk, causal=causal, norm=norm, out_dtype=torch.float32)
+    kv = H.quantize_kv(dk, dv, dsi, Hq=Hq, Nq=Nq)
+    o, lse = H.attention_fwd_q(dq, kv, ds, causal=causal, norm=norm, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert torch.equal(o, o_ref) and torch.equal(lse, l_ref)
+    if shape == (1, 4, 2, 384, 384, 128):
+        ref = oracle.attention_rows(shape, oracle.all_rows(B, Hq, Nq), packed=oracle.quantize_qkv(q, k, v, s, si),
+                                    causal=causal, norm_mode=0 if norm == "p_reorder" else 1)
+        max_abs, rel = U.row_errors(o.cpu().numpy().reshape(-1, D), ref["O"])
+        assert max_abs <= O_MAX_ABS and rel.max() <= O_ROW_REL
+        assert np.abs(lse.cpu().numpy().ravel() - ref["lse"]).max() <= LSE_ABS
