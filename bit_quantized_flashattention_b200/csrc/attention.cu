@@ -725,11 +725,15 @@ __global__ void __launch_bounds__(Cfg<D, PREORDER, DEC>::THREADS, 1)
             // tile (64-byte K-major rows, 64B swizzle) and the MMA-ready scale
             // atoms; then arrive on q_ready (also after a failed wait).
             ok = __all_sync(0xFFFFFFFFu, mbar_wait(&bars->q_full, 0, ctl));
+            HIFA4_TRACE_POINT(qt, 61, 0);
             uint32_t w[16];
             uint32_t sfa[2] = {0u, 0u};
 #pragma unroll
             for (int i = 0; i < 16; ++i) w[i] = 0u;
             if (ok && valid) {
+                // the smoothing factors may come from the previous kernel of the
+                // stream: read them only once it has completed
+                if (p.q_scale != nullptr) grid_dependency_wait();
                 const float* sc = p.q_scale != nullptr ? p.q_scale + (size_t)(grp % p.Hkv) * D : nullptr;
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {   // 64 elements (4 blocks) at a time
@@ -794,6 +798,7 @@ __global__ void __launch_bounds__(Cfg<D, PREORDER, DEC>::THREADS, 1)
             for (int a = 0; a < 2; ++a) sts_u32(sbase + C::OFF_SFQ + qt * C::SFQK_BYTES + 512 * a + ao, sfa[a]);
             fence_proxy_async_smem();
             mbar_arrive(&bars->q_ready);
+            HIFA4_TRACE_POINT(qt, 61, 1);
         }
         // XT = 1, 2: the score bias of a step's kv tile is staged in shared memory
         // one step ahead, a warp at a time: lane l loads 4 of the 128 values of
