@@ -19,6 +19,11 @@ namespace {
 
 constexpr unsigned long long kDefaultWaitNs = 2000000000ull;   // 2 s
 std::atomic<long long> g_wait_limit_ns{0};
+
+unsigned long long wait_limit_ns() {
+    const long long lim = g_wait_limit_ns.load();
+    return lim > 0 ? (unsigned long long)lim : kDefaultWaitNs;
+}
 std::atomic<int> g_stall_loads{0};
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -196,8 +201,7 @@ hifa4_status attention_impl(const hifa4_packed* in, int B, int Hq, int Hkv, int 
     p.n_work = (int)n_work;
     p.heavy_first = (!dec && causal && Nq % (128 * nqt) == 0) ? 1 : 0;
     p.c = (float)((double)sm_scale * 1.4426950408889634074);
-    const long long lim = g_wait_limit_ns.load();
-    p.wait_limit_ns = lim > 0 ? (unsigned long long)lim : kDefaultWaitNs;
+    p.wait_limit_ns = wait_limit_ns();
     p.stall_loads = g_stall_loads.load();
     const int out = o_dtype == HIFA4_F16 ? 0 : (o_dtype == HIFA4_BF16 ? 1 : 2);
     return from_cuda(launch_attention(&tq, &tk, &tv, p, D, (int)norm, causal, out, xt, dec,
@@ -281,6 +285,7 @@ hifa4_status hifa4_quantize_qkv_ex(const void* q, const void* k, const void* v, 
     a.ks = static_cast<uint8_t*>(out->ks);
     a.vtc = static_cast<uint8_t*>(out->vtc);
     a.vts = static_cast<uint8_t*>(out->vts);
+    a.wait_limit_ns = wait_limit_ns();
     return from_cuda(launch_quantize_qkv(a, reinterpret_cast<cudaStream_t>(stream)));
 }
 
@@ -330,6 +335,7 @@ hifa4_status hifa4_append_kv(const void* k, const void* v, hifa4_dtype dtype, in
     a.ks = static_cast<uint8_t*>(cache->ks);
     a.vtc = static_cast<uint8_t*>(cache->vtc);
     a.vts = static_cast<uint8_t*>(cache->vts);
+    a.wait_limit_ns = wait_limit_ns();
     return from_cuda(launch_quantize_qkv(a, reinterpret_cast<cudaStream_t>(stream)));
 }
 
@@ -446,8 +452,7 @@ hifa4_status hifa4_attention_fwd_q(const void* q, hifa4_dtype q_dtype, const flo
     p.n_work = (int)n_work;
     p.heavy_first = (causal && Nq % (128 * nqt) == 0) ? 1 : 0;
     p.c = (float)((double)sm_scale * 1.4426950408889634074);
-    const long long lim = g_wait_limit_ns.load();
-    p.wait_limit_ns = lim > 0 ? (unsigned long long)lim : kDefaultWaitNs;
+    p.wait_limit_ns = wait_limit_ns();
     p.stall_loads = g_stall_loads.load();
     const int out = o_dtype == HIFA4_F16 ? 0 : (o_dtype == HIFA4_BF16 ? 1 : 2);
     return from_cuda(launch_attention(&tq, &tk, &tv, p, D, (int)norm, causal, out, 3, false,
@@ -468,10 +473,12 @@ hifa4_status hifa4_get_status(void* workspace, hifa4_stream_t stream) {
     if (workspace == nullptr) return HIFA4_ERR_INVALID_ARG;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if (from_cuda(cudaStreamSynchronize(st)) != HIFA4_OK) return HIFA4_ERR_CUDA;
-    uint32_t word = 0;
+    uint32_t word = 0, qword = 0;
     if (from_cuda(cudaMemcpy(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost)) != HIFA4_OK)
         return HIFA4_ERR_CUDA;
     if (word != 0 && from_cuda(cudaMemset(workspace, 0, sizeof(word))) != HIFA4_OK) return HIFA4_ERR_CUDA;
+    if (from_cuda(take_quantize_status(&qword)) != HIFA4_OK) return HIFA4_ERR_CUDA;
+    if (word == 0) word = qword;
     return word == 0 ? HIFA4_OK : (hifa4_status)word;
 }
 

@@ -93,7 +93,8 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const 
     }
 }
 
-// Wait that ignores the abort flag (used while draining copies in flight).
+// Bounded wait that ignores the abort flag (copy completion, and draining
+// copies in flight before a CTA exits). False when the limit passed.
 __device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
     const uint64_t t0 = global_timer_ns();
     while (!mbar_try_wait(bar, parity)) {

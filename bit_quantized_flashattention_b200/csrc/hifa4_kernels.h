@@ -31,9 +31,14 @@ struct QuantArgs {
     const float* q_mean;          // [B*Hq, D] or null
     float* s_bias;                // [B*Hq, nkv]
     uint8_t *qc, *qs, *kc, *ks, *vtc, *vts;
+    unsigned long long wait_limit_ns;   // bound of the copy waits of the row pass
 };
 
 cudaError_t launch_quantize_qkv(const QuantArgs& a, cudaStream_t st);
+
+// Synchronous: the quantize pass's status word (0, or HIFA4_ERR_TIMEOUT when
+// a bounded wait expired in it since the last call), then clears it.
+cudaError_t take_quantize_status(uint32_t* out);
 
 // Q-Mean: mean [B*Hq, D] of the pre-quantization Q (RoPE, smoothing as above).
 struct QMeanArgs {

@@ -18,6 +18,21 @@
 
 namespace hifa4 {
 
+// Set (to the timeout status) when a bounded wait of the row pass expires;
+// read and cleared by take_quantize_status.
+__device__ uint32_t g_quantize_status;
+
+cudaError_t take_quantize_status(uint32_t* out) {
+    uint32_t word = 0;
+    cudaError_t e = cudaMemcpyFromSymbol(&word, g_quantize_status, sizeof(word));
+    if (e == cudaSuccess && word != 0) {
+        const uint32_t zero = 0;
+        e = cudaMemcpyToSymbol(g_quantize_status, &zero, sizeof(zero));
+    }
+    *out = word;
+    return e;
+}
+
 template <typename T>
 __device__ __forceinline__ float to_f32(T x);
 template <>
@@ -43,21 +58,6 @@ __device__ __forceinline__ void build_rcp_lut(float* lut) {
     __syncthreads();
 }
 
-// Quantize 16 elements held by one thread (the rule in the file header).
-__device__ __forceinline__ uint32_t quant_block16_lut(const float (&x)[16], const float* lut, uint32_t& lo,
-                                                      uint32_t& hi) {
-    float amax = fabsf(x[0]);
-#pragma unroll
-    for (int i = 1; i < 16; ++i) amax = fmaxf(amax, fabsf(x[i]));
-    const uint32_t sf = cvt_e4m3(__fmul_rn(amax, rn_one_sixth()));
-    const float r = lut[sf & 127u];
-    float y[16];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) y[i] = __fmul_rn(x[i], r);
-    lo = cvt_e2m1x8(y[0], y[1], y[2], y[3], y[4], y[5], y[6], y[7]);
-    hi = cvt_e2m1x8(y[8], y[9], y[10], y[11], y[12], y[13], y[14], y[15]);
-    return sf;
-}
 
 // ------------------------------------------------- before quantization
 
@@ -79,21 +79,22 @@ __device__ __forceinline__ RopeChunk load_rope(const float* cos_t, const float* 
     return RopeChunk{__ldg(c4), __ldg(c4 + 1), __ldg(s4), __ldg(s4 + 1)};
 }
 
-// The rotation of one chunk, rotate-half pairing: channel d < D/2 pairs with
-// d + D/2, which sits in chunk c ^ (D/16) of the same row (a neighbouring lane
-// group: the row's D/8 chunks are consecutive lanes). Each product and sum is
+// The rotation of one 8-channel chunk, rotate-half pairing: channel d < D/2
+// pairs with d + D/2, which sits in chunk c ^ (D/16) of the same row, held by
+// the lane LANE_XOR away (D/16 when a lane holds one chunk of the row, D/32
+// when it holds two). Each product and sum is
 // rounded on its own (no fused multiply-add):
 //   first half   x <- RN(RN(x*cos) - RN(x_pair*sin))
 //   second half  x <- RN(RN(x*cos) + RN(x_pair*sin))
 // Every lane of the warp calls this (it shuffles).
-template <typename T, int D>
+template <typename T, int D, unsigned LANE_XOR = D / 16>
 __device__ __forceinline__ void rope_chunk(const uint4& raw, unsigned chunk, const RopeChunk& t, float (&v)[8]) {
     constexpr unsigned HALF = D / 16;
     uint4 pr;
-    pr.x = __shfl_xor_sync(0xFFFFFFFFu, raw.x, HALF);
-    pr.y = __shfl_xor_sync(0xFFFFFFFFu, raw.y, HALF);
-    pr.z = __shfl_xor_sync(0xFFFFFFFFu, raw.z, HALF);
-    pr.w = __shfl_xor_sync(0xFFFFFFFFu, raw.w, HALF);
+    pr.x = __shfl_xor_sync(0xFFFFFFFFu, raw.x, LANE_XOR);
+    pr.y = __shfl_xor_sync(0xFFFFFFFFu, raw.y, LANE_XOR);
+    pr.z = __shfl_xor_sync(0xFFFFFFFFu, raw.z, LANE_XOR);
+    pr.w = __shfl_xor_sync(0xFFFFFFFFu, raw.w, LANE_XOR);
     float w[8];
     unpack8<T>(pr, w);
     const float cs[8] = {t.c0.x, t.c0.y, t.c0.z, t.c0.w, t.c1.x, t.c1.y, t.c1.z, t.c1.w};
@@ -154,98 +155,162 @@ struct VJob {
     unsigned warps_per_group;
 };
 
-// Each lane owns one 8-element chunk of a row (a warp instruction reads 512
-// contiguous bytes); a CTA walks a contiguous range of its group's rows, four
-// row steps per iteration so that four loads per lane are in flight. The
-// lane's 8 smoothing factors stay in registers. The two halves of a
-// 16-element block sit in neighbouring lanes (one shuffle for the maximum),
-// and the 4 scale bytes of a 64-element K step are gathered by shuffles into
-// one 32-bit word of the MMA-ready atom. Before quantization, in order: RoPE
-// (ROPE variant), the smoothing multiply, the Q-Mean subtraction; on K rows
-// with bias_mean the Q-Mean score bias mean . K' of every head of the group is
-// reduced across the row's lanes from the same pre-quantization values.
+// A CTA quantizes a contiguous range of at most 4 row steps of its group (at
+// most 32 KB of input, contiguous in memory). One thread moves the range into
+// shared memory at the start with bulk copies, one per row step, each
+// completing its own mbarrier: the whole range is in flight at once, and the
+// arithmetic on a step starts as soon as it lands. Each lane owns one whole
+// 16-element scale block of a row (its maximum needs no shuffle) and keeps
+// that block's 16 smoothing factors in registers; products are formed two at
+// a time (packed fp32 multiplies, each lane rounded on its own). The 4 scale
+// bytes of a 64-element K step sit in 4 neighbouring lanes and are gathered by
+// two shuffles into one 32-bit word of the MMA-ready atom. Before
+// quantization, in order: RoPE (ROPE variant), the smoothing multiply, the
+// Q-Mean subtraction; on K rows with bias_mean the Q-Mean score bias mean . K'
+// of every head of the group is reduced across the row's lanes from the same
+// pre-quantization values.
+constexpr unsigned kRowStages = 4;                    // row steps (copy chunks) per CTA
+constexpr unsigned kRowStageBytes = 4u * 256u * 32u;  // 4 row steps x 256 lanes x 32 bytes
+
+// Sixteen values times sixteen factors, two at a time: v[i] <- RN(v[i] * f[i]).
+__device__ __forceinline__ void mul16(float (&v)[16], const float (&f)[16]) {
+#pragma unroll
+    for (int i = 0; i < 16; i += 2) unpack2(fmul2(pack2(v[i], v[i + 1]), pack2(f[i], f[i + 1])), v[i], v[i + 1]);
+}
+
+// Maximum of |v| over 16 values (three-input maxima; the maximum is exact).
+__device__ __forceinline__ float absmax16(const float (&v)[16]) {
+    float a[6];
+#pragma unroll
+    for (int i = 0; i < 5; ++i) a[i] = fmax3f(fabsf(v[3 * i]), fabsf(v[3 * i + 1]), fabsf(v[3 * i + 2]));
+    a[5] = fabsf(v[15]);
+    return fmax3f(fmax3f(a[0], a[1], a[2]), fmax3f(a[3], a[4], a[5]), 0.0f);
+}
+
+// Quantize 16 elements held by one thread (the rule in the file header).
+__device__ __forceinline__ uint32_t quant_block16_lut(float (&x)[16], const float* lut, uint32_t& lo, uint32_t& hi) {
+    const uint32_t sf = cvt_e4m3(__fmul_rn(absmax16(x), rn_one_sixth()));
+    const float r = lut[sf & 127u];
+    const float rr[16] = {r, r, r, r, r, r, r, r, r, r, r, r, r, r, r, r};
+    mul16(x, rr);
+    lo = cvt_e2m1x8(x[0], x[1], x[2], x[3], x[4], x[5], x[6], x[7]);
+    hi = cvt_e2m1x8(x[8], x[9], x[10], x[11], x[12], x[13], x[14], x[15]);
+    return sf;
+}
+
 template <typename T, int D, bool ROPE, bool QM>
-__device__ __forceinline__ void quantize_rows_cta(const RowJob& jb, unsigned cta, const float* lut) {
-    constexpr unsigned CPR = D / 8;                        // chunks per row
+__device__ __forceinline__ void quantize_rows_cta(const RowJob& jb, unsigned cta, const float* lut, uint8_t* stage,
+                                                  uint64_t* bars, unsigned long long limit_ns) {
+    constexpr unsigned CPR = D / 16;                       // lanes (scale blocks) per row
     constexpr unsigned RPB = 256 / CPR;                    // rows per CTA step
-    constexpr unsigned UNROLL = 4;
+    constexpr unsigned ROW_BYTES = D * sizeof(T);
     constexpr unsigned KS = D / 64;
     const unsigned grp = cta / jb.blocks_per_group;
     const unsigned part = cta % jb.blocks_per_group;
-    const unsigned c = threadIdx.x % CPR;
+    const unsigned c = threadIdx.x % CPR;                  // the lane's block of the row
     const unsigned steps = (jb.padded + RPB - 1) / RPB;
     const unsigned s0 = (unsigned)(((unsigned long long)steps * part) / jb.blocks_per_group);
     const unsigned s1 = (unsigned)(((unsigned long long)steps * (part + 1)) / jb.blocks_per_group);
-    float sc[8];
-    if (jb.scale != nullptr) load8(jb.scale + (size_t)(grp % jb.hkv) * D + c * 8, sc);
+    float sc[16];
+    if (jb.scale != nullptr) {
+        const float* sp = jb.scale + (size_t)(grp % jb.hkv) * D + c * 16;
+        float a[8], b[8];
+        load8(sp, a);
+        load8(sp + 8, b);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) { sc[i] = a[i]; sc[8 + i] = b[i]; }
+    }
     const T* xg = static_cast<const T*>(jb.x) + (size_t)grp * jb.rows_in * D;
     uint8_t* cg = jb.codes + ((size_t)grp * jb.rows_out + jb.row0) * (D / 2);
     uint8_t* sg = jb.sfs + (size_t)grp * jb.tiles_out * KS * 512;
     const unsigned r_in = threadIdx.x / CPR;
-    for (unsigned st = s0; st < s1; st += UNROLL) {
-        uint4 raw[UNROLL];
-#pragma unroll
-        for (unsigned u = 0; u < UNROLL; ++u) {
-            const unsigned pp = (st + u) * RPB + r_in;
-            const bool real = st + u < s1 && pp < jb.rows_in;
-            raw[u] = real ? *reinterpret_cast<const uint4*>(xg + (size_t)pp * D + c * 8) : make_uint4(0u, 0u, 0u, 0u);
+    const unsigned row_first = s0 * RPB;                   // first row of the range
+    if (threadIdx.x == 0) {
+        for (unsigned k = 0; k < kRowStages; ++k) {
+            const unsigned a = min(min(s0 + k, s1) * RPB, jb.rows_in);
+            const unsigned b = min(min(s0 + k + 1, s1) * RPB, jb.rows_in);
+            if (b > a) {
+                mbar_arrive_expect_tx(&bars[k], (b - a) * ROW_BYTES);
+                bulk_load(stage + (a - row_first) * ROW_BYTES, xg + (size_t)a * D, (b - a) * ROW_BYTES, &bars[k]);
+            } else {
+                mbar_arrive(&bars[k]);
+            }
         }
-#pragma unroll
-        for (unsigned u = 0; u < UNROLL; ++u) {
-            const unsigned p = (st + u) * RPB + r_in;
-            const bool in_range = st + u < s1;             // warp-uniform
-            const bool real = in_range && p < jb.rows_in;
-            float v[8];
-            unpack8<T>(raw[u], v);
+    }
+    for (unsigned st = s0, k = 0; st < s1; ++st, ++k) {
+        // step k has landed (bounded: on expiry the status is recorded, the
+        // remaining copies are drained and the CTA stops)
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait_drain(&bars[k], 0, limit_ns))) {
+            if (threadIdx.x == 0) {
+                atomicExch(&g_quantize_status, kStatusTimeout);
+                for (unsigned kk = k; kk < kRowStages; ++kk) mbar_wait_drain(&bars[kk], 0, limit_ns);
+            }
+            return;
+        }
+        const unsigned p = st * RPB + r_in;
+        const bool real = p < jb.rows_in;
+        uint4 raw0 = make_uint4(0u, 0u, 0u, 0u), raw1 = raw0;
+        if (real) {
+            const uint4* src = reinterpret_cast<const uint4*>(stage + (p - row_first) * ROW_BYTES + c * 32);
+            raw0 = src[0];
+            raw1 = src[1];
+        }
+        float v[16];
+        {
+            float a[8], b[8];
+            unpack8<T>(raw0, a);
+            unpack8<T>(raw1, b);
             if constexpr (ROPE) {
                 // the table rows are cache hits: loaded where they are used
-                const RopeChunk rc = load_rope<D>(jb.rope_cos, jb.rope_sin, jb.pos, real ? p % jb.n_tok : 0u, jb.n_pos, c);
-                rope_chunk<T, D>(raw[u], c, rc, v);
+                const unsigned tok = real ? p % jb.n_tok : 0u;
+                rope_chunk<T, D, D / 32>(raw0, 2 * c, load_rope<D>(jb.rope_cos, jb.rope_sin, jb.pos, tok, jb.n_pos, 2 * c), a);
+                rope_chunk<T, D, D / 32>(raw1, 2 * c + 1,
+                                         load_rope<D>(jb.rope_cos, jb.rope_sin, jb.pos, tok, jb.n_pos, 2 * c + 1), b);
             }
-            if (jb.scale != nullptr) {
 #pragma unroll
-                for (int i = 0; i < 8; ++i) v[i] = __fmul_rn(v[i], sc[i]);
-            }
-            if (QM && jb.mean != nullptr && real) {
-                float m[8];
-                load8(jb.mean + ((size_t)grp * jb.G + p / jb.n_tok) * D + c * 8, m);
-#pragma unroll
-                for (int i = 0; i < 8; ++i) v[i] = __fsub_rn(v[i], m[i]);
-            }
-            if (QM && jb.bias_mean != nullptr) {
-                // score bias of this key for every q head of the group
-                for (unsigned hl = 0; hl < jb.G; ++hl) {
-                    float acc = 0.0f;
-                    if (real) {
-                        float m[8];
-                        load8(jb.bias_mean + ((size_t)grp * jb.G + hl) * D + c * 8, m);
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) acc = __fmaf_rn(m[i], v[i], acc);
-                    }
-#pragma unroll
-                    for (unsigned o = CPR / 2; o >= 1; o >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, o);
-                    if (real && c == 0) jb.bias[((size_t)grp * jb.G + hl) * jb.rows_out + jb.row0 + p] = acc;
-                }
-            }
-            float amax = 0.0f;
-#pragma unroll
-            for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
-            amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
-            const uint32_t sf = cvt_e4m3(__fmul_rn(amax, rn_one_sixth()));
-            const float r = lut[sf & 127u];
-            float y[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) y[i] = __fmul_rn(v[i], r);
-            const uint32_t w = cvt_e2m1x8(y[0], y[1], y[2], y[3], y[4], y[5], y[6], y[7]);
-            if (real) *reinterpret_cast<uint32_t*>(cg + (size_t)p * (D / 2) + c * 4) = w;
-            uint32_t word = ((c & 1u) == 0u) ? (sf << (8u * ((c >> 1) & 3u))) : 0u;
-            word |= __shfl_xor_sync(0xFFFFFFFFu, word, 2);
-            word |= __shfl_xor_sync(0xFFFFFFFFu, word, 4);
-            const unsigned q = jb.row0 + p;                // output row
-            if (in_range && p < jb.padded && (c & 7u) == 0u)
-                *reinterpret_cast<uint32_t*>(sg + ((size_t)(q >> 7) * KS + c / 8) * 512 + atom_offset(q & 127u)) =
-                    real ? word : 0u;
+            for (int i = 0; i < 8; ++i) { v[i] = a[i]; v[8 + i] = b[i]; }
         }
+        if (jb.scale != nullptr) mul16(v, sc);
+        if (QM && jb.mean != nullptr && real) {
+            const float* mp = jb.mean + ((size_t)grp * jb.G + p / jb.n_tok) * D + c * 16;
+            float a[8], b[8];
+            load8(mp, a);
+            load8(mp + 8, b);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                v[i] = __fsub_rn(v[i], a[i]);
+                v[8 + i] = __fsub_rn(v[8 + i], b[i]);
+            }
+        }
+        if (QM && jb.bias_mean != nullptr) {
+            // score bias of this key for every q head of the group
+            for (unsigned hl = 0; hl < jb.G; ++hl) {
+                float acc = 0.0f;
+                if (real) {
+                    const float* mp = jb.bias_mean + ((size_t)grp * jb.G + hl) * D + c * 16;
+                    float a[8], b[8];
+                    load8(mp, a);
+                    load8(mp + 8, b);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) acc = __fmaf_rn(a[i], v[i], acc);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) acc = __fmaf_rn(b[i], v[8 + i], acc);
+                }
+#pragma unroll
+                for (unsigned o = CPR / 2; o >= 1; o >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, o);
+                if (real && c == 0) jb.bias[((size_t)grp * jb.G + hl) * jb.rows_out + jb.row0 + p] = acc;
+            }
+        }
+        uint32_t lo, hi;
+        const uint32_t sf = quant_block16_lut(v, lut, lo, hi);
+        if (real) *reinterpret_cast<uint2*>(cg + (size_t)p * (D / 2) + c * 8) = make_uint2(lo, hi);
+        uint32_t word = sf << (8u * (c & 3u));
+        word |= __shfl_xor_sync(0xFFFFFFFFu, word, 1);
+        word |= __shfl_xor_sync(0xFFFFFFFFu, word, 2);
+        const unsigned q = jb.row0 + p;                    // output row
+        if (p < jb.padded && (c & 3u) == 0u)
+            *reinterpret_cast<uint32_t*>(sg + ((size_t)(q >> 7) * KS + c / 4) * 512 + atom_offset(q & 127u)) =
+                real ? word : 0u;
     }
 }
 
@@ -322,17 +387,23 @@ __device__ __forceinline__ void quantize_v_warp(const VJob& jb, unsigned gw_all,
 // K rows, the rest V (8 warps per CTA).
 template <typename T, int D, bool ROPE, bool QM>
 __global__ void __launch_bounds__(256) quantize_qkv_kernel(RowJob q, RowJob k, VJob v, unsigned nq, unsigned nk,
-                                                           unsigned v_warps) {
+                                                           unsigned v_warps, unsigned long long limit_ns) {
     __shared__ float lut[128];
+    __shared__ uint64_t bars[kRowStages];
+    extern __shared__ __align__(128) uint8_t stage[];      // kRowStageBytes (row CTAs)
     // the next kernel (attention) may be scheduled as these CTAs retire; it
     // waits for this grid's completion before reading the packed operands
     launch_dependents();
-    build_rcp_lut(lut);
     const unsigned b = blockIdx.x;
+    if (threadIdx.x == 0 && b < nq + nk) {
+        for (unsigned i = 0; i < kRowStages; ++i) mbar_init(&bars[i], 1);
+        fence_barrier_init();
+    }
+    build_rcp_lut(lut);                                    // ends with a CTA barrier
     if (b < nq) {
-        quantize_rows_cta<T, D, ROPE, QM>(q, b, lut);
+        quantize_rows_cta<T, D, ROPE, QM>(q, b, lut, stage, bars, limit_ns);
     } else if (b < nq + nk) {
-        quantize_rows_cta<T, D, ROPE, QM>(k, b - nq, lut);
+        quantize_rows_cta<T, D, ROPE, QM>(k, b - nq, lut, stage, bars, limit_ns);
     } else {
         const unsigned gw = (b - nq - nk) * 8 + (threadIdx.x >> 5);
         if (gw < v_warps) quantize_v_warp<T, D>(v, gw, lut);
@@ -480,13 +551,13 @@ __global__ void calib_finalize_kernel(float* __restrict__ s, float* __restrict__
 template <typename T, int D>
 static cudaError_t launch_qkv_t(const QuantArgs& a, cudaStream_t st) {
     const long long n_grp = a.n_groups;
-    // small CTAs (at most 8 row steps of 256/(D/8) rows each): many CTAs per SM
-    // overlap one CTA's loads with another's arithmetic
-    const long long rows_per_step = 256 / (D / 8);
+    // small CTAs (at most kRowStages row steps of 256/(D/16) rows each): many
+    // CTAs per SM overlap one CTA's loads with another's arithmetic
+    const long long rows_per_step = 256 / (D / 16);
     auto per_group = [&](long long padded_rows) -> long long {
         if (padded_rows == 0) return 0;
         const long long steps = (padded_rows + rows_per_step - 1) / rows_per_step;
-        return (steps + 7) / 8;
+        return (steps + kRowStages - 1) / kRowStages;
     };
     const bool rope = a.rope_cos != nullptr;
     RowJob jq{};
@@ -544,7 +615,11 @@ static cudaError_t launch_qkv_t(const QuantArgs& a, cudaStream_t st) {
     const bool qm = a.q_mean != nullptr;
     auto kern = rope ? (qm ? quantize_qkv_kernel<T, D, true, true> : quantize_qkv_kernel<T, D, true, false>)
                      : (qm ? quantize_qkv_kernel<T, D, false, true> : quantize_qkv_kernel<T, D, false, false>);
-    kern<<<(unsigned)total, 256, 0, st>>>(jq, jk, jv, (unsigned)nq, (unsigned)nk, (unsigned)v_warps);
+    const int smem = (nq + nk > 0) ? (int)kRowStageBytes : 0;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kRowStageBytes);
+    if (e != cudaSuccess) return e;
+    kern<<<(unsigned)total, 256, smem, st>>>(jq, jk, jv, (unsigned)nq, (unsigned)nk, (unsigned)v_warps,
+                                              a.wait_limit_ns);
     return cudaGetLastError();
 }
 

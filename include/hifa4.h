@@ -322,7 +322,10 @@ hifa4_status hifa4_attention_fwd_noalloc(const hifa4_packed* in, int B, int Hq, 
 
 /* Synchronises `stream`, then returns the status a kernel recorded in
  * `workspace` (HIFA4_OK or HIFA4_ERR_TIMEOUT) or HIFA4_ERR_CUDA if the stream
- * reported an error. Clears the recorded status. */
+ * reported an error. Clears the recorded status. It also reports (as
+ * HIFA4_ERR_TIMEOUT) and clears the device-wide status word of the quantize
+ * passes (hifa4_quantize_qkv*, hifa4_quantize_kv, hifa4_append_kv), which a
+ * bounded wait for the pass's own input copies sets when it expires. */
 hifa4_status hifa4_get_status(void* workspace, hifa4_stream_t stream);
 
 /* Test hook for the timeout path: sets the wait limit (nanoseconds) that the
