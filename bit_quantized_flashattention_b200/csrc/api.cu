@@ -286,6 +286,7 @@ hifa4_status hifa4_quantize_qkv_ex(const void* q, const void* k, const void* v, 
     a.vtc = static_cast<uint8_t*>(out->vtc);
     a.vts = static_cast<uint8_t*>(out->vts);
     a.wait_limit_ns = wait_limit_ns();
+    a.stall_loads = g_stall_loads.load();
     return from_cuda(launch_quantize_qkv(a, reinterpret_cast<cudaStream_t>(stream)));
 }
 
@@ -336,6 +337,7 @@ hifa4_status hifa4_append_kv(const void* k, const void* v, hifa4_dtype dtype, in
     a.vtc = static_cast<uint8_t*>(cache->vtc);
     a.vts = static_cast<uint8_t*>(cache->vts);
     a.wait_limit_ns = wait_limit_ns();
+    a.stall_loads = g_stall_loads.load();
     return from_cuda(launch_quantize_qkv(a, reinterpret_cast<cudaStream_t>(stream)));
 }
 

@@ -32,6 +32,7 @@ struct QuantArgs {
     float* s_bias;                // [B*Hq, nkv]
     uint8_t *qc, *qs, *kc, *ks, *vtc, *vts;
     unsigned long long wait_limit_ns;   // bound of the copy waits of the row pass
+    int stall_loads;                    // test hook: the row pass issues no copies (its waits time out)
 };
 
 cudaError_t launch_quantize_qkv(const QuantArgs& a, cudaStream_t st);

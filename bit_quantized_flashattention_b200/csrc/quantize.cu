@@ -200,7 +200,7 @@ __device__ __forceinline__ uint32_t quant_block16_lut(float (&x)[16], const floa
 
 template <typename T, int D, bool ROPE, bool QM>
 __device__ __forceinline__ void quantize_rows_cta(const RowJob& jb, unsigned cta, const float* lut, uint8_t* stage,
-                                                  uint64_t* bars, unsigned long long limit_ns) {
+                                                  uint64_t* bars, unsigned long long limit_ns, bool stall) {
     constexpr unsigned CPR = D / 16;                       // lanes (scale blocks) per row
     constexpr unsigned RPB = 256 / CPR;                    // rows per CTA step
     constexpr unsigned ROW_BYTES = D * sizeof(T);
@@ -225,7 +225,7 @@ __device__ __forceinline__ void quantize_rows_cta(const RowJob& jb, unsigned cta
     uint8_t* sg = jb.sfs + (size_t)grp * jb.tiles_out * KS * 512;
     const unsigned r_in = threadIdx.x / CPR;
     const unsigned row_first = s0 * RPB;                   // first row of the range
-    if (threadIdx.x == 0) {
+    if (threadIdx.x == 0 && !stall) {
         for (unsigned k = 0; k < kRowStages; ++k) {
             const unsigned a = min(min(s0 + k, s1) * RPB, jb.rows_in);
             const unsigned b = min(min(s0 + k + 1, s1) * RPB, jb.rows_in);
@@ -243,7 +243,8 @@ __device__ __forceinline__ void quantize_rows_cta(const RowJob& jb, unsigned cta
         if (!__all_sync(0xFFFFFFFFu, mbar_wait_drain(&bars[k], 0, limit_ns))) {
             if (threadIdx.x == 0) {
                 atomicExch(&g_quantize_status, kStatusTimeout);
-                for (unsigned kk = k; kk < kRowStages; ++kk) mbar_wait_drain(&bars[kk], 0, limit_ns);
+                if (!stall)
+                    for (unsigned kk = k; kk < kRowStages; ++kk) mbar_wait_drain(&bars[kk], 0, limit_ns);
             }
             return;
         }
@@ -387,7 +388,7 @@ __device__ __forceinline__ void quantize_v_warp(const VJob& jb, unsigned gw_all,
 // K rows, the rest V (8 warps per CTA).
 template <typename T, int D, bool ROPE, bool QM>
 __global__ void __launch_bounds__(256) quantize_qkv_kernel(RowJob q, RowJob k, VJob v, unsigned nq, unsigned nk,
-                                                           unsigned v_warps, unsigned long long limit_ns) {
+                                                           unsigned v_warps, unsigned long long limit_ns, int stall) {
     __shared__ float lut[128];
     __shared__ uint64_t bars[kRowStages];
     extern __shared__ __align__(128) uint8_t stage[];      // kRowStageBytes (row CTAs)
@@ -401,9 +402,9 @@ __global__ void __launch_bounds__(256) quantize_qkv_kernel(RowJob q, RowJob k, V
     }
     build_rcp_lut(lut);                                    // ends with a CTA barrier
     if (b < nq) {
-        quantize_rows_cta<T, D, ROPE, QM>(q, b, lut, stage, bars, limit_ns);
+        quantize_rows_cta<T, D, ROPE, QM>(q, b, lut, stage, bars, limit_ns, stall != 0);
     } else if (b < nq + nk) {
-        quantize_rows_cta<T, D, ROPE, QM>(k, b - nq, lut, stage, bars, limit_ns);
+        quantize_rows_cta<T, D, ROPE, QM>(k, b - nq, lut, stage, bars, limit_ns, stall != 0);
     } else {
         const unsigned gw = (b - nq - nk) * 8 + (threadIdx.x >> 5);
         if (gw < v_warps) quantize_v_warp<T, D>(v, gw, lut);
@@ -619,7 +620,7 @@ static cudaError_t launch_qkv_t(const QuantArgs& a, cudaStream_t st) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kRowStageBytes);
     if (e != cudaSuccess) return e;
     kern<<<(unsigned)total, 256, smem, st>>>(jq, jk, jv, (unsigned)nq, (unsigned)nk, (unsigned)v_warps,
-                                              a.wait_limit_ns);
+                                              a.wait_limit_ns, a.stall_loads);
     return cudaGetLastError();
 }
 

@@ -329,10 +329,11 @@ hifa4_status hifa4_attention_fwd_noalloc(const hifa4_packed* in, int B, int Hq, 
 hifa4_status hifa4_get_status(void* workspace, hifa4_stream_t stream);
 
 /* Test hook for the timeout path: sets the wait limit (nanoseconds) that the
- * attention kernel's bounded waits use from the next launch on (0 restores the
- * default of 2 s), and, when `stall_loads` is nonzero, makes the next launches'
- * load warp issue no loads, so every consumer wait runs out with nothing in
- * flight. Returns the previous limit. */
+ * bounded waits of the attention kernel and of the quantize passes use from
+ * the next launch on (0 restores the default of 2 s), and, when `stall_loads`
+ * is nonzero, makes the next launches issue no loads (the attention kernel's
+ * load warp, the quantize pass's Q/K row copies), so every wait on them runs
+ * out with nothing in flight. Returns the previous limit. */
 long long hifa4_debug_set_wait_limit(long long limit_ns, int stall_loads);
 
 /* Description of the last CUDA error behind an HIFA4_ERR_CUDA returned to

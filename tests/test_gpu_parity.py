@@ -220,6 +220,31 @@ def test_timeout_path_reports_status(H):
     assert torch.isfinite(o).all()
 
 
+def test_quantize_timeout_path_reports_status(H):
+    """Row copies of the quantize pass stalled on purpose: its bounded waits run
+    out with nothing in flight, the pass records the timeout in its status word
+    (reported by get_status) and stops; the next pass runs normally and matches
+    the oracle."""
+    shape = (1, 2, 1, 128, 256, 128)
+    B, Hq, Hkv, Nq, Nkv, D = shape
+    rng = np.random.default_rng(18)
+    q = W.round_to_dtype(_rand(rng, (B, Hq, Nq, D)), "bf16")
+    k = W.round_to_dtype(_rand(rng, (B, Hkv, Nkv, D)), "bf16")
+    v = W.round_to_dtype(_rand(rng, (B, Hkv, Nkv, D)), "bf16")
+    dq, dk, dv = (U.to_device(x, "bf16") for x in (q, k, v))
+    ws = H.alloc_workspace(*shape)
+    assert H.get_status(ws) == 0
+    H.debug_set_wait_limit(20_000_000, stall_loads=True)       # 20 ms
+    try:
+        H.quantize_qkv(dq, dk, dv)
+        assert H.get_status(ws) == 4
+    finally:
+        H.debug_set_wait_limit(0, stall_loads=False)
+    pk = H.quantize_qkv(dq, dk, dv)
+    assert H.get_status(ws) == 0
+    _compare_packed(pk, oracle.quantize_qkv(q, k, v), shape)
+
+
 @pytest.mark.parametrize("shape,dtype,smooth", [
     ((2, 2, 384, 128), "bf16", True),
     ((1, 3, 256, 64), "fp16", False),
