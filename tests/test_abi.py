@@ -39,6 +39,55 @@ def test_library_exports_every_declared_symbol(lib):
         assert n in _lib.EXPORTS, n
 
 
+def declared_prototypes():
+    """{name: (return type, [parameter declarations])} of every function in the header."""
+    text = open(os.path.join(ROOT, "include", "hifa4.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"^\s*#.*$", "", text, flags=re.M)
+    protos = {}
+    for ret, name, params in re.findall(r"([A-Za-z_][\w ]*?\**)\s*\b(hifa4_[a-z0-9_]+)\s*\(([^;{}]*?)\)\s*;", text, flags=re.S):
+        plist = [p.strip() for p in params.split(",") if p.strip()]
+        if plist == ["void"]:
+            plist = []
+        protos[name] = (" ".join(ret.split()), plist)
+    return protos
+
+
+def _ctype_kind(t):
+    if t in (ctypes.c_void_p, ctypes.c_char_p) or (isinstance(t, type) and issubclass(t, ctypes._Pointer)):
+        return "pointer"
+    return {ctypes.c_int: "int", ctypes.c_uint: "unsigned", ctypes.c_float: "float",
+            ctypes.c_size_t: "size_t", ctypes.c_longlong: "long long"}.get(t, repr(t))
+
+
+def _c_kind(decl):
+    d = " ".join(decl.split())
+    if "*" in d or "[" in d or d.startswith("hifa4_stream_t") or d.startswith("const hifa4_stream_t"):
+        return "pointer"
+    for k in ("size_t", "long long", "unsigned", "float"):
+        if d.startswith(k) or d.startswith("const " + k):
+            return k
+    # int and the library's enums (status, dtype, norm mode) travel as int
+    return "int"
+
+
+def test_binding_signatures_match_the_header(lib):
+    """The thin ctypes binding declares, for every exported call, the same
+    number of parameters with the same kinds (pointer / int / unsigned /
+    float / size_t / long long) and the same return kind as the header."""
+    from bit_quantized_flashattention_b200 import _lib
+    protos = declared_prototypes()
+    assert set(protos) == set(declared_functions())
+    for name, (ret, params) in protos.items():
+        fn = getattr(lib, name)
+        assert fn.argtypes is not None, name
+        got = [_ctype_kind(t) for t in fn.argtypes]
+        want = [_c_kind(p) for p in params]
+        assert got == want, (name, got, want)
+        want_ret = "pointer" if ("*" in ret) else _c_kind(ret)
+        assert _ctype_kind(fn.restype) == want_ret, (name, fn.restype, ret)
+
+
 def test_size_queries(lib):
     out = (ctypes.c_size_t * 6)()
     total = lib.hifa4_packed_bytes(1, 32, 8, 4096, 4096, 128, out)
