@@ -9,7 +9,7 @@ quantized probabilities that feed PV. The computation lives in libhifa4.so
 from ._lib import HiFA4Error, load  # noqa: F401
 from .api import (PackedQKV, Rope, alloc_packed, alloc_workspace, append_kv, attention_fwd,  # noqa: F401
                   attention_fwd_debug, attention_fwd_ex, attention_fwd_q, attention_fwd_noalloc, attention_splits, calibrate_smooth,
-                  debug_set_wait_limit, get_status, packed_bytes, q_mean, quantize_kv, quantize_qkv, tile_stats,
-                  workspace_bytes)
+                  debug_set_wait_limit, get_status, packed_bytes, q_mean, quantize_kv, quantize_q, quantize_qkv,
+                  tile_stats, workspace_bytes)
 
 __version__ = "0.1.0"

@@ -17,7 +17,8 @@ EXPORTS = ["hifa4_packed_bytes", "hifa4_workspace_bytes", "hifa4_calibrate_smoot
            "hifa4_quantize_kv", "hifa4_attention_fwd", "hifa4_attention_fwd_debug", "hifa4_get_status",
            "hifa4_debug_set_wait_limit", "hifa4_status_string", "hifa4_version", "hifa4_attention_fwd_noalloc",
            "hifa4_last_cuda_error", "hifa4_attention_splits", "hifa4_quantize_qkv_ex", "hifa4_q_mean",
-           "hifa4_append_kv", "hifa4_attention_fwd_ex", "hifa4_tile_stats", "hifa4_attention_fwd_q"]
+           "hifa4_append_kv", "hifa4_attention_fwd_ex", "hifa4_tile_stats", "hifa4_attention_fwd_q",
+           "hifa4_quantize_q"]
 
 
 class Packed(ctypes.Structure):
@@ -76,6 +77,8 @@ def load():
     pre = ctypes.POINTER(Prequant)
     L.hifa4_quantize_qkv_ex.argtypes = [vp, vp, vp, ci] + [ci] * 6 + [pre, pk, vp]
     L.hifa4_quantize_qkv_ex.restype = ci
+    L.hifa4_quantize_q.argtypes = [vp, ci, ci, ci, ci, ci, ci, pre, pk, vp]
+    L.hifa4_quantize_q.restype = ci
     L.hifa4_q_mean.argtypes = [vp, ci, ci, ci, ci, ci, ci, pre, vp, vp]
     L.hifa4_q_mean.restype = ci
     L.hifa4_append_kv.argtypes = [vp, vp, ci, ci, ci, ci, ci, pre, pk, ci, ci, vp]

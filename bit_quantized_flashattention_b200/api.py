@@ -160,6 +160,22 @@ def quantize_qkv(q, k, v, s=None, s_inv=None, out: PackedQKV | None = None, stre
     return out
 
 
+def quantize_q(q, out: PackedQKV, s=None, rope: Rope | None = None, q_mean=None, stream=None) -> PackedQKV:
+    """Quantize Q alone into ``out.qc`` / ``out.qs`` (e.g. a decode step's new
+    queries into the Q buffers of a packed KV cache from quantize_kv), after
+    RoPE (rope.q_pos), Smooth-QK (s) and the Q-Mean subtraction (q_mean), in
+    that order; out's B, Hq, Hkv, Nq and D must match q."""
+    _check_input(q, "q")
+    B, Hq, Nq, D = q.shape
+    if (B, Hq, Nq, D) != (out.B, out.Hq, out.Nq, out.D):
+        raise ValueError("q does not match the packed operands' Q shape")
+    pq = _prequant(s, s, rope, q_mean)
+    st = out.struct()
+    L.check(L.load().hifa4_quantize_q(_ptr(q), _DT[q.dtype], B, Hq, out.Hkv, Nq, D, ctypes.byref(pq),
+                                      ctypes.byref(st), _stream(stream)), "quantize_q")
+    return out
+
+
 def q_mean(q, s=None, rope: Rope | None = None, out=None, Hkv: int | None = None, stream=None) -> torch.Tensor:
     """Q-Mean auxiliary: per-(b, h, channel) mean [B,Hq,D] fp32 of Q after RoPE
     and smoothing (s needs Hkv, the kv heads it is indexed by)."""

@@ -290,6 +290,48 @@ hifa4_status hifa4_quantize_qkv_ex(const void* q, const void* k, const void* v, 
     return from_cuda(launch_quantize_qkv(a, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+hifa4_status hifa4_quantize_q(const void* q, hifa4_dtype dtype, int B, int Hq, int Hkv, int Nq, int D,
+                              const hifa4_prequant* pre, const hifa4_packed* out, hifa4_stream_t stream) {
+    if (q == nullptr || out == nullptr) return HIFA4_ERR_INVALID_ARG;
+    if (dtype != HIFA4_F16 && dtype != HIFA4_BF16) return HIFA4_ERR_INVALID_ARG;
+    if (!shape_ok(B, Hq, Hkv, Nq, 128, D)) return HIFA4_ERR_UNSUPPORTED;
+    const void* ptrs[3] = {q, out->qc, out->qs};
+    for (const void* p : ptrs)
+        if (p == nullptr || !aligned16(p)) return HIFA4_ERR_INVALID_ARG;
+    hifa4_prequant x{};
+    if (pre != nullptr) x = *pre;
+    if (x.s_bias != nullptr) return HIFA4_ERR_INVALID_ARG;
+    const float* mean = x.q_mean;
+    if (!aligned16(mean)) return HIFA4_ERR_INVALID_ARG;
+    x.q_mean = nullptr;
+    x.s_inv = x.s;                                  // only s applies to Q (pairing checked on s alone)
+    const hifa4_status pc = check_prequant(x, true, false);
+    if (pc != HIFA4_OK) return pc;
+    x.s_inv = nullptr;
+    x.k_pos = nullptr;
+    if ((long long)B * Hq * Nq > INT32_MAX) return HIFA4_ERR_UNSUPPORTED;
+    const Sizes sz = sizes_of(B, Hq, Hkv, Nq, 128, D);
+    QuantArgs a{};
+    a.bf16 = dtype == HIFA4_BF16;
+    a.D = D;
+    a.G = Hq / Hkv;
+    a.hkv = Hkv;
+    a.nq = Nq;
+    a.nkv = 0;
+    a.nkv_in = 0;                                   // no K / V work
+    a.kv_start = 0;
+    a.tiles_q = sz.Tq;
+    a.n_groups = (long long)B * Hkv;
+    a.q = q;
+    set_prequant(a, x);
+    a.q_mean = mean;
+    a.qc = static_cast<uint8_t*>(out->qc);
+    a.qs = static_cast<uint8_t*>(out->qs);
+    a.wait_limit_ns = wait_limit_ns();
+    a.stall_loads = g_stall_loads.load();
+    return from_cuda(launch_quantize_qkv(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 hifa4_status hifa4_quantize_qkv(const void* q, const void* k, const void* v, hifa4_dtype dtype, int B, int Hq, int Hkv,
                                 int Nq, int Nkv, int D, const float* s, const float* s_inv, const hifa4_packed* out,
                                 hifa4_stream_t stream) {

@@ -12,7 +12,8 @@ namespace hifa4 {
 // multiply (s / s_inv non-null), the Q-Mean subtraction on Q (q_mean
 // non-null; the K pass then writes the score bias s_bias). The K and V input
 // tokens [0, nkv_in) land at tokens [kv_start, kv_start + nkv_in) of an output
-// of nkv tokens (a KV-cache append; the plain pass has nkv_in = nkv, kv_start = 0).
+// of nkv tokens (a KV-cache append; the plain pass has nkv_in = nkv, kv_start = 0;
+// nkv_in = 0 quantizes Q alone).
 struct QuantArgs {
     bool bf16;
     int D, G, hkv, nq, nkv, tiles_q;

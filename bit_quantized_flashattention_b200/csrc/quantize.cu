@@ -604,7 +604,8 @@ static cudaError_t launch_qkv_t(const QuantArgs& a, cudaStream_t st) {
     jv.nkv = a.nkv;
     jv.start = a.kv_start;
     jv.half0 = (unsigned)(a.kv_start / 64);
-    const unsigned halves = (unsigned)((a.kv_start + a.nkv_in - 1) / 64 - a.kv_start / 64 + 1);
+    const unsigned halves =
+        a.nkv_in > 0 ? (unsigned)((a.kv_start + a.nkv_in - 1) / 64 - a.kv_start / 64 + 1) : 0u;   // 0: Q only
     jv.warps_per_group = halves * (D / 32);
     const long long v_warps = n_grp * jv.warps_per_group;
     const long long v_ctas = (v_warps + 7) / 8;

@@ -197,6 +197,18 @@ hifa4_status hifa4_quantize_qkv_ex(const void* q, const void* k, const void* v, 
 hifa4_status hifa4_q_mean(const void* q, hifa4_dtype dtype, int B, int Hq, int Hkv, int Nq, int D,
                           const hifa4_prequant* pre, float* q_mean, hifa4_stream_t stream);
 
+/* Quantize Q alone, e.g. a decode step's new queries against a packed KV cache
+ * (HiFA4 abstract: Smooth-QK "after RoPE ... before quantization"). Rules,
+ * steps and layout are those of the Q part of hifa4_quantize_qkv_ex: RoPE
+ * (pre->rope_cos / rope_sin with pre->q_pos), the Smooth-QK multiply (pre->s,
+ * indexed by kv head h / (Hq / Hkv)) and the Q-Mean subtraction (pre->q_mean)
+ * may be set; pre->s_inv and pre->k_pos are ignored and pre->s_bias must be
+ * NULL (the score bias belongs to the K pass). q: [B,Hq,Nq,D] in `dtype`.
+ * Writes out->qc and out->qs (sized by hifa4_packed_bytes for these B, Hq,
+ * Hkv, Nq, D and any Nkv); the other pointers of `out` are ignored. */
+hifa4_status hifa4_quantize_q(const void* q, hifa4_dtype dtype, int B, int Hq, int Hkv, int Nq, int D,
+                              const hifa4_prequant* pre, const hifa4_packed* out, hifa4_stream_t stream);
+
 /* KV-cache append: quantize n_new new K and V tokens ([B, Hkv, n_new, D]) into
  * token slots [start, start + n_new) of a packed cache that holds
  * cache_tokens tokens (cache->kc, ks, vtc, vts sized by hifa4_packed_bytes
@@ -324,7 +336,8 @@ hifa4_status hifa4_attention_fwd_noalloc(const hifa4_packed* in, int B, int Hq, 
  * `workspace` (HIFA4_OK or HIFA4_ERR_TIMEOUT) or HIFA4_ERR_CUDA if the stream
  * reported an error. Clears the recorded status. It also reports (as
  * HIFA4_ERR_TIMEOUT) and clears the device-wide status word of the quantize
- * passes (hifa4_quantize_qkv*, hifa4_quantize_kv, hifa4_append_kv), which a
+ * passes (hifa4_quantize_qkv*, hifa4_quantize_q, hifa4_quantize_kv,
+ * hifa4_append_kv), which a
  * bounded wait for the pass's own input copies sets when it expires. */
 hifa4_status hifa4_get_status(void* workspace, hifa4_stream_t stream);
 

@@ -162,7 +162,7 @@ def test_noalloc_checks_arguments_before_any_cuda_call(lib):
 
 
 def test_extension_calls_validate_on_the_host(lib):
-    """RoPE / Q-Mean / append / extras / tile-statistics calls reject bad
+    """RoPE / Q-Mean / Q-only / append / extras / tile-statistics calls reject bad
     arguments before any CUDA call (a CUDA call would fail without a GPU)."""
     from bit_quantized_flashattention_b200 import _lib as L
     fake = ctypes.c_void_p(1 << 20)
@@ -185,6 +185,20 @@ def test_extension_calls_validate_on_the_host(lib):
     assert qx(pre(rope_cos=odd, rope_sin=fake, n_pos=8, q_pos=fake, k_pos=fake)) == L.ERR_INVALID_ARG
     assert qx(pre(q_mean=fake)) == L.ERR_INVALID_ARG                       # q_mean without s_bias
     assert qx(pre(q_mean=fake, s_bias=odd)) == L.ERR_INVALID_ARG
+
+    def qo(p=None, dtype=L.BF16, Hq=2, Hkv=1, Nq=128, D=128, q=fake, packed=pk):
+        return lib.hifa4_quantize_q(q, dtype, 1, Hq, Hkv, Nq, D, p, ctypes.byref(packed), None)
+
+    assert qo(pre(s_bias=fake)) == L.ERR_INVALID_ARG                       # the bias belongs to the K pass
+    assert qo(pre(q_mean=odd)) == L.ERR_INVALID_ARG
+    assert qo(pre(s=odd)) == L.ERR_INVALID_ARG
+    assert qo(pre(rope_cos=fake, rope_sin=fake, n_pos=8)) == L.ERR_INVALID_ARG      # no q_pos
+    assert qo(dtype=L.F32) == L.ERR_INVALID_ARG
+    assert qo(D=96) == L.ERR_UNSUPPORTED
+    assert qo(Hq=3, Hkv=2) == L.ERR_UNSUPPORTED
+    assert qo(Nq=8) == L.ERR_UNSUPPORTED
+    assert qo(q=None) == L.ERR_INVALID_ARG
+    assert qo(packed=L.Packed(fake, None, None, None, None, None)) == L.ERR_INVALID_ARG   # no qs
 
     def app(n_new=16, start=0, cap=128, p=None):
         return lib.hifa4_append_kv(fake, fake, L.BF16, 1, 1, n_new, 128, p, ctypes.byref(pk), cap, start, None)

@@ -1,5 +1,5 @@
 """GPU parity of the steps around the hot path against the CPU oracle:
-fused RoPE -> Smooth-QK -> quantize, the Q-Mean auxiliary (mean, residual
+fused RoPE -> Smooth-QK -> quantize (also of Q alone), the Q-Mean auxiliary (mean, residual
 quantization, score bias, attention with the bias), KV-cache append
 quantization, and the epsilon-bar tile statistics.
 
@@ -96,6 +96,39 @@ def test_fused_rope_quantize_matches_oracle(H, shape, dtype, smooth):
     vtc, vts = oracle.quantize_v(v)
     _, _, vts_g = U.canonical_scales(pk, B, Hq, Hkv, Nq, Nkv, D)
     assert np.array_equal(U.canonical_vtc(pk.vtc, B, Hkv, Nkv, D), vtc) and np.array_equal(vts_g, vts)
+
+
+@pytest.mark.parametrize("shape,dtype,smooth,rope,qmean", [
+    ((1, 4, 2, 48, 256, 128), "bf16", True, False, False),     # ragged G*Nq = 192 rows: padding rows
+    ((2, 8, 1, 16, 128, 64), "fp16", False, True, False),       # decode-like: 8 heads x 16 queries
+    ((1, 2, 2, 128, 256, 256), "bf16", True, True, True),
+])
+def test_quantize_q_alone_matches_oracle(H, shape, dtype, smooth, rope, qmean):
+    """hifa4_quantize_q writes Q codes and scales (padding bytes included) equal
+    to the oracle's RoPE, smoothing, Q-Mean and quantization steps, into the Q
+    buffers of a packed KV cache, and leaves the cache's K and V untouched."""
+    B, Hq, Hkv, Nq, Nkv, D = shape
+    q, k, v = _inputs(shape, dtype, seed=62, offset=1.0 if qmean else 0.0)
+    q_pos = np.arange(Nq) + (Nkv - Nq)
+    cos_t, sin_t, drope = _rope(H, D, Nkv, q_pos, None)
+    s = oracle.calibrate(q, k)[0] if smooth else None
+    ds = None if s is None else torch.from_numpy(s).cuda()
+    dq = U.to_device(q, dtype)
+    cache = H.quantize_kv(U.to_device(k, dtype), U.to_device(v, dtype), Hq=Hq, Nq=Nq)
+    torch.cuda.synchronize()
+    kv_before = {n: t.clone() for n, t in cache.tensors().items() if n not in ("qc", "qs")}
+    m = H.q_mean(dq, s=ds, rope=drope if rope else None, Hkv=Hkv) if qmean else None
+    H.quantize_q(dq, cache, s=ds, rope=drope if rope else None, q_mean=m)
+    torch.cuda.synchronize()
+    qp = oracle.prequant_rows(q, rope=(cos_t, sin_t, q_pos) if rope else None, scale=s, group=Hq // Hkv,
+                              mean=m.cpu().numpy() if qmean else None)
+    qc, qs = oracle.quantize_rows(qp)
+    qs_g, _, _ = U.canonical_scales(cache, B, Hq, Hkv, Nq, Nkv, D)
+    assert np.array_equal(cache.qc.cpu().numpy().reshape(qc.shape), qc)
+    assert np.array_equal(qs_g, qs)
+    assert U.padding_bytes_ok(cache, B, Hq, Hkv, Nq, Nkv, D)
+    for n, t in kv_before.items():
+        assert torch.equal(getattr(cache, n), t), n
 
 
 # ------------------------------------------------------------------ Q-Mean
