@@ -19,6 +19,8 @@ def test_inputs_must_be_device_tensors():
         H.quantize_qkv(x, x[:, :1], x[:, :1])
     with pytest.raises(ValueError, match="CUDA"):
         H.q_mean(x)
+    with pytest.raises(ValueError, match="CUDA"):
+        H.quantize_q(x, _packed())
 
 
 def test_rope_tables_and_positions_are_checked():
